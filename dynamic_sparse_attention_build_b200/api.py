@@ -1,0 +1,235 @@
+"""Torch-facing wrappers of the C ABI (marshalling only).
+
+Tensors are bf16 CUDA tensors shaped [heads, tokens, d] (any strides with a
+contiguous last dimension; a [tokens, heads, d] tensor viewed with
+``.transpose(0, 1)`` works too).  Device memory for indices, workspace and
+outputs is allocated here with torch; the library itself allocates nothing.
+"""
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass, field
+
+import numpy as np
+import torch
+
+from . import _binding as B
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream_ptr(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def make_problem(Q, K, V=None, O=None, block=64) -> B.dsa_problem:
+    Hq, N, d = Q.shape
+    Hkv = K.shape[0]
+    V = K if V is None else V
+    O = Q if O is None else O
+    p = B.dsa_problem()
+    p.Hq, p.Hkv, p.N, p.d, p.block = Hq, Hkv, N, d, block
+    p.q_head_stride, p.q_token_stride = Q.stride(0), Q.stride(1)
+    p.k_head_stride, p.k_token_stride = K.stride(0), K.stride(1)
+    p.v_head_stride, p.v_token_stride = V.stride(0), V.stride(1)
+    p.o_head_stride, p.o_token_stride = O.stride(0), O.stride(1)
+    return p
+
+
+def make_patterns(patterns):
+    """list of pattern dicts -> ctypes array of dsa_pattern.  A MoBA dict may hold
+    ``conv=(w, b)``: CUDA float32 tensors [d, W] and [d]."""
+    arr = (B.dsa_pattern * len(patterns))()
+    keep = []
+    for h, pd in enumerate(patterns):
+        c = arr[h]
+        c.kind = B.KIND_CODES[pd["kind"]]
+        c.sink = int(pd.get("sink", 0))
+        c.window = int(pd.get("window", 1))
+        c.last_q = int(pd.get("last_q", 0))
+        c.n_vert = int(pd.get("n_vert", 0))
+        c.n_slash = int(pd.get("n_slash", 0))
+        c.topk = int(pd.get("topk", 0))
+        c.alpha = float(pd.get("alpha", 1.0))
+        c.keep_sink = int(pd.get("keep_sink", 1))
+        c.keep_local = int(pd.get("keep_local", 1))
+        conv = pd.get("conv")
+        if conv is not None:
+            w, b = conv
+            w = w.contiguous().float()
+            b = b.contiguous().float()
+            keep += [w, b]
+            c.conv_width = int(w.shape[1])
+            c.conv_weight = w.data_ptr()
+            c.conv_bias = b.data_ptr()
+        else:
+            c.conv_width = 0
+    arr._keep = keep  # keeps conv tensors alive with the array
+    return arr
+
+
+@dataclass
+class IndexBuffers:
+    """Device index arrays (see ``dsa_indices`` in include/dsa.h) and their C view."""
+    Hq: int
+    N: int
+    block: int
+    nqb: int
+    head_info: torch.Tensor
+    blk_ptr: torch.Tensor
+    blk_idx: torch.Tensor
+    dist_ptr: torch.Tensor
+    dist: torch.Tensor
+    col_ptr: torch.Tensor
+    col_idx: torch.Tensor
+    vert_idx: torch.Tensor
+    slash_idx: torch.Tensor
+    workspace: torch.Tensor | None = None
+    c: B.dsa_indices = field(default=None)
+
+    def __post_init__(self):
+        c = B.dsa_indices()
+        c.head_info = self.head_info.data_ptr()
+        c.blk_ptr = self.blk_ptr.data_ptr()
+        c.blk_idx = self.blk_idx.data_ptr()
+        c.dist_ptr = self.dist_ptr.data_ptr()
+        c.dist = self.dist.data_ptr()
+        c.col_ptr = self.col_ptr.data_ptr()
+        c.col_idx = self.col_idx.data_ptr()
+        c.vert_idx = self.vert_idx.data_ptr()
+        c.slash_idx = self.slash_idx.data_ptr()
+        c.blk_cap = self.blk_idx.numel()
+        c.dist_cap = self.dist.numel()
+        c.col_cap = self.col_idx.numel()
+        c.vert_stride = self.vert_idx.numel() // max(1, self.Hq)
+        c.slash_stride = self.slash_idx.numel() // max(1, self.Hq)
+        self.c = c
+
+    def host_lists(self):
+        """Per-head Python view for inspection: dict of numpy arrays."""
+        hi = self.head_info.cpu().numpy().reshape(-1, 4)
+        bp = self.blk_ptr.cpu().numpy()
+        bi = self.blk_idx.cpu().numpy()
+        dp = self.dist_ptr.cpu().numpy()
+        di = self.dist.cpu().numpy()
+        cp = self.col_ptr.cpu().numpy()
+        ci = self.col_idx.cpu().numpy()
+        vs = self.vert_idx.cpu().numpy().reshape(self.Hq, -1)
+        ss = self.slash_idx.cpu().numpy().reshape(self.Hq, -1)
+        out = []
+        for h in range(self.Hq):
+            r0 = h * self.nqb
+            out.append(dict(
+                kind=int(hi[h, 0]), sink=int(hi[h, 1]), window=int(hi[h, 2]),
+                blocks=[bi[bp[r0 + q]:bp[r0 + q + 1]] for q in range(self.nqb)],
+                dist=di[dp[h]:dp[h + 1]],
+                cols=[ci[cp[r0 + q]:cp[r0 + q + 1]] for q in range(self.nqb)],
+                vert=vs[h][vs[h] >= 0], slash=ss[h][ss[h] >= 0]))
+        return out
+
+
+def alloc_indices(problem, pats_c, device="cuda") -> IndexBuffers:
+    sz = B.dsa_workspace_size(problem, pats_c)
+    i32 = dict(dtype=torch.int32, device=device)
+    bufs = IndexBuffers(
+        Hq=problem.Hq, N=problem.N, block=problem.block, nqb=sz.nqb,
+        head_info=torch.zeros(sz.head_info_len, **i32),
+        blk_ptr=torch.zeros(sz.blk_ptr_len, **i32),
+        blk_idx=torch.zeros(sz.blk_cap, **i32),
+        dist_ptr=torch.zeros(sz.dist_ptr_len, **i32),
+        dist=torch.zeros(sz.dist_cap, **i32),
+        col_ptr=torch.zeros(sz.col_ptr_len, **i32),
+        col_idx=torch.zeros(sz.col_cap, **i32),
+        vert_idx=torch.full((problem.Hq * sz.vert_stride,), -1, **i32),
+        slash_idx=torch.full((problem.Hq * sz.slash_stride,), -1, **i32),
+        workspace=torch.empty(int(sz.workspace_bytes), dtype=torch.uint8, device=device),
+    )
+    return bufs
+
+
+def build_indices(Q, K, patterns, block, bufs: IndexBuffers | None = None, stream=None) -> IndexBuffers:
+    """dsa_build_indices on torch tensors; allocates the buffers if none are given."""
+    prob = make_problem(Q, K, block=block)
+    pats_c = patterns if isinstance(patterns, ctypes.Array) else make_patterns(patterns)
+    if bufs is None:
+        bufs = alloc_indices(prob, pats_c, Q.device)
+    st = B.dsa_build_indices(prob, _ptr(Q), _ptr(K), pats_c, bufs.c, _ptr(bufs.workspace),
+                             bufs.workspace.numel(), _stream_ptr(stream))
+    B.check(st, "dsa_build_indices")
+    bufs._pats = pats_c
+    return bufs
+
+
+def sparse_prefill(Q, K, V, idx: IndexBuffers, O=None, lse=None, want_lse=False, stream=None):
+    """dsa_sparse_prefill on torch tensors; returns (O, lse or None)."""
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty(Q.shape[0], Q.shape[1], dtype=torch.float32, device=Q.device)
+    prob = make_problem(Q, K, V, O, block=idx.block)
+    st = B.dsa_sparse_prefill(prob, _ptr(Q), _ptr(K), _ptr(V), idx.c, _ptr(O), _ptr(lse), _stream_ptr(stream))
+    B.check(st, "dsa_sparse_prefill")
+    return O, lse
+
+
+def count_pairs(Q, K, idx: IndexBuffers, stream=None) -> torch.Tensor:
+    """Exact number of allowed (i, j) pairs per head (int64 tensor [Hq])."""
+    pairs = torch.empty(Q.shape[0], dtype=torch.int64, device=Q.device)
+    prob = make_problem(Q, K, block=idx.block)
+    B.check(B.dsa_count_pairs(prob, idx.c, _ptr(pairs), _stream_ptr(stream)), "dsa_count_pairs")
+    return pairs
+
+
+def device_status(stream=None):
+    """(status, detail) of the current device; synchronises the stream."""
+    return B.dsa_get_device_status(_stream_ptr(stream))
+
+
+def indices_from_lists(heads, N, block, device="cuda") -> IndexBuffers:
+    """Index buffers from host lists, one dict per head with keys ``kind`` (name),
+    ``sink``, ``window``, ``blocks`` (list per query block), ``dist`` (VS),
+    ``cols`` (list per query block).  Lets indices from any source reach
+    dsa_sparse_prefill."""
+    Hq = len(heads)
+    nqb = (N + block - 1) // block
+    info = np.zeros((Hq, 4), np.int32)
+    blk_cnt = np.zeros(Hq * nqb, np.int64)
+    col_cnt = np.zeros(Hq * nqb, np.int64)
+    dist_cnt = np.zeros(Hq, np.int64)
+    blk_all, col_all, dist_all = [], [], []
+    for h, hd in enumerate(heads):
+        info[h, 0] = B.KIND_CODES[hd["kind"]]
+        info[h, 1] = hd.get("sink", 0)
+        info[h, 2] = hd.get("window", 0)
+        if hd["kind"] == "vs":
+            d = np.asarray(hd["dist"], np.int32)
+            dist_all.append(d)
+            dist_cnt[h] = d.size
+        for q in range(nqb):
+            if hd["kind"] != "vs":
+                b = np.asarray(hd["blocks"][q], np.int32)
+                blk_all.append(b)
+                blk_cnt[h * nqb + q] = b.size
+            c = np.asarray(hd["cols"][q], np.int32)
+            col_all.append(c)
+            col_cnt[h * nqb + q] = c.size
+
+    def csr(cnt, parts):
+        ptr = np.zeros(cnt.size + 1, np.int32)
+        ptr[1:] = np.cumsum(cnt)
+        data = np.concatenate(parts).astype(np.int32) if parts else np.zeros(0, np.int32)
+        if data.size == 0:
+            data = np.zeros(1, np.int32)
+        return ptr, data
+
+    bp, bi = csr(blk_cnt, blk_all)
+    cp, ci = csr(col_cnt, col_all)
+    dp, di = csr(dist_cnt, dist_all)
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(device)
+    return IndexBuffers(Hq=Hq, N=N, block=block, nqb=nqb, head_info=t(info.ravel()), blk_ptr=t(bp),
+                        blk_idx=t(bi), dist_ptr=t(dp), dist=t(di), col_ptr=t(cp), col_idx=t(ci),
+                        vert_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device),
+                        slash_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device))

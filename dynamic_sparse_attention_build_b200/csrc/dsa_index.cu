@@ -1,0 +1,1165 @@
+// Sparse-index construction for sm_100a.
+//
+// Per head, following its pattern (MInference abstract: indices are built
+// dynamically from the assigned pattern):
+//   A-shape    -- closed-form key blocks of the sink and the local window
+//                 ("MInference 1.0" summary, "3つの疎パターン": fixed mask);
+//   VS         -- coarse attention of the last last_q queries against all keys,
+//                 vertical sums v[j] and slash sums s[o], exact top-k of each,
+//                 then block distances D and per-query-block columns
+//                 ("推論時は軽い近似で動的マスクを作る");
+//   block kinds-- mean-pooled Q and K per block, s_IJ = tau qbar_I . kbar_J over the
+//                 causal triangle, then top-k (MInference block-sparse, MoBA routing)
+//                 or the max-relative threshold of FlashPrefill section 2.2
+//                 (P_IJ >= alpha max_J P_IJ  <=>  s_IJ >= max_J s_IJ + ln alpha);
+//                 MoBA may first run a causal depthwise conv with SiLU and a
+//                 residual over the keys ("2. キーに対する畳み込み適用").
+// Every list is produced by count -> scan -> fill into caller-owned CSR arrays.
+#include <math.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+namespace {
+
+constexpr int MAXH = 256;     // heads per layer this build accepts
+constexpr int MAXKV = 256;
+constexpr int VS_CHUNK = 1024;  // keys per CTA of the VS estimate
+constexpr int VS_SUB = 128;     // keys per sub-tile
+constexpr int VS_MAXL = 128;    // last_q limit
+
+struct HeadTab {
+  int kind[MAXH];
+  int sink[MAXH];
+  int window[MAXH];
+  int last_q[MAXH];
+  int n_vert[MAXH];
+  int n_slash[MAXH];
+  int topk[MAXH];
+  float lnalpha[MAXH];
+  int keep_sink[MAXH];
+  int keep_local[MAXH];
+  int bslot[MAXH];  // slot among block-kind heads, -1 otherwise
+  int vslot[MAXH];  // slot among VS heads, -1 otherwise
+  int bhead[MAXH];  // q-head of block slot s
+  int vhead[MAXH];  // q-head of VS slot s
+};
+
+struct ConvTab {
+  const float* w[MAXKV];
+  const float* b[MAXKV];
+  int width[MAXKV];
+  int need[MAXKV];  // K of this KV head is pooled
+};
+
+struct Layout {
+  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_nchunks, vs_lmax;
+  int64_t off_qbar, off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, total;
+};
+
+__host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// order-preserving float -> uint32 key
+__device__ __forceinline__ uint32_t fkey(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// ---------------------------------------------------------------------------
+// CTA-wide helpers (blockDim.x threads, multiple of 32, <= 1024)
+// ---------------------------------------------------------------------------
+__device__ int block_sum_int(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_sum_int(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int t = 0;
+  for (int i = 0; i < nw; ++i) t += red[i];
+  __syncthreads();
+  return t;
+}
+
+__device__ float block_max_f(float v, float* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  v = warp_max(v);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  float t = -INFINITY;
+  for (int i = 0; i < nw; ++i) t = fmaxf(t, red[i]);
+  __syncthreads();
+  return t;
+}
+
+// Exact top-k of vals[0..n) (ties to the lower index), n > k >= 1.  Finds the
+// k-th largest key T by 4 radix passes of 8 bits, and how many keys equal to T
+// to take.  hist: shared int[256 * nwarps]; red: shared int[64].
+template <typename Loader>
+__device__ void radix_kth(const Loader& load, int n, int k, int* hist, int* red, uint32_t* T_out,
+                          int* take_eq_out) {
+  const int nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5;
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = threadIdx.x; i < 256 * nw; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+      const uint32_t key = fkey(load(i));
+      if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1);
+    }
+    __syncthreads();
+    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+      int s = 0;
+      for (int w = 0; w < nw; ++w) s += hist[w * 256 + b];
+      hist[b] = s;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      int above = 0;
+      int digit = 0;
+      for (int b = 255; b >= 0; --b) {
+        if (above + hist[b] >= need) { digit = b; break; }
+        above += hist[b];
+      }
+      red[0] = digit;
+      red[1] = above;
+    }
+    __syncthreads();
+    prefix |= (uint32_t)red[0] << shift;
+    mask |= 255u << shift;
+    need -= red[1];
+    __syncthreads();
+  }
+  *T_out = prefix;
+  *take_eq_out = need;
+}
+
+// Ordered selection: calls emit(i, rank) for every selected i in ascending i,
+// where selected = key > T, or key == T among the first take_eq such keys.
+// One warp per contiguous segment; coalesced reads; red: shared int[>= 2*nw+2].
+template <typename Loader, typename Emit>
+__device__ void ordered_select(const Loader& load, int n, uint32_t T, int take_eq, int* red, const Emit& emit) {
+  const int nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = ceil_div(ceil_div(n, nw), 32) * 32;
+  const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  int gt = 0, eq = 0;
+  for (int i = beg + lane; i < end; i += 32) {
+    const uint32_t key = fkey(load(i));
+    gt += key > T;
+    eq += key == T;
+  }
+  gt = warp_sum_int(gt);
+  eq = warp_sum_int(eq);
+  if (lane == 0) {
+    red[2 * warp] = gt;
+    red[2 * warp + 1] = eq;
+  }
+  __syncthreads();
+  int out_base = 0, eq_base = 0;
+  for (int w = 0; w < warp; ++w) {
+    eq_base += red[2 * w + 1];
+  }
+  // output position: selected-before = gt of earlier warps + min(eq earlier, take_eq)
+  for (int w = 0; w < warp; ++w) out_base += red[2 * w];
+  out_base += min(eq_base, take_eq);
+  __syncthreads();
+  int eq_run = eq_base;
+  int pos = out_base;
+  for (int i0 = beg; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    bool sel = false, iseq = false;
+    if (i < end) {
+      const uint32_t key = fkey(load(i));
+      iseq = key == T;
+      sel = key > T;
+    }
+    const unsigned eqm = __ballot_sync(0xffffffffu, iseq);
+    const int eq_before = eq_run + __popc(eqm & ((1u << lane) - 1u));
+    if (iseq && eq_before < take_eq) sel = true;
+    eq_run += __popc(eqm);
+    const unsigned sm = __ballot_sync(0xffffffffu, sel);
+    if (sel) emit(i, pos + __popc(sm & ((1u << lane) - 1u)));
+    pos += __popc(sm);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// head info + A-shape / block counts
+// ---------------------------------------------------------------------------
+__global__ void k_head_info(const __grid_constant__ HeadTab ht, int Hq, int32_t* head_info) {
+  const int h = blockIdx.x * blockDim.x + threadIdx.x;
+  if (h >= Hq) return;
+  head_info[h * 4 + 0] = ht.kind[h];
+  head_info[h * 4 + 1] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.sink[h] : 0;
+  head_info[h * 4 + 2] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.window[h] : 0;
+  head_info[h * 4 + 3] = 0;
+}
+
+__device__ __forceinline__ void ashape_range(int qb, int B, int N, int sink, int window, int* a, int* w) {
+  const int r0 = qb * B;
+  const int r1 = min(N - 1, r0 + B - 1);
+  *a = ceil_div(min(sink, r1 + 1), B);          // sink blocks [0, a)
+  *w = max(0, r0 - window + 1) / B;             // window blocks [w, qb]
+}
+
+__global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int32_t* blk_ptr) {
+  const int h = blockIdx.y;
+  if (ht.kind[h] != DSA_KIND_ASHAPE) return;
+  const int qb = blockIdx.x * blockDim.x + threadIdx.x;
+  if (qb >= L.nqb) return;
+  int a, w;
+  ashape_range(qb, L.B, L.N, ht.sink[h], ht.window[h], &a, &w);
+  const int cnt = a + (qb + 1 - max(w, a) > 0 ? qb + 1 - max(w, a) : 0);
+  blk_ptr[1 + h * L.nqb + qb] = cnt;
+}
+
+// ---------------------------------------------------------------------------
+// mean pooling (+ optional causal depthwise key conv with SiLU and residual)
+// ---------------------------------------------------------------------------
+// grid: (nqb, nbh + Hkv); item < nbh pools Q of block slot `item`, else K of KV
+// head item - nbh (skipped unless some block head reads it).
+template <int D>
+__global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht, const __grid_constant__ ConvTab ct,
+                                              Layout L, const __nv_bfloat16* Q, int64_t q_hs, int64_t q_ts,
+                                              const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws) {
+  constexpr int TPR = D / 8;          // threads per row, 8 channels each
+  constexpr int RG = 256 / TPR;       // rows in flight
+  __shared__ float part[RG][D];
+  const int b = blockIdx.x;
+  const int item = blockIdx.y;
+  const bool isq = item < L.nbh;
+  const int kvh = isq ? 0 : item - L.nbh;
+  if (!isq && !ct.need[kvh]) return;
+  const __nv_bfloat16* X;
+  int64_t ts;
+  float* out;
+  int W = 0;
+  const float* cw = nullptr;
+  const float* cb = nullptr;
+  if (isq) {
+    const int h = ht.bhead[item];
+    X = Q + h * q_hs;
+    ts = q_ts;
+    out = reinterpret_cast<float*>(ws + L.off_qbar) + ((int64_t)item * L.nqb + b) * D;
+  } else {
+    X = K + kvh * k_hs;
+    ts = k_ts;
+    out = reinterpret_cast<float*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * D;
+    W = ct.width[kvh];
+    cw = ct.w[kvh];
+    cb = ct.b[kvh];
+  }
+  const int rg = threadIdx.x / TPR;
+  const int c0 = (threadIdx.x % TPR) * 8;
+  const int r_beg = b * L.B;
+  const int r_end = min(L.N, r_beg + L.B);
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int r = r_beg + rg; r < r_end; r += RG) {
+    const uint4 raw = *reinterpret_cast<const uint4*>(X + (int64_t)r * ts + c0);
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    float x[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(e[i]);
+    if (W > 0) {
+      float conv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) conv[i] = cb[c0 + i];
+      for (int t = 0; t < W; ++t) {
+        if (r - t < 0) break;
+        const uint4 rr = (t == 0) ? raw : *reinterpret_cast<const uint4*>(X + (int64_t)(r - t) * ts + c0);
+        const __nv_bfloat16* ee = reinterpret_cast<const __nv_bfloat16*>(&rr);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) conv[i] = fmaf(cw[(c0 + i) * W + t], __bfloat162float(ee[i]), conv[i]);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] += conv[i] / (1.f + expf(-conv[i]));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += x[i];
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) part[rg][c0 + i] = acc[i];
+  __syncthreads();
+  if (threadIdx.x < D) {
+    float s = 0.f;
+    for (int g = 0; g < RG; ++g) s += part[g][threadIdx.x];
+    out[threadIdx.x] = s / (float)(r_end - r_beg);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// block scores + selection: one CTA (256 threads) per (block slot, query block I)
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+                                                      int32_t* blk_ptr) {
+  extern __shared__ float sc[];  // [nkb] scores
+  __shared__ float qv[D];
+  __shared__ int hist[256 * 8];
+  __shared__ int red[64];
+  __shared__ float redf[32];
+  const int I = blockIdx.x;
+  const int slot = blockIdx.y;
+  const int h = ht.bhead[slot];
+  const int kind = ht.kind[h];
+  const int kvh = h / L.G;
+  const float tau = rsqrtf((float)D);
+  const float* qbar = reinterpret_cast<const float*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I) * D;
+  const float* kbar = reinterpret_cast<const float*>(ws + L.off_kbar) + (int64_t)kvh * L.nqb * D;
+  uint32_t* sel = reinterpret_cast<uint32_t*>(ws + L.off_sel) + ((int64_t)slot * L.nqb + I) * L.nkw;
+  for (int c = threadIdx.x; c < D; c += blockDim.x) qv[c] = qbar[c];
+  for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) sel[w] = 0u;
+  __syncthreads();
+  // candidates: J <= I (MoBA: J < I)
+  const int ncand = (kind == DSA_KIND_MOBA) ? I : I + 1;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int J = warp; J < ncand; J += 8) {
+    const float* kr = kbar + (int64_t)J * D;
+    float s = 0.f;
+    for (int c = lane; c < D; c += 32) s = fmaf(qv[c], kr[c], s);
+    s = warp_sum(s);
+    if (lane == 0) sc[J] = s * tau;
+  }
+  __syncthreads();
+  int count = 0;
+  if (kind == DSA_KIND_BLOCK_THRESHOLD) {
+    float mx = -INFINITY;
+    for (int J = threadIdx.x; J < ncand; J += blockDim.x) mx = fmaxf(mx, sc[J]);
+    mx = block_max_f(mx, redf);
+    const float thr = mx + ht.lnalpha[h];
+    for (int J = threadIdx.x; J < ncand; J += blockDim.x)
+      if (sc[J] >= thr) atomicOr(&sel[J >> 5], 1u << (J & 31));
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      if (ht.keep_sink[h]) atomicOr(&sel[0], 1u);
+      if (ht.keep_local[h]) atomicOr(&sel[I >> 5], 1u << (I & 31));
+    }
+    __syncthreads();
+    int c = 0;
+    for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) c += __popc(sel[w]);
+    count = block_sum_int(c, red);
+  } else {
+    const int k = ht.topk[h];
+    if (ncand <= k) {
+      for (int J = threadIdx.x; J < ncand; J += blockDim.x) atomicOr(&sel[J >> 5], 1u << (J & 31));
+      count = ncand;
+    } else if (k > 0) {
+      uint32_t T;
+      int take_eq;
+      auto load = [&](int i) { return sc[i]; };
+      radix_kth(load, ncand, k, hist, red, &T, &take_eq);
+      ordered_select(load, ncand, T, take_eq, red, [&](int i, int) { atomicOr(&sel[i >> 5], 1u << (i & 31)); });
+      count = k;
+    }
+    __syncthreads();
+    if (kind == DSA_KIND_MOBA) {
+      if (threadIdx.x == 0) atomicOr(&sel[I >> 5], 1u << (I & 31));
+      count += 1;
+    }
+  }
+  if (threadIdx.x == 0) blk_ptr[1 + h * L.nqb + I] = count;
+}
+
+// ---------------------------------------------------------------------------
+// VS estimate: logits of the last Lq rows against one chunk of keys, bf16
+// mma.sync m16n8k16 with fp32 accumulate.
+//   PASS 1: per-row max and sum of exp over the chunk -> partials
+//   PASS 2: p = exp(l - m_i) / l_i; v[j] (column sums, owned by this CTA) and
+//           s[o] (diagonal sums, global atomics at the chunk edges)
+// Rows padded to LP = 16 * RT; warps: RT row tiles x (8 / RT) key groups.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <int D, int RT, int PASS>
+__global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, Layout L, const __nv_bfloat16* Q,
+                                            int64_t q_hs, int64_t q_ts, const __nv_bfloat16* K, int64_t k_hs,
+                                            int64_t k_ts, uint8_t* ws) {
+  constexpr int LP = 16 * RT;
+  constexpr int WPR = 8 / RT;            // warps per row tile
+  constexpr int KPW = VS_SUB / WPR;      // keys per warp per sub-tile
+  constexpr int NT = KPW / 8;            // n-tiles per warp
+  constexpr int DP = D + 8;              // padded smem row (bf16)
+  constexpr int PP = VS_SUB + 4;         // padded fp32 row of the P tile
+  extern __shared__ uint8_t smraw[];
+  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smraw);          // [LP][DP]
+  __nv_bfloat16* ks = qs + LP * DP;                                      // [VS_SUB][DP]
+  float* ps = reinterpret_cast<float*>(ks + VS_SUB * DP);                // [LP][PP] (pass 2)
+  float* sbuf = ps + LP * PP;                                            // [VS_CHUNK + LP]
+  float* vbuf = sbuf + VS_CHUNK + LP;                                    // [VS_CHUNK]
+  float* rowm = vbuf + VS_CHUNK;                                         // [LP]
+  float* rowl = rowm + LP;                                               // [LP]
+  float* wpart = rowl + LP;                                              // [8][LP][2] (pass 1)
+
+  // chunk-major order: q-heads of one KV group read the same K chunk back to back
+  const int vslot = blockIdx.x % L.nvs;
+  const int chunk = blockIdx.x / L.nvs;
+  const int h = ht.vhead[vslot];
+  const int kvh = h / L.G;
+  const int Lq = min(ht.last_q[h], L.N);
+  const int i0 = L.N - Lq;  // first estimate row
+  const int j0 = chunk * VS_CHUNK;
+  const int j1 = min(L.N, j0 + VS_CHUNK);
+  const float tau = rsqrtf((float)D);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int rt = warp % RT, kg = warp / RT;
+
+  // Q rows (padding rows are zero)
+  for (int idx = tid; idx < LP * (D / 8); idx += 256) {
+    const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (r < Lq) v = *reinterpret_cast<const uint4*>(Q + h * q_hs + (int64_t)(i0 + r) * q_ts + c);
+    *reinterpret_cast<uint4*>(qs + r * DP + c) = v;
+  }
+  float* part = reinterpret_cast<float*>(ws + L.off_part);
+  float* stat = reinterpret_cast<float*>(ws + L.off_stat);
+  if (PASS == 2) {
+    for (int i = tid; i < VS_CHUNK + LP; i += 256) sbuf[i] = 0.f;
+    for (int i = tid; i < VS_CHUNK; i += 256) vbuf[i] = 0.f;
+    for (int r = tid; r < LP; r += 256) {
+      rowm[r] = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 0] : 0.f;
+      const float l = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 1] : 1.f;
+      rowl[r] = 1.f / l;
+    }
+  }
+  __syncthreads();
+  // A fragments of this warp's row tile, kept in registers
+  uint32_t af[D / 16][4];
+  {
+    const int g = lane >> 2, q = (lane & 3) * 2;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const __nv_bfloat16* base = qs + (rt * 16) * DP + kk * 16;
+      af[kk][0] = *reinterpret_cast<const uint32_t*>(base + g * DP + q);
+      af[kk][1] = *reinterpret_cast<const uint32_t*>(base + (g + 8) * DP + q);
+      af[kk][2] = *reinterpret_cast<const uint32_t*>(base + g * DP + q + 8);
+      af[kk][3] = *reinterpret_cast<const uint32_t*>(base + (g + 8) * DP + q + 8);
+    }
+  }
+  float run_m[2] = {-INFINITY, -INFINITY}, run_l[2] = {0.f, 0.f};
+  const int rA = rt * 16 + (lane >> 2);  // this thread's two rows: rA, rA + 8
+  for (int sub = j0; sub < j1; sub += VS_SUB) {
+    __syncthreads();
+    for (int idx = tid; idx < VS_SUB * (D / 8); idx += 256) {
+      const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (sub + r < j1) v = *reinterpret_cast<const uint4*>(K + kvh * k_hs + (int64_t)(sub + r) * k_ts + c);
+      *reinterpret_cast<uint4*>(ks + r * DP + c) = v;
+    }
+    __syncthreads();
+    float acc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int key = kg * KPW + n * 8 + (lane >> 2);
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const __nv_bfloat16* kb = ks + key * DP + kk * 16 + (lane & 3) * 2;
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
+        mma_bf16_16816(acc[n], af[kk], b0, b1);
+      }
+    }
+    // logits -> natural units, masked (row < Lq, key <= row, key < N)
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = rA + ((e >> 1) << 3);
+        const int j = sub + kg * KPW + n * 8 + (lane & 3) * 2 + (e & 1);
+        const bool ok = (r < Lq) && (j < j1) && (j <= i0 + r);
+        acc[n][e] = ok ? acc[n][e] * tau : -INFINITY;
+      }
+    }
+    if (PASS == 1) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        float mx = -INFINITY;
+#pragma unroll
+        for (int n = 0; n < NT; ++n) mx = fmaxf(mx, fmaxf(acc[n][2 * hr], acc[n][2 * hr + 1]));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float mnew = fmaxf(run_m[hr], mx);
+        const bool live = mnew != -INFINITY;
+        float s = 0.f;
+        if (live) {
+#pragma unroll
+          for (int n = 0; n < NT; ++n) s += expf(acc[n][2 * hr] - mnew) + expf(acc[n][2 * hr + 1] - mnew);
+        }
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (live) {
+          run_l[hr] = run_l[hr] * expf(run_m[hr] - mnew) + s;
+          run_m[hr] = mnew;
+        }
+      }
+    } else {
+      // p into the fp32 tile, then column and diagonal sums
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int r = rA + ((e >> 1) << 3);
+          const int c = kg * KPW + n * 8 + (lane & 3) * 2 + (e & 1);
+          ps[r * PP + c] = (acc[n][e] == -INFINITY) ? 0.f : expf(acc[n][e] - rowm[r]) * rowl[r];
+        }
+      }
+      __syncthreads();
+      if (tid < VS_SUB) {
+        float cs = 0.f;
+        for (int r = 0; r < LP; ++r) cs += ps[r * PP + tid];
+        vbuf[sub - j0 + tid] += cs;
+      }
+      // offsets of this sub-tile: o = (i0 + r) - (sub + c); index into sbuf by
+      // t = o - (i0 - (j0 + VS_CHUNK - 1)), c = (i0 + r) - o - sub
+      const int obase = i0 - (j0 + VS_CHUNK - 1);
+      for (int o = i0 - (sub + VS_SUB - 1) + tid; o <= i0 + LP - 1 - sub; o += 256) {
+        float acc_s = 0.f;
+        for (int r = 0; r < LP; ++r) {
+          const int c = i0 + r - o - sub;
+          if (c >= 0 && c < VS_SUB) acc_s += ps[r * PP + c];
+        }
+        sbuf[o - obase] += acc_s;
+      }
+    }
+  }
+  if (PASS == 1) {
+    // combine the key-group warps of each row tile
+    if ((lane & 3) == 0) {
+#pragma unroll
+      for (int hr = 0; hr < 2; ++hr) {
+        wpart[(kg * LP + rA + 8 * hr) * 2 + 0] = run_m[hr];
+        wpart[(kg * LP + rA + 8 * hr) * 2 + 1] = run_l[hr];
+      }
+    }
+    __syncthreads();
+    for (int r = tid; r < Lq; r += 256) {
+      float m = -INFINITY;
+      for (int g = 0; g < WPR; ++g) m = fmaxf(m, wpart[(g * LP + r) * 2]);
+      float l = 0.f;
+      if (m != -INFINITY)
+        for (int g = 0; g < WPR; ++g) {
+          const float gm = wpart[(g * LP + r) * 2];
+          if (gm != -INFINITY) l += wpart[(g * LP + r) * 2 + 1] * expf(gm - m);
+        }
+      float* pp = part + (((int64_t)vslot * L.vs_nchunks + chunk) * VS_MAXL + r) * 2;
+      pp[0] = m;
+      pp[1] = l;
+    }
+  } else {
+    __syncthreads();
+    float* vout = reinterpret_cast<float*>(ws + L.off_v) + (int64_t)vslot * L.N;
+    float* sout = reinterpret_cast<float*>(ws + L.off_s) + (int64_t)vslot * L.N;
+    for (int j = j0 + tid; j < j1; j += 256) vout[j] = vbuf[j - j0];
+    const int obase = i0 - (j0 + VS_CHUNK - 1);
+    for (int t = tid; t < VS_CHUNK + LP; t += 256) {
+      const int o = obase + t;
+      const float val = sbuf[t];
+      if (o >= 0 && o < L.N && val != 0.f) atomicAdd(&sout[o], val);
+    }
+  }
+}
+
+// merge the per-chunk (max, sum) partials into the row softmax statistics
+__global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws) {
+  const int vslot = blockIdx.x;
+  const int h = ht.vhead[vslot];
+  const int Lq = min(ht.last_q[h], L.N);
+  const float* part = reinterpret_cast<const float*>(ws + L.off_part);
+  float* stat = reinterpret_cast<float*>(ws + L.off_stat);
+  for (int r = threadIdx.x; r < Lq; r += blockDim.x) {
+    float m = -INFINITY;
+    for (int c = 0; c < L.vs_nchunks; ++c)
+      m = fmaxf(m, part[(((int64_t)vslot * L.vs_nchunks + c) * VS_MAXL + r) * 2]);
+    float l = 0.f;
+    for (int c = 0; c < L.vs_nchunks; ++c) {
+      const float* pp = part + (((int64_t)vslot * L.vs_nchunks + c) * VS_MAXL + r) * 2;
+      if (pp[0] != -INFINITY) l += pp[1] * expf(pp[0] - m);
+    }
+    stat[((int64_t)vslot * VS_MAXL + r) * 2 + 0] = m;
+    stat[((int64_t)vslot * VS_MAXL + r) * 2 + 1] = l;
+  }
+}
+
+// exact top-k of v (blockIdx.y == 0) or s (== 1) of one VS head, ascending, -1 padded
+__global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+                                                  int32_t* vert_idx, int vert_stride, int32_t* slash_idx,
+                                                  int slash_stride) {
+  __shared__ int hist[256 * 32];
+  __shared__ int red[80];
+  const int vslot = blockIdx.x;
+  const int which = blockIdx.y;
+  const int h = ht.vhead[vslot];
+  const float* arr = reinterpret_cast<const float*>(ws + (which == 0 ? L.off_v : L.off_s)) + (int64_t)vslot * L.N;
+  const int k = min(which == 0 ? ht.n_vert[h] : ht.n_slash[h], L.N);
+  int32_t* out = which == 0 ? vert_idx + (int64_t)h * vert_stride : slash_idx + (int64_t)h * slash_stride;
+  const int stride = which == 0 ? vert_stride : slash_stride;
+  for (int i = k + threadIdx.x; i < stride; i += blockDim.x) out[i] = -1;
+  if (k <= 0) return;
+  auto load = [&](int i) { return arr[i]; };
+  if (k >= L.N) {
+    for (int i = threadIdx.x; i < L.N; i += blockDim.x) out[i] = i;
+    return;
+  }
+  uint32_t T;
+  int take_eq;
+  radix_kth(load, L.N, k, hist, red, &T, &take_eq);
+  ordered_select(load, L.N, T, take_eq, red, [&](int i, int pos) { out[pos] = i; });
+}
+
+// block distances D of one VS head: {floor(o/B), ceil(o/B)} for the chosen slashes
+__global__ void k_vs_dist(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws, const int32_t* slash_idx,
+                          int slash_stride, int32_t* dist_ptr) {
+  const int vslot = blockIdx.x;
+  const int h = ht.vhead[vslot];
+  uint32_t* dbits = reinterpret_cast<uint32_t*>(ws + L.off_dbits) + (int64_t)vslot * L.nkw;
+  int32_t* dtmp = reinterpret_cast<int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.nqb;
+  for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) dbits[w] = 0u;
+  __syncthreads();
+  const int ns = min(ht.n_slash[h], L.N);
+  for (int t = threadIdx.x; t < ns; t += blockDim.x) {
+    const int o = slash_idx[(int64_t)h * slash_stride + t];
+    if (o < 0) continue;
+    const int lo = o / L.B, hi = (o + L.B - 1) / L.B;
+    if (lo < L.nqb) atomicOr(&dbits[lo >> 5], 1u << (lo & 31));
+    if (hi < L.nqb) atomicOr(&dbits[hi >> 5], 1u << (hi & 31));
+  }
+  __threadfence_block();
+  __syncthreads();
+  // ascending compaction by one warp (word order), counts via popc
+  if (threadIdx.x < 32) {
+    int base = 0;
+    for (int w0 = 0; w0 < L.nkw; w0 += 32) {
+      const int w = w0 + threadIdx.x;
+      const uint32_t bits = (w < L.nkw) ? dbits[w] : 0u;
+      const int c = __popc(bits);
+      int incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if ((int)threadIdx.x >= o) incl += y;
+      }
+      int pos = base + incl - c;
+      uint32_t b = bits;
+      while (b) {
+        const int bit = __ffs(b) - 1;
+        b &= b - 1u;
+        dtmp[pos++] = w * 32 + bit;
+      }
+      base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (threadIdx.x == 0) dist_ptr[1 + h] = base;
+  }
+}
+
+// columns of (VS head, query block): j in V, j <= qb*B+B-1, (qb - j/B) not in D.
+// One warp per query block.  FILL=false writes counts, FILL=true writes lists.
+template <bool FILL>
+__global__ void k_vs_cols(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws, const int32_t* vert_idx,
+                          int vert_stride, int32_t* col_ptr, int32_t* col_idx, int64_t col_cap, unsigned* status) {
+  const int vslot = blockIdx.y;
+  const int h = ht.vhead[vslot];
+  const int qb = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (qb >= L.nqb) return;
+  const uint32_t* dbits = reinterpret_cast<const uint32_t*>(ws + L.off_dbits) + (int64_t)vslot * L.nkw;
+  const int32_t* V = vert_idx + (int64_t)h * vert_stride;
+  const int nv = min(ht.n_vert[h], L.N);
+  const int lim = qb * L.B + L.B - 1;
+  const int row = h * L.nqb + qb;
+  int pos = FILL ? col_ptr[row] : 0;
+  const int end = FILL ? col_ptr[row + 1] : 0;
+  if (FILL && end > col_cap) {
+    if (lane == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_COL);
+    return;
+  }
+  for (int t0 = 0; t0 < nv; t0 += 32) {
+    const int t = t0 + lane;
+    const int j = (t < nv) ? V[t] : -1;
+    bool take = false;
+    if (j >= 0 && j <= lim) {
+      const int delta = qb - j / L.B;
+      take = !((dbits[delta >> 5] >> (delta & 31)) & 1u);
+    }
+    const unsigned m = __ballot_sync(0xffffffffu, take);
+    if (FILL && take) col_idx[pos + __popc(m & ((1u << lane) - 1u))] = j;
+    pos += __popc(m);
+    if (__shfl_sync(0xffffffffu, j, 31) > lim) break;  // V is ascending
+  }
+  if (!FILL && lane == 0) col_ptr[1 + row] = pos;
+}
+
+// in-place inclusive scan of ptr[0..n) (ptr[0] == 0, ptr[r+1] == count of row r)
+__global__ void __launch_bounds__(1024) k_scan(int32_t* p0, int n0, int64_t cap0, int32_t* p1, int n1, int64_t cap1,
+                                               int32_t* p2, int n2, int64_t cap2, unsigned* status) {
+  __shared__ int wsum[32];
+  int32_t* p = blockIdx.x == 0 ? p0 : (blockIdx.x == 1 ? p1 : p2);
+  const int n = blockIdx.x == 0 ? n0 : (blockIdx.x == 1 ? n1 : n2);
+  const int64_t cap = blockIdx.x == 0 ? cap0 : (blockIdx.x == 1 ? cap1 : cap2);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int seg = ceil_div(ceil_div(n, 32), 32) * 32;
+  const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  int s = 0;
+  for (int i = beg + lane; i < end; i += 32) s += p[i];
+  s = warp_sum_int(s);
+  if (lane == 0) wsum[warp] = s;
+  __syncthreads();
+  int carry = 0;
+  for (int w = 0; w < warp; ++w) carry += wsum[w];
+  for (int i0 = beg; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    int v = (i < end) ? p[i] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, v, o);
+      if (lane >= o) v += y;
+    }
+    if (i < end) p[i] = v + carry;
+    carry += __shfl_sync(0xffffffffu, v, 31);
+  }
+  __syncthreads();
+  if (threadIdx.x == 0 && n > 0 && (int64_t)p[n - 1] > cap) {
+    const unsigned det = blockIdx.x == 0 ? DETAIL_CAP_BLK : (blockIdx.x == 1 ? DETAIL_CAP_COL : DETAIL_CAP_DIST);
+    report(status, DSA_ERR_CAPACITY, det);
+  }
+}
+
+// fill block lists: A-shape closed form, block kinds from the selection bitmap
+__global__ void k_blk_fill(const __grid_constant__ HeadTab ht, Layout L, const uint8_t* ws, const int32_t* blk_ptr,
+                           int32_t* blk_idx, int64_t blk_cap, unsigned* status) {
+  const int h = blockIdx.y;
+  const int kind = ht.kind[h];
+  if (kind == DSA_KIND_VS) return;
+  const int qb = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (qb >= L.nqb) return;
+  const int row = h * L.nqb + qb;
+  const int beg = blk_ptr[row], end = blk_ptr[row + 1];
+  if (end > blk_cap) {
+    if (lane == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_BLK);
+    return;
+  }
+  if (kind == DSA_KIND_ASHAPE) {
+    int a, w;
+    ashape_range(qb, L.B, L.N, ht.sink[h], ht.window[h], &a, &w);
+    const int w2 = max(w, a);
+    const int n = a + max(0, qb + 1 - w2);
+    for (int t = lane; t < n && beg + t < end; t += 32) blk_idx[beg + t] = (t < a) ? t : (w2 + t - a);
+    return;
+  }
+  const uint32_t* sel = reinterpret_cast<const uint32_t*>(ws + L.off_sel) + ((int64_t)ht.bslot[h] * L.nqb + qb) * L.nkw;
+  int pos = beg;
+  for (int w0 = 0; w0 < L.nkw; w0 += 32) {
+    const int w = w0 + lane;
+    const uint32_t bits = (w < L.nkw) ? sel[w] : 0u;
+    const int c = __popc(bits);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int p = pos + incl - c;
+    uint32_t b = bits;
+    while (b) {
+      const int bit = __ffs(b) - 1;
+      b &= b - 1u;
+      if (p < end) blk_idx[p] = w * 32 + bit;
+      ++p;
+    }
+    pos += __shfl_sync(0xffffffffu, incl, 31);
+  }
+}
+
+__global__ void k_dist_fill(const __grid_constant__ HeadTab ht, Layout L, const uint8_t* ws, const int32_t* dist_ptr,
+                            int32_t* dist, int64_t dist_cap, unsigned* status) {
+  const int vslot = blockIdx.x;
+  const int h = ht.vhead[vslot];
+  const int beg = dist_ptr[h], end = dist_ptr[h + 1];
+  if (end > dist_cap) {
+    if (threadIdx.x == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_DIST);
+    return;
+  }
+  const int32_t* dtmp = reinterpret_cast<const int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.nqb;
+  for (int t = threadIdx.x; t < end - beg; t += blockDim.x) dist[beg + t] = dtmp[t];
+}
+
+// ---------------------------------------------------------------------------
+// exact |M| per head (selected pairs), from the lists
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ bool sorted_contains(const int32_t* a, int n, int x) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (a[mid] < x) lo = mid + 1; else hi = mid;
+  }
+  return lo < n && a[lo] == x;
+}
+
+__device__ __forceinline__ int64_t ashape_pairs_in_block(int kb, int B, int r0, int r1, int sink, int window) {
+  // sum over rows i in [r0, r1] of |{j in block kb : j <= i, (j < sink or i - j < window)}|
+  int64_t tot = 0;
+  const int k0 = kb * B, k1 = kb * B + B - 1;
+  for (int i = r0; i <= r1; ++i) {
+    const int hi = min(k1, i);
+    if (hi < k0) continue;
+    // union of [k0, min(hi, sink-1)] and [max(k0, i-window+1), hi]
+    const int a_hi = min(hi, sink - 1);
+    const int na = a_hi >= k0 ? a_hi - k0 + 1 : 0;
+    const int b_lo = max(k0, i - window + 1);
+    const int nb = hi >= b_lo ? hi - b_lo + 1 : 0;
+    int overlap = 0;
+    if (na > 0 && nb > 0) {
+      const int olo = max(k0, b_lo), ohi = min(a_hi, hi);
+      overlap = ohi >= olo ? ohi - olo + 1 : 0;
+    }
+    tot += na + nb - overlap;
+  }
+  return tot;
+}
+
+__global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head_info, const int32_t* blk_ptr,
+                              const int32_t* blk_idx, const int32_t* dist_ptr, const int32_t* dist,
+                              const int32_t* col_ptr, const int32_t* col_idx, unsigned long long* pairs) {
+  const int qb = blockIdx.x;
+  const int h = blockIdx.y;
+  const int kind = head_info[h * 4];
+  const int sink = head_info[h * 4 + 1], window = head_info[h * 4 + 2];
+  const int r0 = qb * B, r1 = min(N - 1, r0 + B - 1);
+  const int nrows = r1 - r0 + 1;
+  int64_t tot = 0;
+  const int32_t* lst;
+  int nl;
+  int dsel = 0;
+  if (kind == DSA_KIND_VS) {
+    lst = dist + dist_ptr[h];
+    nl = dist_ptr[h + 1] - dist_ptr[h];
+    dsel = 1;
+  } else {
+    lst = blk_idx + blk_ptr[h * nqb + qb];
+    nl = blk_ptr[h * nqb + qb + 1] - blk_ptr[h * nqb + qb];
+  }
+  for (int e = threadIdx.x; e < nl; e += blockDim.x) {
+    const int kb = dsel ? qb - lst[e] : lst[e];
+    if (kb < 0 || kb > qb) continue;
+    if (e > 0 && (dsel ? lst[e - 1] == lst[e] : lst[e - 1] == lst[e])) continue;  // repeated entry
+    if (kind == DSA_KIND_ASHAPE) {
+      tot += ashape_pairs_in_block(kb, B, r0, r1, sink, window);
+    } else if (kb < qb) {
+      tot += (int64_t)nrows * B;
+    } else {
+      // diagonal block: row i sees keys r0 .. i
+      tot += (int64_t)nrows * (nrows + 1) / 2;
+    }
+  }
+  const int cb = col_ptr[h * nqb + qb], ce = col_ptr[h * nqb + qb + 1];
+  for (int e = cb + threadIdx.x; e < ce; e += blockDim.x) {
+    const int j = col_idx[e];
+    if (j < 0 || j > r1) continue;
+    const int kb = j / B;
+    const bool covered = dsel ? sorted_contains(lst, nl, qb - kb) : sorted_contains(lst, nl, kb);
+    if (covered) continue;
+    tot += r1 - max(j, r0) + 1;
+  }
+  __shared__ unsigned long long sh[32];
+  unsigned long long v = (unsigned long long)tot;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) sh[threadIdx.x >> 5] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long s = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) s += sh[i];
+    atomicAdd(&pairs[h], s);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host planning
+// ---------------------------------------------------------------------------
+dsa_status check_pattern(const dsa_problem& p, const dsa_pattern& q) {
+  switch (q.kind) {
+    case DSA_KIND_ASHAPE:
+      if (q.sink < 0 || q.window < 1) return DSA_ERR_INVALID_ARG;
+      return DSA_OK;
+    case DSA_KIND_VS:
+      if (q.last_q < 1 || q.n_vert < 0 || q.n_slash < 0) return DSA_ERR_INVALID_ARG;
+      if (q.last_q > VS_MAXL) return DSA_ERR_UNSUPPORTED;
+      return DSA_OK;
+    case DSA_KIND_BLOCK_TOPK:
+      if (q.topk < 1) return DSA_ERR_INVALID_ARG;
+      return DSA_OK;
+    case DSA_KIND_BLOCK_THRESHOLD:
+      if (!(q.alpha > 0.f && q.alpha <= 1.f)) return DSA_ERR_INVALID_ARG;
+      return DSA_OK;
+    case DSA_KIND_MOBA:
+      if (q.topk < 0 || q.conv_width < 0 || q.conv_width > 8) return DSA_ERR_INVALID_ARG;
+      if (q.conv_width > 0 && (q.conv_weight == nullptr || q.conv_bias == nullptr)) return DSA_ERR_INVALID_ARG;
+      return DSA_OK;
+    default:
+      return DSA_ERR_INVALID_ARG;
+  }
+  (void)p;
+}
+
+bool is_block_kind(int k) {
+  return k == DSA_KIND_BLOCK_TOPK || k == DSA_KIND_BLOCK_THRESHOLD || k == DSA_KIND_MOBA;
+}
+
+int vs_rows_pad(int lq) {
+  int rt = 1;
+  while (rt * 16 < lq) rt *= 2;
+  return rt;
+}
+
+dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L, HeadTab* ht, ConvTab* ct,
+                       dsa_sizes* sz) {
+  if (p.Hq > MAXH || p.Hkv > MAXKV) return DSA_ERR_UNSUPPORTED;
+  L->Hq = p.Hq;
+  L->Hkv = p.Hkv;
+  L->G = p.Hq / p.Hkv;
+  L->N = p.N;
+  L->d = p.d;
+  L->B = p.block;
+  L->nqb = ceil_div(p.N, p.block);
+  L->nkw = ceil_div(L->nqb, 32);
+  L->nbh = 0;
+  L->nvs = 0;
+  L->vs_lmax = 0;
+  L->vs_nchunks = ceil_div(p.N, VS_CHUNK);
+  if (ht) memset(ht, 0, sizeof(HeadTab));
+  if (ct) memset(ct, 0, sizeof(ConvTab));
+  int64_t blk = 0, dcap = 0, ccap = 0;
+  int vstride = 1, sstride = 1;
+  const int nqb = L->nqb, B = p.block, N = p.N;
+  for (int h = 0; h < p.Hq; ++h) {
+    const dsa_pattern& q = pats[h];
+    dsa_status s = check_pattern(p, q);
+    if (s != DSA_OK) return s;
+    if (ht) {
+      ht->kind[h] = q.kind;
+      ht->sink[h] = q.sink;
+      ht->window[h] = q.window;
+      ht->last_q[h] = q.last_q;
+      ht->n_vert[h] = q.n_vert;
+      ht->n_slash[h] = q.n_slash;
+      ht->topk[h] = q.topk;
+      ht->lnalpha[h] = q.kind == DSA_KIND_BLOCK_THRESHOLD ? logf(q.alpha) : 0.f;
+      ht->keep_sink[h] = q.keep_sink;
+      ht->keep_local[h] = q.keep_local;
+      ht->bslot[h] = -1;
+      ht->vslot[h] = -1;
+    }
+    if (is_block_kind(q.kind)) {
+      if (ht) {
+        ht->bslot[h] = L->nbh;
+        ht->bhead[L->nbh] = h;
+      }
+      L->nbh++;
+      const int kvh = h / L->G;
+      if (ct) {
+        if (ct->need[kvh]) {
+          const int w = q.kind == DSA_KIND_MOBA ? q.conv_width : 0;
+          if (ct->width[kvh] != w || (w > 0 && (ct->w[kvh] != q.conv_weight || ct->b[kvh] != q.conv_bias)))
+            return DSA_ERR_INVALID_ARG;  // block heads of one KV group must share the key conv
+        } else {
+          ct->need[kvh] = 1;
+          ct->width[kvh] = q.kind == DSA_KIND_MOBA ? q.conv_width : 0;
+          ct->w[kvh] = ct->width[kvh] ? q.conv_weight : nullptr;
+          ct->b[kvh] = ct->width[kvh] ? q.conv_bias : nullptr;
+        }
+      }
+      for (int qb = 0; qb < nqb; ++qb) {
+        if (q.kind == DSA_KIND_BLOCK_TOPK) blk += std::min(q.topk, qb + 1);
+        else if (q.kind == DSA_KIND_MOBA) blk += std::min(q.topk, qb) + 1;
+        else blk += qb + 1;
+      }
+    } else if (q.kind == DSA_KIND_ASHAPE) {
+      for (int qb = 0; qb < nqb; ++qb) {
+        const int r0 = qb * B, r1 = std::min(N - 1, r0 + B - 1);
+        const int a = ceil_div(std::min(q.sink, r1 + 1), B);
+        const int w = std::max(0, r0 - q.window + 1) / B;
+        blk += a + std::max(0, qb + 1 - std::max(w, a));
+      }
+    } else {  // VS
+      if (ht) {
+        ht->vslot[h] = L->nvs;
+        ht->vhead[L->nvs] = h;
+      }
+      L->nvs++;
+      const int nv = std::min(q.n_vert, N), ns = std::min(q.n_slash, N);
+      vstride = std::max(vstride, nv);
+      sstride = std::max(sstride, ns);
+      dcap += std::min<int64_t>(2 * (int64_t)ns, nqb);
+      for (int qb = 0; qb < nqb; ++qb) ccap += std::min<int64_t>(nv, (int64_t)qb * B + B);
+      L->vs_lmax = std::max(L->vs_lmax, 16 * vs_rows_pad(std::min(q.last_q, N)));
+    }
+  }
+  if (blk > INT32_MAX || ccap > INT32_MAX || (int64_t)p.Hq * nqb + 1 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
+  if (L->nbh > 0 && L->nqb > 16384) return DSA_ERR_UNSUPPORTED;  // block scores live in shared memory
+  const int64_t d = p.d;
+  int64_t off = 0;
+  L->off_qbar = off; off = align256(off + (int64_t)L->nbh * nqb * d * 4);
+  L->off_kbar = off; off = align256(off + (L->nbh ? (int64_t)p.Hkv * nqb * d * 4 : 0));
+  L->off_sel = off;  off = align256(off + (int64_t)L->nbh * nqb * L->nkw * 4);
+  L->off_v = off;    off = align256(off + (int64_t)L->nvs * N * 4);
+  L->off_s = off;    off = align256(off + (int64_t)L->nvs * N * 4);
+  L->off_part = off; off = align256(off + (int64_t)L->nvs * L->vs_nchunks * VS_MAXL * 2 * 4);
+  L->off_stat = off; off = align256(off + (int64_t)L->nvs * VS_MAXL * 2 * 4);
+  L->off_dtmp = off; off = align256(off + (int64_t)L->nvs * nqb * 4);
+  L->off_dbits = off; off = align256(off + (int64_t)L->nvs * L->nkw * 4);
+  L->total = std::max<int64_t>(off, 256);
+  if (sz) {
+    sz->nqb = nqb;
+    sz->vert_stride = vstride;
+    sz->slash_stride = sstride;
+    sz->reserved = 0;
+    sz->head_info_len = 4 * (int64_t)p.Hq;
+    sz->blk_ptr_len = (int64_t)p.Hq * nqb + 1;
+    sz->blk_cap = std::max<int64_t>(blk, 1);
+    sz->dist_ptr_len = p.Hq + 1;
+    sz->dist_cap = std::max<int64_t>(dcap, 1);
+    sz->col_ptr_len = (int64_t)p.Hq * nqb + 1;
+    sz->col_cap = std::max<int64_t>(ccap, 1);
+    sz->workspace_bytes = L->total;
+  }
+  return DSA_OK;
+}
+
+template <int D>
+dsa_status launch_vs(const HeadTab& ht, const Layout& L, const void* Q, int64_t q_hs, int64_t q_ts, const void* K,
+                     int64_t k_hs, int64_t k_ts, uint8_t* ws, cudaStream_t st) {
+  const int RT = L.vs_lmax / 16;
+  const int LP = L.vs_lmax;
+  const size_t smem = (size_t)(LP + VS_SUB) * (D + 8) * 2 + (size_t)LP * (VS_SUB + 4) * 4 +
+                      (size_t)(VS_CHUNK + LP + VS_CHUNK + 2 * LP + 16 * LP) * 4;
+  const dim3 grid(L.vs_nchunks * L.nvs);
+  const auto* q = static_cast<const __nv_bfloat16*>(Q);
+  const auto* k = static_cast<const __nv_bfloat16*>(K);
+#define DSA_VS_LAUNCH(R)                                                                                   \
+  do {                                                                                                     \
+    cudaFuncSetAttribute(k_vs<D, R, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
+    cudaFuncSetAttribute(k_vs<D, R, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
+    k_vs<D, R, 1><<<grid, 256, smem, st>>>(ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);                        \
+    k_vs_rowstats<<<L.nvs, 128, 0, st>>>(ht, L, ws);                                                       \
+    k_vs<D, R, 2><<<grid, 256, smem, st>>>(ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);                        \
+  } while (0)
+  switch (RT) {
+    case 1: DSA_VS_LAUNCH(1); break;
+    case 2: DSA_VS_LAUNCH(2); break;
+    case 4: DSA_VS_LAUNCH(4); break;
+    case 8: DSA_VS_LAUNCH(8); break;
+    default: return DSA_ERR_UNSUPPORTED;
+  }
+#undef DSA_VS_LAUNCH
+  return DSA_OK;
+}
+
+}  // namespace
+
+dsa_status plan_sizes(const dsa_problem& p, const dsa_pattern* pats, dsa_sizes* out) {
+  static thread_local ConvTab ct;  // validates the per-group key conv as well
+  Layout L;
+  return make_layout(p, pats, &L, nullptr, &ct, out);
+}
+
+dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void* K, const dsa_pattern* pats,
+                                const dsa_indices& out, void* ws_v, size_t ws_bytes, cudaStream_t st,
+                                unsigned* status) {
+  static thread_local HeadTab ht;
+  static thread_local ConvTab ct;
+  Layout L;
+  dsa_sizes sz;
+  dsa_status s = make_layout(p, pats, &L, &ht, &ct, &sz);
+  if (s != DSA_OK) return s;
+  if ((int64_t)ws_bytes < sz.workspace_bytes) return DSA_ERR_CAPACITY;
+  if (out.blk_cap < sz.blk_cap || out.dist_cap < sz.dist_cap || out.col_cap < sz.col_cap) return DSA_ERR_CAPACITY;
+  if (L.nvs > 0 && (!out.vert_idx || !out.slash_idx || out.vert_stride < sz.vert_stride ||
+                    out.slash_stride < sz.slash_stride))
+    return DSA_ERR_CAPACITY;
+  uint8_t* ws = static_cast<uint8_t*>(ws_v);
+  const int nrows = p.Hq * L.nqb + 1;
+  cudaError_t e;
+#define DSA_CK(x)                          \
+  do {                                     \
+    e = (x);                               \
+    if (e != cudaSuccess) return cuda_fail(e); \
+  } while (0)
+  DSA_CK(cudaMemsetAsync(out.blk_ptr, 0, sizeof(int32_t) * nrows, st));
+  DSA_CK(cudaMemsetAsync(out.col_ptr, 0, sizeof(int32_t) * nrows, st));
+  DSA_CK(cudaMemsetAsync(out.dist_ptr, 0, sizeof(int32_t) * (p.Hq + 1), st));
+  k_head_info<<<ceil_div(p.Hq, 128), 128, 0, st>>>(ht, p.Hq, out.head_info);
+  k_ashape_count<<<dim3(ceil_div(L.nqb, 128), p.Hq), 128, 0, st>>>(ht, L, out.blk_ptr);
+  const auto* q = static_cast<const __nv_bfloat16*>(Q);
+  const auto* k = static_cast<const __nv_bfloat16*>(K);
+  if (L.nbh > 0) {
+    const size_t sel_smem = (size_t)L.nqb * 4;
+    if (p.d == 128) {
+      k_pool<128><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
+                                                             p.k_head_stride, p.k_token_stride, ws);
+      DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
+      k_block_select<128><<<dim3(L.nqb, L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+    } else {
+      k_pool<64><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
+                                                            p.k_head_stride, p.k_token_stride, ws);
+      DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
+      k_block_select<64><<<dim3(L.nqb, L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+    }
+  }
+  if (L.nvs > 0) {
+    DSA_CK(cudaMemsetAsync(ws + L.off_s, 0, (size_t)L.nvs * p.N * 4, st));
+    s = (p.d == 128) ? launch_vs<128>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
+                                      p.k_token_stride, ws, st)
+                     : launch_vs<64>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
+                                     p.k_token_stride, ws, st);
+    if (s != DSA_OK) return s;
+    k_vs_topk<<<dim3(L.nvs, 2), 1024, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride, out.slash_idx,
+                                                out.slash_stride);
+    k_vs_dist<<<L.nvs, 256, 0, st>>>(ht, L, ws, out.slash_idx, out.slash_stride, out.dist_ptr);
+    k_vs_cols<false><<<dim3(ceil_div(L.nqb, 8), L.nvs), 256, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride,
+                                                                      out.col_ptr, out.col_idx, out.col_cap, status);
+  }
+  k_scan<<<3, 1024, 0, st>>>(out.blk_ptr, nrows, out.blk_cap, out.col_ptr, nrows, out.col_cap, out.dist_ptr,
+                             p.Hq + 1, out.dist_cap, status);
+  k_blk_fill<<<dim3(ceil_div(L.nqb, 8), p.Hq), 256, 0, st>>>(ht, L, ws, out.blk_ptr, out.blk_idx, out.blk_cap,
+                                                            status);
+  if (L.nvs > 0) {
+    k_dist_fill<<<L.nvs, 256, 0, st>>>(ht, L, ws, out.dist_ptr, out.dist, out.dist_cap, status);
+    k_vs_cols<true><<<dim3(ceil_div(L.nqb, 8), L.nvs), 256, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride,
+                                                                     out.col_ptr, out.col_idx, out.col_cap, status);
+  }
+  DSA_CK(cudaGetLastError());
+#undef DSA_CK
+  return DSA_OK;
+}
+
+dsa_status launch_count_pairs(const dsa_problem& p, const dsa_indices& idx, int64_t* pairs, cudaStream_t st,
+                              unsigned* status) {
+  (void)status;
+  const int nqb = ceil_div(p.N, p.block);
+  cudaError_t e = cudaMemsetAsync(pairs, 0, sizeof(int64_t) * p.Hq, st);
+  if (e != cudaSuccess) return cuda_fail(e);
+  k_count_pairs<<<dim3(nqb, p.Hq), 128, 0, st>>>(p.Hq, p.N, p.block, nqb, idx.head_info, idx.blk_ptr, idx.blk_idx,
+                                                 idx.dist_ptr, idx.dist, idx.col_ptr, idx.col_idx,
+                                                 reinterpret_cast<unsigned long long*>(pairs));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e);
+  return DSA_OK;
+}
+
+}  // namespace dsa

@@ -1,0 +1,37 @@
+// Host-side declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "dsa.h"
+
+namespace dsa {
+
+// Device address of this device's status word (4 x uint32), or nullptr on failure.
+unsigned* status_ptr();
+
+// Records a CUDA error for dsa_last_cuda_error and returns DSA_ERR_CUDA.
+dsa_status cuda_fail(cudaError_t e);
+
+// Default bound on every in-kernel wait (ns of global time).
+constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+dsa_status validate_problem(const dsa_problem* p);
+dsa_status validate_indices_ptrs(const dsa_indices* idx, bool for_build);
+
+dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K, const void* V,
+                              const dsa_indices& idx, void* O, float* lse, cudaStream_t stream,
+                              unsigned* status);
+
+dsa_status launch_count_pairs(const dsa_problem& p, const dsa_indices& idx, int64_t* pairs,
+                              cudaStream_t stream, unsigned* status);
+
+dsa_status plan_sizes(const dsa_problem& p, const dsa_pattern* pats, dsa_sizes* out);
+
+dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void* K,
+                                const dsa_pattern* pats, const dsa_indices& out, void* ws,
+                                size_t ws_bytes, cudaStream_t stream, unsigned* status);
+
+}  // namespace dsa

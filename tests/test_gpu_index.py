@@ -1,0 +1,142 @@
+"""GPU parity of dsa_build_indices against the fp64 oracle.
+
+Index sets must match exactly, except for entries whose oracle score lies within
+1e-3 (relative) of the top-k / threshold cut.  Integer steps that follow a
+selection (VS distances and columns) are compared bit-exactly against the
+oracle's rule applied to the GPU's own selection, so a near-tie cannot cascade.
+The attention output with the GPU's indices is then checked against the oracle
+evaluating the same indices."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import dsa_oracle as orc
+from tests._parity import (assert_close_outputs, assert_lse_close, gpu_lists_to_oracle_heads,
+                           threshold_set_ok, to64, topk_set_ok)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import dynamic_sparse_attention_build_b200 as m
+    return m
+
+
+def check_indices(bufs, ref_heads, pats, N, B, convs_ref=None):
+    gl = bufs.host_lists()
+    nqb = (N + B - 1) // B
+    for h, (g, r, p) in enumerate(zip(gl, ref_heads, pats)):
+        kind = p["kind"]
+        if kind == "ashape":
+            assert g["kind"] == 0 and g["sink"] == p["sink"] and g["window"] == p["window"]
+            for qb in range(nqb):
+                assert list(g["blocks"][qb]) == list(r.blocks[qb]), (h, qb)
+        elif kind == "vs":
+            ok, msg = topk_set_ok(g["vert"], r.V, r.vscore, p["n_vert"])
+            assert ok, f"head {h} verticals: {msg}"
+            ok, msg = topk_set_ok(g["slash"], r.S, r.sscore, p["n_slash"])
+            assert ok, f"head {h} slashes: {msg}"
+            assert list(g["vert"]) == sorted(g["vert"]) and list(g["slash"]) == sorted(g["slash"])
+            D = orc.vs_distance_set(np.asarray(g["slash"], np.int64), B, nqb)
+            assert list(g["dist"]) == list(D), f"head {h} distances"
+            for qb in range(nqb):
+                want = orc.vs_columns(np.asarray(g["vert"], np.int64), D, qb, B)
+                assert list(g["cols"][qb]) == list(want), (h, qb)
+        else:
+            sc = r.block_scores
+            for I in range(nqb):
+                gs, rs = g["blocks"][I], r.blocks[I]
+                assert list(gs) == sorted(set(gs.tolist())), (h, I)
+                if kind == "block_threshold":
+                    forced = {0, I}
+                    ok, msg = threshold_set_ok(gs, rs, sc[I], I, p["alpha"], forced)
+                elif kind == "moba":
+                    assert I in set(gs.tolist())
+                    ok, msg = topk_set_ok([x for x in gs if x != I], [x for x in rs if x != I], sc[I][:I],
+                                          p["topk"], logit=True) if I > 0 else (True, "")
+                else:
+                    ok, msg = topk_set_ok(gs, rs, sc[I][: I + 1], p["topk"], logit=True)
+                assert ok, f"head {h} block {I}: {msg}"
+
+
+def run(dsa, Q, K, V, pats, B, rows=None, convs=None):
+    N = Q.shape[1]
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    dpats = []
+    G = Q.shape[0] // K.shape[0]
+    for h, p in enumerate(pats):
+        p = dict(p)
+        if convs is not None and p["kind"] == "moba":
+            w, b = convs[h // G]
+            p["conv"] = (w.cuda(), b.cuda())
+        dpats.append(p)
+    bufs = dsa.build_indices(Qd, Kd, dpats, B)
+    torch.cuda.synchronize()
+    st, det = dsa.device_status()
+    assert st == 0, (st, det)
+    oconvs = None
+    if convs is not None:
+        oconvs = [(convs[h // G][0].double().numpy(), convs[h // G][1].double().numpy()) for h in range(len(pats))]
+    ref = orc.build_indices(to64(Q), to64(K), pats, B, oconvs)
+    check_indices(bufs, ref, pats, N, B)
+    # attention with the GPU's own indices
+    O, lse = dsa.sparse_prefill(Qd, Kd, Vd, bufs, want_lse=True)
+    torch.cuda.synchronize()
+    heads = gpu_lists_to_oracle_heads(bufs, N, B)
+    rows = np.arange(N) if rows is None else np.asarray(rows)
+    O_ref, lse_ref = orc.sparse_attention(to64(Q), to64(K), to64(V), heads, rows)
+    assert_close_outputs(to64(O)[:, rows], O_ref, "O")
+    assert_lse_close(lse.cpu().double().numpy()[:, rows], lse_ref, "lse")
+    # exact pair count of the index mask
+    pairs = dsa.count_pairs(Qd, Kd, bufs).cpu().numpy()
+    if N <= 1500:
+        want = [orc.selected_pairs(hh) for hh in heads]
+        assert list(pairs) == want
+    return bufs
+
+
+def test_vs_tiny_workload(dsa):
+    w = synth.workload(1)
+    Q, K, V, planted = synth.make_inputs(w)
+    bufs = run(dsa, Q, K, V, synth.head_patterns(w), w["B"])
+    assert set(planted["vert"][0].tolist()) <= set(bufs.host_lists()[0]["vert"].tolist())
+
+
+def test_mixed_gqa_ragged(dsa):
+    N, d, B = 1500, 128, 64
+    Q, K, V = synth.random_qkv(8, 2, N, d, seed=21)
+    pats = [dict(kind="vs", last_q=64, n_vert=60, n_slash=50),
+            dict(kind="ashape", sink=100, window=300),
+            dict(kind="block_topk", topk=5),
+            dict(kind="vs", last_q=20, n_vert=2000, n_slash=7),
+            dict(kind="block_threshold", alpha=0.5, keep_sink=1, keep_local=1),
+            dict(kind="block_topk", topk=100),
+            dict(kind="vs", last_q=128, n_vert=0, n_slash=1),
+            dict(kind="ashape", sink=0, window=1)]
+    run(dsa, Q, K, V, pats, B)
+
+
+@pytest.mark.parametrize("B", [128, 512])
+@pytest.mark.parametrize("conv", [False, True])
+def test_moba(dsa, B, conv):
+    w = synth.workload(4, N=1400 if B == 128 else 2600, Hq=2, Hkv=2, B=B, conv_width=4 if conv else 0)
+    Q, K, V, _ = synth.make_inputs(w)
+    convs = synth.conv_weights(w)
+    run(dsa, Q, K, V, synth.head_patterns(w), B, convs=convs,
+        rows=np.r_[0:64, 500:600, w["N"] - 200:w["N"]])
+
+
+def test_threshold_topics(dsa):
+    w = synth.workload(3, N=4096, Hq=4, Hkv=2)
+    Q, K, V, planted = synth.make_inputs(w)
+    bufs = run(dsa, Q, K, V, synth.head_patterns(w), w["B"], rows=np.r_[0:130, 2000:2100, 3900:4096])
+    # same-topic blocks are found: every kept block J < I shares I's topic, and
+    # the blocks earlier in the sequence with I's topic are kept
+    topic = planted["topic"][0].numpy()
+    lists = bufs.host_lists()[0]["blocks"]
+    hits = sum(int(all(topic[J] == topic[I] for J in lists[I] if J not in (0, I))) for I in range(len(lists)))
+    assert hits >= 0.9 * len(lists)
