@@ -1,0 +1,370 @@
+"""Benchmark of one dynamic-sparse-attention prefill layer on B200.
+
+One step = the whole hot path over one layer of synthetic input: build the
+per-head sparse indices (dsa_build_indices) and run the sparse attention forward
+(dsa_sparse_prefill).  The default workload is the Llama-3-8B-shaped layer:
+32 q / 8 KV heads, d = 128, N = 32768 tokens, bf16, per-head patterns drawn from
+the seed (20% A-shape 128/1024, 60% Vertical-Slash 64/1000/6096, 20% block
+top-100), block 64.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
+
+With torchrun (N > 1) every rank runs its own independent layer (heads and
+layers shard with no data-path exchange: weak scaling); the only collectives are
+the timing barrier and the max-over-ranks reduction.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "sparse prefill tokens/s per layer and % of B200 bf16 tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if "Active" in r[5 + k]
+                          and "Not" not in r[5 + k]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def algorithmic_index_bytes(w, pats):
+    """Bytes the index build must move: Q read once for pooled-Q heads, K read once
+    per KV head that is pooled or scanned by a VS estimate, the last_q query rows,
+    the VS score arrays written and read once, and the index lists written."""
+    N, d, Bk, G = w["N"], w["d"], w["B"], w["Hq"] // w["Hkv"]
+    nqb = (N + Bk - 1) // Bk
+    byt = 0
+    kv_read = set()
+    for h, p in enumerate(pats):
+        if p["kind"] in ("block_topk", "block_threshold", "moba"):
+            byt += N * d * 2
+            kv_read.add(h // G)
+        elif p["kind"] == "vs":
+            byt += min(p["last_q"], N) * d * 2 + 2 * 2 * 4 * N
+            kv_read.add(h // G)
+    byt += len(kv_read) * N * d * 2
+    return byt, nqb
+
+
+def build_workload(w, device, seed_offset=0):
+    w = dict(w)
+    w["seed"] = w["seed"] + seed_offset
+    Q, K, V, planted = synth.make_inputs(w, device=device)
+    pats = synth.head_patterns(w)
+    convs = synth.conv_weights(w, device=device)
+    if convs is not None:
+        G = w["Hq"] // w["Hkv"]
+        pats = [dict(p, conv=convs[h // G]) if p["kind"] == "moba" else p for h, p in enumerate(pats)]
+    return Q, K, V, pats
+
+
+def kernel_launches_per_step(pats):
+    kinds = [p["kind"] for p in pats]
+    n = 4  # head info, A-shape counts, scan, block fill
+    if any(k in ("block_topk", "block_threshold", "moba") for k in kinds):
+        n += 2  # pool, block score/select
+    if "vs" in kinds:
+        n += 8  # VS pass 1, row stats, pass 2, top-k, distances, column count, distance fill, column fill
+    return n + 1  # attention
+
+
+# --------------------------------------------------------------------------- oracle timing
+def oracle_sample(w, Q, K, V, pats, target_s=15.0):
+    """Times the CPU oracle on a bounded sample of the layer and extrapolates to
+    the whole layer.  Sample: the full index build of one head of each pattern
+    kind present, and the attention of evenly spaced rows of those heads (time per
+    row scales with the row's allowed keys, so rows are spread over the sequence).
+    Returns (estimated layer seconds, description, threads)."""
+    from oracle import dsa_oracle as orc
+    N, B, G = w["N"], w["B"], w["Hq"] // w["Hkv"]
+    q = Q.to("cpu", torch.float64).numpy()
+    k = K.to("cpu", torch.float64).numpy()
+    v = V.to("cpu", torch.float64).numpy()
+    by_kind = {}
+    for h, p in enumerate(pats):
+        by_kind.setdefault(p["kind"], []).append(h)
+    est = 0.0
+    parts = []
+    budget_rows = 0
+    t_idx = {}
+    heads = {}
+    for kind, hs in by_kind.items():
+        h = hs[0]
+        conv = None
+        p = dict(pats[h])
+        if "conv" in p:
+            cw, cb = p.pop("conv")
+            conv = (cw.double().cpu().numpy(), cb.double().cpu().numpy())
+        t0 = time.perf_counter()
+        heads[kind] = orc.build_head_index(q[h], k[h // G], p, B, conv)
+        t_idx[kind] = time.perf_counter() - t0
+        est += t_idx[kind] * len(hs)
+    # attention: rows spread over the sequence, grown until the budget is used
+    t_att = {}
+    n_rows = 8
+    spent = sum(t_idx.values())
+    while True:
+        rows = np.unique(np.linspace(0, N - 1, n_rows).astype(np.int64))
+        t_att = {}
+        for kind, hs in by_kind.items():
+            h = hs[0]
+            t0 = time.perf_counter()
+            orc.attention_rows(q[h], k[h // G], v[h // G], heads[kind], rows)
+            t_att[kind] = time.perf_counter() - t0
+        spent += sum(t_att.values())
+        if spent > target_s or n_rows >= N:
+            break
+        n_rows *= 2
+    for kind, hs in by_kind.items():
+        est += t_att[kind] / rows.size * N * len(hs)
+    budget_rows = rows.size
+    desc = (f"full index build of one head per pattern kind ({', '.join(sorted(by_kind))}) and attention of "
+            f"{budget_rows} evenly spaced rows of each; extrapolated to {w['Hq']} heads x {N} rows")
+    threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    return est, desc, threads, spent
+
+
+# --------------------------------------------------------------------------- main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
+    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    args = ap.parse_args()
+    rank, world, local = dist_env()
+    w = synth.workload(args.workload)
+
+    if args.impl == "reference":
+        # the oracle, as it stands, on the host cores; rank 0 only
+        if rank != 0:
+            return
+        torch.manual_seed(0)
+        Q, K, V, pats = build_workload(w, "cuda" if torch.cuda.is_available() else "cpu")
+        per_step = min(15.0, max(2.0, 150.0 / max(1, args.steps + args.warmup)))
+        for _ in range(args.warmup):
+            oracle_sample(w, Q, K, V, pats, target_s=1.0)
+        times = []
+        desc = threads = None
+        for _ in range(args.steps):
+            est, desc, threads, spent = oracle_sample(w, Q, K, V, pats, target_s=per_step)
+            times.append(est)
+        t = statistics.mean(times)
+        val = w["N"] / t
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": w["name"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
+                           "block": w["B"]},
+                "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                 "sample": desc},
+                "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    import dynamic_sparse_attention_build_b200 as dsa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=dev)
+    Q, K, V, pats = build_workload(w, dev, seed_offset=rank)
+    N, Hq, d = w["N"], w["Hq"], w["d"]
+    pats_c = dsa.make_patterns(pats)
+    bufs = dsa.build_indices(Q, K, pats_c, w["B"])
+    O = torch.empty_like(Q)
+    O, _ = dsa.sparse_prefill(Q, K, V, bufs, O=O)
+    torch.cuda.synchronize()
+    st, det = dsa.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det}")
+    pairs = dsa.count_pairs(Q, K, bufs).sum().item()
+    f_sel = 4.0 * d * pairs
+    causal_pairs = Hq * N * (N + 1) / 2
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsa.build_indices(Q, K, pats_c, w["B"], bufs=bufs)
+        if ev is not None:
+            ev[1].record(stream)
+        dsa.sparse_prefill(Q, K, V, bufs, O=O)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    for i in range(args.steps):
+        flush.zero_()  # L2 flush between timed steps, outside the step's events
+        step(evs[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    t_build = [e[0].elapsed_time(e[1]) for e in evs]
+    t_attn = [e[1].elapsed_time(e[2]) for e in evs]
+    t_step = [a + b for a, b in zip(t_build, t_attn)]
+    tot = torch.tensor([sum(t_step), sum(t_build), sum(t_attn)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
+    ms_step = tot[0].item() / args.steps
+    ms_build = tot[1].item() / args.steps
+    ms_attn = tot[2].item() / args.steps
+    st, det = dsa.device_status()
+    if st != 0:
+        raise RuntimeError(f"device status {st} detail {det}")
+
+    # end to end through the public API with pinned host buffers
+    Qh = Q.cpu().pin_memory()
+    Kh = K.cpu().pin_memory()
+    Vh = V.cpu().pin_memory()
+    Oh = torch.empty_like(Qh).pin_memory()
+    Qe, Ke, Ve = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+
+    def e2e_step():
+        Qe.copy_(Qh, non_blocking=True)
+        Ke.copy_(Kh, non_blocking=True)
+        Ve.copy_(Vh, non_blocking=True)
+        dsa.build_indices(Qe, Ke, pats_c, w["B"], bufs=bufs)
+        dsa.sparse_prefill(Qe, Ke, Ve, bufs, O=O)
+        Oh.copy_(O, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = e2e_ms.item()
+
+    pk, pk_src = peaks()
+    tflops = f_sel / (ms_attn * 1e-3) / 1e12
+    peak_tf = pk["bf16_tflops"]
+    idx_bytes, nqb = algorithmic_index_bytes(w, pats)
+    idx_gbs = idx_bytes / (ms_build * 1e-3) / 1e9
+    traffic = None
+    tp = os.path.join(ROOT, "profiles", "attention_traffic.json")
+    if os.path.exists(tp):
+        tr = json.load(open(tp))
+        if tr.get("workload") == w["name"]:
+            traffic = tr.get("dram_bytes_per_launch")
+
+    line = {
+        "metric": METRIC, "value": N * world / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
+                   "patterns": "seeded per head: 20% A-shape 128/1024, 60% VS 64/1000/6096, 20% block top-100",
+                   "l2": "flushed by a 256 MiB write before every timed step (outside its events)",
+                   "parallelism": f"independent layer per rank x{world}"},
+        "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
+                     "frac": tflops / peak_tf, "traffic": traffic,
+                     "kernel": "sparse_attn_kernel<128>", "peak_source": f"{pk_src} bf16 burst (cuBLAS)",
+                     "work": f"F_sel = 4*d*|M| = {f_sel:.4e} FLOP per launch ({pairs} allowed pairs)"},
+        "attention": {"ms": ms_attn, "tflops": tflops, "frac_peak": tflops / peak_tf,
+                      "density_vs_causal": pairs / causal_pairs},
+        "index_build": {"ms": ms_build, "algorithmic_bytes": idx_bytes, "gbs": idx_gbs,
+                        "frac_hbm": idx_gbs / pk["hbm_gbs"], "hbm_peak_source": pk_src},
+        "e2e": {"value": N * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+                "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * 2,
+                "d2h_bytes_per_step": O.numel() * 2, "ms_per_step": e2e_ms},
+        "gpu_launches": kernel_launches_per_step(pats) * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, desc, threads, spent = oracle_sample(w, Q, K, V, pats)
+        line["cpu_baseline"] = {"value": N / est, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                                "sample": desc + f" ({spent:.1f} s of CPU work)"}
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
