@@ -198,9 +198,10 @@ def main():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--N", type=int, default=0, help="override the token count (smaller profiling cases)")
     args = ap.parse_args()
     rank, world, local = dist_env()
-    w = synth.workload(args.workload)
+    w = synth.workload(args.workload, **({"N": args.N} if args.N else {}))
 
     if args.impl == "reference":
         # the oracle, as it stands, on the host cores; rank 0 only
