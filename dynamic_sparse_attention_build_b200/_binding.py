@@ -31,7 +31,7 @@ KIND_CODES = {"ashape": DSA_KIND_ASHAPE, "vs": DSA_KIND_VS, "block_topk": DSA_KI
 
 EXPORTS = ("dsa_workspace_size", "dsa_build_indices", "dsa_sparse_prefill", "dsa_count_pairs",
            "dsa_get_device_status", "dsa_selftest_wait_timeout", "dsa_status_string",
-           "dsa_last_cuda_error")
+           "dsa_last_cuda_error", "dsa_build_indices_static")
 
 
 class dsa_problem(ctypes.Structure):
@@ -87,6 +87,8 @@ def lib():
                                         P(dsa_indices), ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]
         L.dsa_sparse_prefill.argtypes = [P(dsa_problem), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                          P(dsa_indices), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+        L.dsa_build_indices_static.argtypes = [P(dsa_problem), ctypes.c_void_p, ctypes.c_void_p,
+                                               P(dsa_pattern), P(dsa_indices), ctypes.c_void_p]
         L.dsa_count_pairs.argtypes = [P(dsa_problem), P(dsa_indices), ctypes.c_void_p, ctypes.c_void_p]
         L.dsa_get_device_status.argtypes = [ctypes.c_void_p, P(ctypes.c_int32)]
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
@@ -124,6 +126,11 @@ def dsa_workspace_size(problem, patterns):
 def dsa_build_indices(problem, Q_ptr, K_ptr, patterns, indices, ws_ptr, ws_bytes, stream_ptr):
     return lib().dsa_build_indices(ctypes.byref(problem), Q_ptr, K_ptr, patterns, ctypes.byref(indices),
                                    ws_ptr, ws_bytes, stream_ptr)
+
+
+def dsa_build_indices_static(problem, Q_ptr, K_ptr, patterns, indices, stream_ptr):
+    return lib().dsa_build_indices_static(ctypes.byref(problem), Q_ptr, K_ptr, patterns,
+                                          ctypes.byref(indices), stream_ptr)
 
 
 def dsa_sparse_prefill(problem, Q_ptr, K_ptr, V_ptr, indices, O_ptr, lse_ptr, stream_ptr):

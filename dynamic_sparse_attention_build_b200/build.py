@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
-SOURCES = ["dsa_api.cu", "dsa_attn.cu", "dsa_index.cu"]
+SOURCES = ["dsa_api.cu", "dsa_attn.cu", "dsa_index.cu", "dsa_noalloc.cu"]
 LIB = os.path.join(HERE, "libdsa.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -197,6 +197,24 @@ dsa_status dsa_get_device_status(dsa_stream stream, int32_t* detail);
  * timeout reporting without faulting or hanging the GPU. */
 dsa_status dsa_selftest_wait_timeout(uint32_t timeout_us, dsa_stream stream);
 
+/* dsa_build_indices without a workspace argument, for callers that cannot
+ * allocate device memory (a plugin inside another runtime that owns all device
+ * memory, or a latency-critical path where cudaMalloc would synchronise the
+ * device).  The pages have no counterpart: this is a deployment variant of the
+ * same index builder, with identical results.
+ * Scratch comes from a 16 MiB buffer compiled into the library: every GPU that
+ * loads the library holds it until the process exits.  A problem whose
+ * sizes.workspace_bytes exceeds 16 MiB returns DSA_ERR_CAPACITY and enqueues
+ * nothing.  The library allocates and frees nothing in this call.
+ * The first call on a device (with that device current) looks up the buffer's
+ * device address; make that first call before any stream capture.
+ * All calls on a device share the buffer and it keeps the previous call's
+ * contents (the builder clears what it needs zeroed); calls whose work overlaps
+ * on the GPU race on it, so order them (one stream, or events). */
+dsa_status dsa_build_indices_static(const dsa_problem* p, const void* Q, const void* K,
+                                    const dsa_pattern* pats, const dsa_indices* out,
+                                    dsa_stream stream);
+
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status s);
 
