@@ -8,19 +8,24 @@
 // (CSR blocks, or qb - delta for the VS distances), plus its listed columns, and
 // for A-shape heads only those with j < sink or i - j < window.
 //
-// Design (one CTA = 128 query rows of one head):
+// Design (one CTA = 128 query rows of one head, two CTAs per SM):
 //   * the tile's two 64-row halves each belong to one query block (two different
-//     blocks when B = 64, the same block otherwise).  Their key lists are turned
-//     into two bitmaps over 64-key units in shared memory; the union is walked
-//     in ascending order, two units (128 keys) per KV tile, and each unit carries
-//     a 2-bit flag saying which half listed it (the other half masks it out);
+//     blocks when B = 64, the same block otherwise).  Their key lists become two
+//     bitmaps over 64-key units in shared memory; the union is walked in
+//     ascending order, two units (128 keys) per KV tile, each unit flagged with
+//     the halves that listed it (the other half masks it out);
 //   * column lists are gathered into dense 128-key tiles (gather-and-densify);
-//   * warp 0 issues TMA loads of K/V units (SWIZZLE_128B boxes of 64x64),
-//     warps 0,2,3 gather column rows, warp 1 issues tcgen05.mma (S = Q K^T into
-//     a double-buffered TMEM tile, O += P V into a TMEM accumulator), warps 4-7
-//     run the online softmax (one thread per row) and the epilogue;
-//   * online softmax keeps a stale running max unless it grows by more than 2^8,
-//     which avoids most O rescales and is exact after the final division.
+//     a column inside a block the half already keeps is masked out;
+//   * warp 0 issues TMA loads (SWIZZLE_128B boxes of 64 x 64), warps 0,2,3 gather
+//     column rows, warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
+//     O += P V with P read straight from TMEM (it overwrites S); warps 4-7 run the
+//     online softmax, one thread per row, and the epilogue;
+//   * each CTA holds 256 TMEM columns and ~100 KB of shared memory, so two CTAs
+//     share an SM and one's softmax overlaps the other's tensor-core work;
+//   * K and V have separate single buffers with their own full/empty barriers:
+//     K of the next tile streams in while this tile's softmax runs;
+//   * the running max is only raised when it grows by more than 2^8, which skips
+//     most O rescales and is exact after the final division.
 // No cluster, no multicast; every wait is bounded (status word + early exit).
 #include <cudaTypedefs.h>
 
@@ -33,17 +38,17 @@ namespace {
 constexpr int BM = 128;          // query rows per CTA
 constexpr int UNIT = 64;         // keys per unit (TMA box rows)
 constexpr int BN = 128;          // keys per KV tile (2 units)
-constexpr int STAGES = 2;
 constexpr int SLAB = 128 * 128;  // bytes of one 128-row x 64-column bf16 slab
 constexpr int NTHREADS = 256;
-constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_COLS = 256;  // O at [0, 128), S / P at [128, 256)
+constexpr uint32_t S_COL = 128;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 struct StageInfo {
-  int type;      // 0 = two units, 1 = column tile
-  int u0, u1;    // unit ids (type 0); u1 = -1 when the second slot is padding
+  int type;            // 0 = two units, 1 = column tile
+  int u0, u1;          // unit ids (type 0); u1 = -1 when the second slot is padding
   int flags0, flags1;  // half bits for u0/u1 (type 0) or the column tile (flags0)
-  int ncols;     // valid columns (type 1)
+  int ncols;           // valid columns (type 1)
   int pad[2];
 };
 
@@ -72,20 +77,21 @@ struct Smem {
   static constexpr int DS = D / 64;  // 64-column slabs
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + DS * SLAB;
-  static constexpr int V_OFF = K_OFF + STAGES * DS * SLAB;
-  static constexpr int P_OFF = V_OFF + STAGES * DS * SLAB;
-  static constexpr int COL_OFF = P_OFF + 2 * SLAB;
-  static constexpr int INFO_OFF = COL_OFF + STAGES * BN * 4;
-  static constexpr int BAR_OFF = INFO_OFF + STAGES * (int)sizeof(StageInfo);
-  static constexpr int NBAR = 16;
+  static constexpr int V_OFF = K_OFF + DS * SLAB;
+  static constexpr int COL_OFF = V_OFF + DS * SLAB;           // int [2][BN]
+  static constexpr int INFO_OFF = COL_OFF + 2 * BN * 4;       // StageInfo [2]
+  static constexpr int BAR_OFF = INFO_OFF + 2 * (int)sizeof(StageInfo);
+  static constexpr int NBAR = 12;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BITS_OFF = MISC_OFF + 64;
   static int bytes(int nwords) { return BITS_OFF + 2 * nwords * 4 + 1024; }
 };
 
 // barrier slots
-enum { B_QFULL = 0, B_KFULL = 1, B_VFULL = 3, B_EMPTY = 5, B_SFULL = 7, B_SFREE = 9, B_PFULL = 11,
-       B_ODONE = 12, B_DRAIN = 13 };
+// B_INFO + (t & 1): the tile's StageInfo (and column list) is written; it
+// completes once per two tiles, and a slot is rewritten only after the softmax
+// has finished with it (the next K load needs the previous P.V to be done).
+enum { B_QFULL = 0, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_ODONE, B_DRAIN, B_INFO };
 
 // One lane waits, the whole warp learns the outcome (keeps warp-collective
 // tcgen05 and shuffle instructions converged even when a wait runs out).
@@ -102,8 +108,38 @@ __device__ __forceinline__ uint32_t swz(int row, int chunk) {  // byte offset in
   return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
 }
 
+__device__ __forceinline__ float fast_ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
+  return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
+}
+
+// O[tmem] (+)= P[tmem] * V[smem desc]: A operand read from tensor memory.
+__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]),
+      "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15])
+      : "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   using L = Smem<D>;
@@ -112,13 +148,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
   int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
-  // misc: [0] tmem base, [1] T total tiles, [2] abort, [3] unit count, [4] col count half0,
-  //       [5] col count half1, [6] col base half0, [7] col base half1, [8] shared-list flag
+  // misc: [0] tmem base, [2] abort, [3] unit count, [4] col count half0, [5] col count half1,
+  //       [6] col base half0, [7] col base half1, [8] shared-list flag, [9] loader go flag
   volatile int* abort_flag = misc + 2;
   uint32_t* bits0 = reinterpret_cast<uint32_t*>(sm + L::BITS_OFF);
   uint32_t* bits1 = bits0 + a.nwords;
   StageInfo* info = reinterpret_cast<StageInfo*>(sm + L::INFO_OFF);
   int* colsm = reinterpret_cast<int*>(sm + L::COL_OFF);
+  uint8_t* ksm = sm + L::K_OFF;
+  uint8_t* vsm = sm + L::V_OFF;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -134,8 +172,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(&bars[i], (i == B_SFREE || i == B_SFREE + 1 || i == B_PFULL) ? 4u : 1u);
+    for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], i == B_PFULL ? 4u : 1u);
     fence_barrier_init();
     misc[2] = 0;
     misc[3] = 0;
@@ -216,7 +253,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   __syncthreads();
   const int n_units = misc[3];
   const int T_u = (n_units + 1) >> 1;
-  const int ccount[2] = {misc[4], misc[5]};
+  const int ccount[2] = {max(0, misc[4]), max(0, misc[5])};
   const int cbase[2] = {misc[6], misc[7]};
   const int cflags[2] = {misc[8] ? 3 : 1, 2};
   const int T_c0 = ceil_div(ccount[0], BN), T_c1 = ceil_div(ccount[1], BN);
@@ -224,17 +261,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const uint32_t tmem_base = static_cast<uint32_t>(misc[0]);
   const uint32_t tmem_O = tmem_base;
-  const uint32_t q_addr = smem_u32(sm + L::Q_OFF);
+  const uint32_t tmem_S = tmem_base + S_COL;
   const uint64_t limit = a.wait_limit_ns;
 
   if (warp == 0 || warp == 2 || warp == 3) {
     // ------------------------------------------------------------ loaders
     const int ltid = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
     if (warp == 0 && lane == 0) {
-      // Q tile
       mbar_arrive_expect_tx(&bars[B_QFULL], DS * SLAB);
       for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * SLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
-      // unit tiles
       int w = 0;
       uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
       auto next_unit = [&](int& fl) -> int {
@@ -248,30 +283,30 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         return w * 32 + b;
       };
       for (int t = 0; t < T_u; ++t) {
-        const int st = t % STAGES;
-        if (!mbar_wait(&bars[B_EMPTY + st], ((t / STAGES) & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
+        if (!mbar_wait(&bars[B_KEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
         int f0 = 0, f1 = 0;
         const int u0 = next_unit(f0);
         int u1 = next_unit(f1);
         if (u1 < 0) f1 = 0;
-        info[st].type = 0;
-        info[st].u0 = u0;
-        info[st].u1 = u1;
-        info[st].flags0 = f0;
-        info[st].flags1 = f1;
-        info[st].ncols = 0;
+        StageInfo& si = info[t & 1];
+        si.type = 0;
+        si.u0 = u0;
+        si.u1 = u1;
+        si.flags0 = f0;
+        si.flags1 = f1;
+        si.ncols = 0;
+        mbar_arrive(&bars[B_INFO + (t & 1)]);
         const int ul = (u1 < 0) ? u0 : u1;
-        uint8_t* kst = sm + L::K_OFF + st * DS * SLAB;
-        uint8_t* vst = sm + L::V_OFF + st * DS * SLAB;
-        mbar_arrive_expect_tx(&bars[B_KFULL + st], DS * SLAB);
+        mbar_arrive_expect_tx(&bars[B_KFULL], DS * SLAB);
         for (int c = 0; c < DS; ++c) {
-          tma_load_3d(kst + c * SLAB, &tmK, &bars[B_KFULL + st], c * 64, u0 * UNIT, kvh);
-          tma_load_3d(kst + c * SLAB + SLAB / 2, &tmK, &bars[B_KFULL + st], c * 64, ul * UNIT, kvh);
+          tma_load_3d(ksm + c * SLAB, &tmK, &bars[B_KFULL], c * 64, u0 * UNIT, kvh);
+          tma_load_3d(ksm + c * SLAB + SLAB / 2, &tmK, &bars[B_KFULL], c * 64, ul * UNIT, kvh);
         }
-        mbar_arrive_expect_tx(&bars[B_VFULL + st], DS * SLAB);
+        if (!mbar_wait(&bars[B_VEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
+        mbar_arrive_expect_tx(&bars[B_VFULL], DS * SLAB);
         for (int c = 0; c < DS; ++c) {
-          tma_load_3d(vst + c * SLAB, &tmV, &bars[B_VFULL + st], c * 64, u0 * UNIT, kvh);
-          tma_load_3d(vst + c * SLAB + SLAB / 2, &tmV, &bars[B_VFULL + st], c * 64, ul * UNIT, kvh);
+          tma_load_3d(vsm + c * SLAB, &tmV, &bars[B_VFULL], c * 64, u0 * UNIT, kvh);
+          tma_load_3d(vsm + c * SLAB + SLAB / 2, &tmV, &bars[B_VFULL], c * 64, ul * UNIT, kvh);
         }
       }
     }
@@ -282,16 +317,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int hh = 0; go && hh < 2; ++hh) {
       const int nt = hh ? T_c1 : T_c0;
       for (int ct = 0; ct < nt; ++ct, ++t) {
-        const int st = t % STAGES;
-        if (ltid == 0)
-          misc[9] = mbar_wait(&bars[B_EMPTY + st], ((t / STAGES) & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY,
-                              abort_flag) ? 1 : 0;
+        if (ltid == 0) {
+          bool ok = mbar_wait(&bars[B_KEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
+          ok = ok && mbar_wait(&bars[B_VEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
+          misc[9] = ok ? 1 : 0;
+        }
         named_barrier(1, 96);
         if (misc[9] == 0) { go = false; break; }
         const int first = cbase[hh] + ct * BN;
         const int nc = min(BN, ccount[hh] - ct * BN);
-        uint8_t* kst = sm + L::K_OFF + st * DS * SLAB;
-        uint8_t* vst = sm + L::V_OFF + st * DS * SLAB;
+        int* cj = colsm + (t & 1) * BN;
         constexpr int CH = D / 8;  // 16-byte chunks per row
         for (int i = ltid; i < BN * CH; i += 96) {
           const int slot = i / CH;
@@ -310,28 +345,29 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               const int cov = (int)((bits0[u >> 5] >> (u & 31)) & 1u) | ((int)((bits1[u >> 5] >> (u & 31)) & 1u) << 1);
               v = j | (cov << 24);
             }
-            colsm[st * BN + slot] = v;
+            cj[slot] = v;
           }
           const int jr = j < 0 ? 0 : j;
           const uint4 kv = __ldg(reinterpret_cast<const uint4*>(a.K + kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
           const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.V + kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
           const uint32_t off = (ch >> 3) * SLAB + swz(slot, ch & 7);
-          *reinterpret_cast<uint4*>(kst + off) = kv;
-          *reinterpret_cast<uint4*>(vst + off) = vv;
+          *reinterpret_cast<uint4*>(ksm + off) = kv;
+          *reinterpret_cast<uint4*>(vsm + off) = vv;
         }
         fence_proxy_async_smem();
         named_barrier(1, 96);
         if (ltid == 0) {
-          info[st].type = 1;
-          info[st].u0 = -1;
-          info[st].u1 = -1;
-          info[st].flags0 = cflags[hh];
-          info[st].flags1 = 0;
-          info[st].ncols = nc;
-          mbar_arrive(&bars[B_KFULL + st]);
-          mbar_arrive(&bars[B_VFULL + st]);
+          StageInfo& si = info[t & 1];
+          si.type = 1;
+          si.u0 = -1;
+          si.u1 = -1;
+          si.flags0 = cflags[hh];
+          si.flags1 = 0;
+          si.ncols = nc;
+          mbar_arrive(&bars[B_INFO + (t & 1)]);
+          mbar_arrive(&bars[B_KFULL]);
+          mbar_arrive(&bars[B_VFULL]);
         }
-        named_barrier(1, 96);  // misc[9] is reused by the next tile
       }
     }
     __syncwarp();
@@ -340,42 +376,35 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
-      const uint32_t p_addr = smem_u32(sm + L::P_OFF);
+      const uint32_t q_addr = smem_u32(sm + L::Q_OFF);
+      const uint32_t k_addr = smem_u32(ksm);
+      const uint32_t v_addr = smem_u32(vsm);
       bool ok = mbar_wait(&bars[B_QFULL], 0, limit, a.status, DETAIL_WAIT_Q, abort_flag);
-      auto issue_pv = [&](int u) -> bool {
-        const int st = u % STAGES;
-        if (!mbar_wait(&bars[B_PFULL], u & 1, limit, a.status, DETAIL_WAIT_P, abort_flag)) return false;
-        if (!mbar_wait(&bars[B_VFULL + st], (u / STAGES) & 1, limit, a.status, DETAIL_WAIT_V, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sm + L::V_OFF + st * DS * SLAB);
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t ad = smem_desc(p_addr + (kk >> 2) * SLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-          const uint64_t bd = smem_desc(v_addr + kk * 2048, SLAB, 1024, SWZ_128B);
-          tc_mma_f16(tmem_O, ad, bd, IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
-        }
-        tc_commit(&bars[B_ODONE]);
-        tc_commit(&bars[B_EMPTY + st]);
-        return true;
-      };
       for (int t = 0; ok && t < T; ++t) {
-        const int st = t % STAGES;
-        const int b = t & 1;
-        if (!mbar_wait(&bars[B_KFULL + st], (t / STAGES) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) { ok = false; break; }
-        if (t >= 2 && !mbar_wait(&bars[B_SFREE + b], ((t >> 1) & 1) ^ 1, limit, a.status, DETAIL_WAIT_SFREE, abort_flag)) { ok = false; break; }
+        const uint32_t ph = t & 1;
+        if (!mbar_wait(&bars[B_KFULL], ph, limit, a.status, DETAIL_WAIT_K, abort_flag)) break;
+        // P of the previous tile lives where S is about to be written
+        if (t > 0 && !mbar_wait(&bars[B_ODONE], ph ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) break;
         tc_fence_after();
-        const uint32_t k_addr = smem_u32(sm + L::K_OFF + st * DS * SLAB);
-        const uint32_t s_tmem = tmem_base + 128 + 128 * b;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t ad = smem_desc(q_addr + (kk >> 2) * SLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
           const uint64_t bd = smem_desc(k_addr + (kk >> 2) * SLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-          tc_mma_f16(s_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+          tc_mma_f16(tmem_S, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        tc_commit(&bars[B_SFULL + b]);
-        if (t >= 1 && !issue_pv(t - 1)) { ok = false; break; }
+        tc_commit(&bars[B_SFULL]);
+        tc_commit(&bars[B_KEMPTY]);
+        if (!mbar_wait(&bars[B_PFULL], ph, limit, a.status, DETAIL_WAIT_P, abort_flag)) break;
+        if (!mbar_wait(&bars[B_VFULL], ph, limit, a.status, DETAIL_WAIT_V, abort_flag)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk) {
+          const uint64_t bd = smem_desc(v_addr + kk * 2048, SLAB, 1024, SWZ_128B);
+          tc_mma_ts(tmem_O, tmem_S + kk * 8, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+        }
+        tc_commit(&bars[B_ODONE]);
+        tc_commit(&bars[B_VEMPTY]);
       }
-      if (ok && T > 0) issue_pv(T - 1);
       // drain every MMA this thread issued before TMEM is released
       tc_commit(&bars[B_DRAIN]);
       mbar_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag);
@@ -387,73 +416,76 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     const int q4 = warp & 3;          // TMEM lane quadrant of this warp
     const int row = row0 + r;
     const int half = r >> 6;
+    const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    uint8_t* p_sm = sm + L::P_OFF;
+    const uint32_t s_t = tmem_S + lane_off;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    float s[BN];
     for (int t = 0; t < T; ++t) {
-      const int st = t % STAGES;
-      const int b = t & 1;
-      if (!warp_wait(&bars[B_KFULL + st], (t / STAGES) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) { ok = false; break; }
-      const StageInfo si = info[st];
-      if (!warp_wait(&bars[B_SFULL + b], (t >> 1) & 1, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t s_tmem = tmem_base + lane_off + 128 + 128 * b;
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(s_tmem + c * 32, s + c * 32);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_SFREE + b]);
-      // masks
-      const int hbit = 1 << half;
-      float mt = -INFINITY;
+      const uint32_t ph = t & 1;
+      if (!warp_wait(&bars[B_INFO + (t & 1)], (t >> 1) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
+        ok = false;
+        break;
+      }
+      const StageInfo si = info[t & 1];
+      // allowed-key bits of this row, 32 columns per word
+      uint32_t mw[4];
       if (si.type == 0) {
         const bool ok0 = (si.flags0 & hbit) != 0;
         const bool ok1 = (si.u1 >= 0) && ((si.flags1 & hbit) != 0);
-        const int k0 = si.u0 * UNIT, k1 = si.u1 * UNIT;
-        const bool full = ok0 && ok1 && (max(k0, k1) + UNIT - 1 <= row) && kind != DSA_KIND_ASHAPE;
-        if (full) {
 #pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            s[c] *= a.scale_log2;
-            mt = fmaxf(mt, s[c]);
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < BN; ++c) {
-            const int j = (c < UNIT) ? (k0 + c) : (k1 + c - UNIT);
-            bool al = (c < UNIT) ? ok0 : ok1;
-            al = al && (j <= row);
-            if (kind == DSA_KIND_ASHAPE) al = al && (j < sink || row - j < window);
-            s[c] = al ? s[c] * a.scale_log2 : -INFINITY;
-            mt = fmaxf(mt, s[c]);
-          }
+        for (int c = 0; c < 4; ++c) {
+          const bool oks = (c < 2) ? ok0 : ok1;
+          const int j0 = ((c < 2) ? si.u0 : si.u1) * UNIT + (c & 1) * 32;
+          uint32_t bits = oks ? low_bits(row - j0 + 1) : 0u;
+          if (kind == DSA_KIND_ASHAPE) bits &= low_bits(sink - j0) | ~low_bits(row - window + 1 - j0);
+          mw[c] = bits;
         }
       } else {
+        const int* cj = colsm + (t & 1) * BN;
         const bool okh = (si.flags0 & hbit) != 0;
-        const int* cj = colsm + st * BN;
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int v = cj[c];
-          const int j = v & 0xFFFFFF;
-          const bool al = okh && (c < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) && (j <= row);
-          s[c] = al ? s[c] * a.scale_log2 : -INFINITY;
-          mt = fmaxf(mt, s[c]);
+        for (int c = 0; c < 4; ++c) {
+          uint32_t bits = 0u;
+#pragma unroll 8
+          for (int i = 0; i < 32; ++i) {
+            const int v = cj[c * 32 + i];
+            const bool al = okh && (c * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
+                            ((v & 0xFFFFFF) <= row);
+            bits |= (al ? 1u : 0u) << i;
+          }
+          mw[c] = bits;
         }
       }
-      const float m_new = fmaxf(m, mt);
+      if (!warp_wait(&bars[B_SFULL], ph, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      // pass 1: tile max of the allowed raw scores
+      float mt = -INFINITY;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float s[32];
+        tmem_ld32(s_t + c * 32, s);
+        tmem_wait_ld();
+        const uint32_t bits = mw[c];
+        if (bits == 0xffffffffu) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, s[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, ((bits >> i) & 1u) ? s[i] : -INFINITY);
+        }
+      }
+      const float m_new = fmaxf(m, mt * a.scale_log2);
       const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
       float alpha = 1.f;
       if (need) {
-        alpha = exp2f(m - m_new);
+        alpha = fast_ex2(m - m_new);
         l *= alpha;
         m = m_new;
       }
       if (t > 0) {
-        // P.V of the previous tile must be done before O is rescaled or P is overwritten
-        if (!warp_wait(&bars[B_ODONE], (t - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
+        // P.V of the previous tile must be done before O is rescaled
+        if (!warp_wait(&bars[B_ODONE], ph ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
           const uint32_t o_t = tmem_O + lane_off;
@@ -466,28 +498,31 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             for (int i = 0; i < 32; ++i) o[i] *= alpha;
             tmem_st32(o_t + c * 32, o);
           }
-          tmem_wait_st();
         }
       }
-      // P = exp2(s - m), rounded to bf16, into the swizzled K-major P tile
-      float lsum = 0.f;
+      // pass 2: P = exp2(s * scale - m) as bf16 pairs, written over S
       const bool dead = (m == -INFINITY);
+      const float negm = dead ? 0.f : -m;
+      float lsum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float s[32];
+        tmem_ld32(s_t + c * 32, s);
+        tmem_wait_ld();
+        const uint32_t bits = dead ? 0u : mw[c];
+        uint32_t pk[16];
 #pragma unroll
-      for (int c8 = 0; c8 < BN / 8; ++c8) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float p0 = dead ? 0.f : exp2f(s[c8 * 8 + 2 * i] - m);
-          const float p1 = dead ? 0.f : exp2f(s[c8 * 8 + 2 * i + 1] - m);
+        for (int i = 0; i < 16; ++i) {
+          const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(fmaf(s[2 * i], a.scale_log2, negm)) : 0.f;
+          const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(fmaf(s[2 * i + 1], a.scale_log2, negm)) : 0.f;
           lsum += p0 + p1;
           __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        const uint32_t off = (c8 >> 3) * SLAB + swz(r, c8 & 7);
-        *reinterpret_cast<uint4*>(p_sm + off) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st16(s_t + c * 16, pk);
       }
       l += lsum;
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PFULL]);
@@ -606,7 +641,8 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   a.status = status;
   a.wait_limit_ns = kWaitLimitNs;
   int smem = Smem<D>::bytes(a.nwords);
-  if (smem < 120 * 1024) smem = 120 * 1024;  // one CTA per SM: each CTA holds 512 TMEM columns
+  // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
+  if (smem < 80 * 1024) smem = 80 * 1024;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = a.n_qtiles * p.Hq;
