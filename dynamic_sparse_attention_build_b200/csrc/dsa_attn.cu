@@ -18,8 +18,9 @@
 //     a column inside a block the half already keeps is masked out;
 //   * warp 0 issues TMA loads (SWIZZLE_128B boxes of 64 x 64), warps 0,2,3 gather
 //     column rows, warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
-//     O += P V with P read straight from TMEM (it overwrites S); warps 4-7 run the
-//     online softmax, one thread per row, and the epilogue;
+//     O += P V with P read straight from TMEM (it overwrites S); warps 4-11 run
+//     the online softmax, two threads per row (64 key columns each), and the
+//     epilogue;
 //   * each CTA holds 256 TMEM columns and ~100 KB of shared memory, so two CTAs
 //     share an SM and one's softmax overlaps the other's tensor-core work;
 //   * K and V have separate single buffers with their own full/empty barriers:
@@ -39,7 +40,7 @@ constexpr int BM = 128;          // query rows per CTA
 constexpr int UNIT = 64;         // keys per unit (TMA box rows)
 constexpr int BN = 128;          // keys per KV tile (2 units)
 constexpr int SLAB = 128 * 128;  // bytes of one 128-row x 64-column bf16 slab
-constexpr int NTHREADS = 256;
+constexpr int NTHREADS = 384;  // warps 0,2,3 load, warp 1 issues MMAs, warps 4-11 softmax
 constexpr uint32_t TMEM_COLS = 256;  // O at [0, 128), S / P at [128, 256)
 constexpr uint32_t S_COL = 128;
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
@@ -81,9 +82,10 @@ struct Smem {
   static constexpr int COL_OFF = V_OFF + DS * SLAB;           // int [2][BN]
   static constexpr int INFO_OFF = COL_OFF + 2 * BN * 4;       // StageInfo [2]
   static constexpr int BAR_OFF = INFO_OFF + 2 * (int)sizeof(StageInfo);
-  static constexpr int NBAR = 12;
+  static constexpr int NBAR = 16;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int BITS_OFF = MISC_OFF + 64;
+  static constexpr int RED_OFF = MISC_OFF + 64;                // float [2][2][BM] maxima, [2][BM] sums
+  static constexpr int BITS_OFF = RED_OFF + 6 * BM * 4;
   static int bytes(int nwords) { return BITS_OFF + 2 * nwords * 4 + 1024; }
 };
 
@@ -91,7 +93,9 @@ struct Smem {
 // B_INFO + (t & 1): the tile's StageInfo (and column list) is written; it
 // completes once per two tiles, and a slot is rewritten only after the softmax
 // has finished with it (the next K load needs the previous P.V to be done).
-enum { B_QFULL = 0, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_ODONE, B_DRAIN, B_INFO };
+// B_PMAX + (t & 1): both halves of every row have posted their partial max.
+enum { B_QFULL = 0, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_ODONE, B_DRAIN, B_INFO,
+       B_PMAX = B_INFO + 2, B_LSUM = B_PMAX + 2 };
 
 // One lane waits, the whole warp learns the outcome (keeps warp-collective
 // tcgen05 and shuffle instructions converged even when a wait runs out).
@@ -112,6 +116,16 @@ __device__ __forceinline__ float fast_ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// (x0, x1) = (a0, a1) * b + c with one packed f32x2 fused multiply-add
+__device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float& x0, float& x1) {
+  uint64_t av, bv, cv, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a0), "f"(a1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(bv) : "f"(b), "f"(b));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(cv) : "f"(c), "f"(c));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(bv), "l"(cv));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(r));
 }
 
 __device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
@@ -172,7 +186,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], i == B_PFULL ? 4u : 1u);
+    for (int i = 0; i < L::NBAR; ++i)
+      mbar_init(&bars[i], (i == B_PFULL || i == B_PMAX || i == B_PMAX + 1 || i == B_LSUM) ? 8u : 1u);
     fence_barrier_init();
     misc[2] = 0;
     misc[3] = 0;
@@ -400,7 +415,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk) {
           const uint64_t bd = smem_desc(v_addr + kk * 2048, SLAB, 1024, SWZ_128B);
-          tc_mma_ts(tmem_O, tmem_S + kk * 8, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          // P of keys 0-63 sits in S columns 0-31, of keys 64-127 in columns 64-95
+          tc_mma_ts(tmem_O, tmem_S + (kk >> 2) * 64 + (kk & 3) * 8, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
         }
         tc_commit(&bars[B_ODONE]);
         tc_commit(&bars[B_VEMPTY]);
@@ -412,13 +428,22 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int r = tid - 128;          // row within the tile == TMEM lane
-    const int q4 = warp & 3;          // TMEM lane quadrant of this warp
+    // Warps 4..11, two threads per row: ch selects the 64 key columns of the tile
+    // (and the half of O's columns) this thread owns.  The two halves agree on the
+    // row max through shared memory before any exponent is taken, so every P of a
+    // row uses the same running max.
+    const int q4 = warp & 3;           // TMEM lane quadrant of this warp
+    const int ch = (warp - 4) >> 2;    // column half
+    const int r = q4 * 32 + lane;      // row within the tile == TMEM lane
     const int row = row0 + r;
     const int half = r >> 6;
     const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t s_t = tmem_S + lane_off;
+    const uint32_t s_t = tmem_S + lane_off + ch * 64;  // this thread's 64 score columns
+    float* pmax = reinterpret_cast<float*>(sm + L::RED_OFF);  // [2 tiles][2 halves][BM rows]
+    float* lpart = pmax + 4 * BM;                              // [2 halves][BM rows]
+    constexpr int OC = D / 2;                                  // O columns per thread
+    const uint32_t o_t = tmem_O + lane_off + ch * OC;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
@@ -428,53 +453,57 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         break;
       }
       const StageInfo si = info[t & 1];
-      // allowed-key bits of this row, 32 columns per word
-      uint32_t mw[4];
+      // allowed-key bits of this thread's 64 columns, 32 per word
+      uint32_t mw[2];
       if (si.type == 0) {
-        const bool ok0 = (si.flags0 & hbit) != 0;
-        const bool ok1 = (si.u1 >= 0) && ((si.flags1 & hbit) != 0);
+        const int u = ch ? si.u1 : si.u0;  // columns 64ch.. are exactly unit slot ch
+        const bool oks = ch ? ((si.u1 >= 0) && (si.flags1 & hbit)) : ((si.flags0 & hbit) != 0);
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const bool oks = (c < 2) ? ok0 : ok1;
-          const int j0 = ((c < 2) ? si.u0 : si.u1) * UNIT + (c & 1) * 32;
+        for (int k = 0; k < 2; ++k) {
+          const int j0 = u * UNIT + k * 32;
           uint32_t bits = oks ? low_bits(row - j0 + 1) : 0u;
           if (kind == DSA_KIND_ASHAPE) bits &= low_bits(sink - j0) | ~low_bits(row - window + 1 - j0);
-          mw[c] = bits;
+          mw[k] = bits;
         }
       } else {
-        const int* cj = colsm + (t & 1) * BN;
+        const int* cj = colsm + (t & 1) * BN + ch * 64;
         const bool okh = (si.flags0 & hbit) != 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int k = 0; k < 2; ++k) {
           uint32_t bits = 0u;
 #pragma unroll 8
           for (int i = 0; i < 32; ++i) {
-            const int v = cj[c * 32 + i];
-            const bool al = okh && (c * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
+            const int v = cj[k * 32 + i];
+            const bool al = okh && (ch * 64 + k * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
                             ((v & 0xFFFFFF) <= row);
             bits |= (al ? 1u : 0u) << i;
           }
-          mw[c] = bits;
+          mw[k] = bits;
         }
       }
       if (!warp_wait(&bars[B_SFULL], ph, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: tile max of the allowed raw scores
-      float mt = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      // pass 1: max of the allowed raw scores over this thread's columns
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
         float s[32];
-        tmem_ld32(s_t + c * 32, s);
+        tmem_ld32(s_t + k * 32, s);
         tmem_wait_ld();
-        const uint32_t bits = mw[c];
-        if (bits == 0xffffffffu) {
+        const uint32_t bits = mw[k];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, s[i]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mt = fmaxf(mt, ((bits >> i) & 1u) ? s[i] : -INFINITY);
-        }
+        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[i] : -INFINITY);
       }
+      float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      // exchange with the other half of the row
+      pmax[((t & 1) * 2 + ch) * BM + r] = mt;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_PMAX + (t & 1)]);
+      if (!warp_wait(&bars[B_PMAX + (t & 1)], (t >> 1) & 1, limit, a.status, DETAIL_WAIT_S, abort_flag)) {
+        ok = false;
+        break;
+      }
+      mt = fmaxf(mt, pmax[((t & 1) * 2 + (ch ^ 1)) * BM + r]);
       const float m_new = fmaxf(m, mt * a.scale_log2);
       const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
       float alpha = 1.f;
@@ -488,9 +517,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!warp_wait(&bars[B_ODONE], ph ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (__any_sync(0xffffffffu, need)) {
-          const uint32_t o_t = tmem_O + lane_off;
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < OC / 32; ++c) {
             float o[32];
             tmem_ld32(o_t + c * 32, o);
             tmem_wait_ld();
@@ -500,46 +528,55 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
       }
-      // pass 2: P = exp2(s * scale - m) as bf16 pairs, written over S
+      // pass 2: P = exp2(s * scale - m) as bf16 pairs, written into the first 32
+      // of this thread's 64 columns (already read), keys 64ch .. 64ch+63
       const bool dead = (m == -INFINITY);
       const float negm = dead ? 0.f : -m;
-      float lsum = 0.f;
-#pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
+      float ls[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
         float s[32];
-        tmem_ld32(s_t + c * 32, s);
+        tmem_ld32(s_t + k * 32, s);
         tmem_wait_ld();
-        const uint32_t bits = dead ? 0u : mw[c];
+        const uint32_t bits = dead ? 0u : mw[k];
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(fmaf(s[2 * i], a.scale_log2, negm)) : 0.f;
-          const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(fmaf(s[2 * i + 1], a.scale_log2, negm)) : 0.f;
-          lsum += p0 + p1;
+          float x0, x1;
+          fma2(s[2 * i], s[2 * i + 1], a.scale_log2, negm, x0, x1);
+          const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(x0) : 0.f;
+          const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(x1) : 0.f;
+          ls[i & 3] += p0 + p1;
           __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
           pk[i] = *reinterpret_cast<uint32_t*>(&v2);
         }
-        tmem_st16(s_t + c * 16, pk);
+        tmem_st16(s_t + k * 16, pk);
       }
-      l += lsum;
+      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[B_PFULL]);
     }
-    // epilogue
+    // epilogue: the two halves of a row add their sums, then each writes its
+    // half of O's columns
     const bool have = ok && T > 0;
     if (have) {
       if (!warp_wait(&bars[B_ODONE], (T - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) ok = false;
       tc_fence_after();
     }
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = a.O + h * a.o_hs + (int64_t)row * a.o_ts;
+    lpart[ch * BM + r] = l;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[B_LSUM]);
+    if (!warp_wait(&bars[B_LSUM], 0, limit, a.status, DETAIL_WAIT_S, abort_flag)) ok = false;
+    const float lt = l + lpart[(ch ^ 1) * BM + r];
+    const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
+    __nv_bfloat16* orow = a.O + h * a.o_hs + (int64_t)row * a.o_ts + ch * OC;
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = 0; c < OC / 32; ++c) {
       float o[32];
       if (have && ok) {
-        tmem_ld32(tmem_O + lane_off + c * 32, o);
+        tmem_ld32(o_t + c * 32, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -558,8 +595,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-    if (a.lse != nullptr && row < a.N)
-      a.lse[(int64_t)h * a.N + row] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+    if (ch == 0 && a.lse != nullptr && row < a.N)
+      a.lse[(int64_t)h * a.N + row] = (lt > 0.f) ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
     __syncwarp();
   }
 
