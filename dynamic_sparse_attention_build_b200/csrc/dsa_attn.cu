@@ -12,21 +12,22 @@
 //   * the tile's two 64-row halves each belong to one query block (two different
 //     blocks when B = 64, the same block otherwise).  Their key lists become two
 //     bitmaps over 64-key units in shared memory; the union is walked in
-//     ascending order, two units (128 keys) per KV tile, each unit flagged with
-//     the halves that listed it (the other half masks it out);
-//   * column lists are gathered into dense 128-key tiles (gather-and-densify);
-//     a column inside a block the half already keeps is masked out;
-//   * warp 0 issues TMA loads (SWIZZLE_128B boxes of 64 x 64), warps 0,2,3 gather
-//     column rows, warp 1 issues tcgen05.mma: S = Q K^T into TMEM, then
-//     O += P V with P read straight from TMEM (it overwrites S); warps 4-11 run
-//     the online softmax, two threads per row (64 key columns each), and the
-//     epilogue;
-//   * each CTA holds 256 TMEM columns and ~100 KB of shared memory, so two CTAs
-//     share an SM and one's softmax overlaps the other's tensor-core work;
-//   * K and V have separate single buffers with their own full/empty barriers:
-//     K of the next tile streams in while this tile's softmax runs;
-//   * the running max is only raised when it grows by more than 2^8, which skips
-//     most O rescales and is exact after the final division.
+//     ascending order, one unit (64 keys) per KV tile, each unit flagged with the
+//     halves that listed it (the other half masks it out);
+//   * column lists are gathered into dense 64-key tiles (gather-and-densify); a
+//     column inside a block the half already keeps is masked out;
+//   * warp 0 issues TMA loads (SWIZZLE_128B boxes of 64 x 64) into two K and two V
+//     buffers, warps 0,2,3 gather column rows, warp 1 issues tcgen05.mma, warps
+//     4-7 run the online softmax (one thread per row) and the epilogue;
+//   * TMEM (256 columns per CTA): O at [0, 128), two S buffers of 64 columns at
+//     128 and 192.  S(t+1) = Q K(t+1)^T is computed while the softmax works on
+//     S(t); the softmax writes P(t) as bf16 pairs over the first 32 columns of its
+//     S buffer and O += P(t) V(t) reads it from there;
+//   * the running max is only raised when it grows by more than 2^8; only then
+//     does the softmax wait for the previous P.V and rescale O, so in the common
+//     case the softmax of one tile overlaps the P.V of the one before;
+//   * ~100 KB of shared memory and 256 TMEM columns per CTA let two CTAs share an
+//     SM, so one CTA's softmax also overlaps the other's tensor-core work.
 // No cluster, no multicast; every wait is bounded (status word + early exit).
 #include <cudaTypedefs.h>
 
@@ -36,21 +37,22 @@
 namespace dsa {
 namespace {
 
-constexpr int BM = 128;          // query rows per CTA
-constexpr int UNIT = 64;         // keys per unit (TMA box rows)
-constexpr int BN = 128;          // keys per KV tile (2 units)
-constexpr int SLAB = 128 * 128;  // bytes of one 128-row x 64-column bf16 slab
-constexpr int NTHREADS = 384;  // warps 0,2,3 load, warp 1 issues MMAs, warps 4-11 softmax
-constexpr uint32_t TMEM_COLS = 256;  // O at [0, 128), S / P at [128, 256)
-constexpr uint32_t S_COL = 128;
+constexpr int BM = 128;            // query rows per CTA
+constexpr int UNIT = 64;           // keys per KV tile (one TMA box of rows)
+constexpr int BN = UNIT;
+constexpr int QSLAB = 128 * 128;   // bytes of one 128-row x 64-column bf16 slab (Q)
+constexpr int KSLAB = 64 * 128;    // bytes of one 64-row x 64-column bf16 slab (K, V)
+constexpr int NTHREADS = 256;      // warps 0,2,3 load, warp 1 issues MMAs, warps 4-7 softmax
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t S_COL = 128;    // S buffer b at S_COL + 64 b
+constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after its softmax ended)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 
 struct StageInfo {
-  int type;            // 0 = two units, 1 = column tile
-  int u0, u1;          // unit ids (type 0); u1 = -1 when the second slot is padding
-  int flags0, flags1;  // half bits for u0/u1 (type 0) or the column tile (flags0)
-  int ncols;           // valid columns (type 1)
-  int pad[2];
+  int type;   // 0 = key unit, 1 = column tile
+  int u;      // unit id (type 0)
+  int flags;  // bit h: half h of the rows uses this tile
+  int ncols;  // valid columns (type 1)
 };
 
 struct AttnArgs {
@@ -77,25 +79,32 @@ template <int D>
 struct Smem {
   static constexpr int DS = D / 64;  // 64-column slabs
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + DS * SLAB;
-  static constexpr int V_OFF = K_OFF + DS * SLAB;
-  static constexpr int COL_OFF = V_OFF + DS * SLAB;           // int [2][BN]
-  static constexpr int INFO_OFF = COL_OFF + 2 * BN * 4;       // StageInfo [2]
-  static constexpr int BAR_OFF = INFO_OFF + 2 * (int)sizeof(StageInfo);
-  static constexpr int NBAR = 16;
+  static constexpr int K_OFF = Q_OFF + DS * QSLAB;         // [2 buffers][DS slabs]
+  static constexpr int V_OFF = K_OFF + 2 * DS * KSLAB;
+  static constexpr int COL_OFF = V_OFF + 2 * DS * KSLAB;   // int [NINFO][BN]
+  static constexpr int INFO_OFF = COL_OFF + NINFO * BN * 4;
+  static constexpr int BAR_OFF = INFO_OFF + NINFO * (int)sizeof(StageInfo);
+  static constexpr int NBAR = 20;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int RED_OFF = MISC_OFF + 64;                // float [2][2][BM] maxima, [2][BM] sums
-  static constexpr int BITS_OFF = RED_OFF + 6 * BM * 4;
+  static constexpr int BITS_OFF = MISC_OFF + 64;
   static int bytes(int nwords) { return BITS_OFF + 2 * nwords * 4 + 1024; }
 };
 
-// barrier slots
-// B_INFO + (t & 1): the tile's StageInfo (and column list) is written; it
-// completes once per two tiles, and a slot is rewritten only after the softmax
-// has finished with it (the next K load needs the previous P.V to be done).
-// B_PMAX + (t & 1): both halves of every row have posted their partial max.
-enum { B_QFULL = 0, B_KFULL, B_KEMPTY, B_VFULL, B_VEMPTY, B_SFULL, B_PFULL, B_ODONE, B_DRAIN, B_INFO,
-       B_PMAX = B_INFO + 2, B_LSUM = B_PMAX + 2 };
+// Barrier slots.  Per-buffer barriers (K, V, S, P) complete once per use of their
+// buffer, i.e. once per two tiles; B_ODONE completes once per P.V in order.
+// B_INFO + s completes when StageInfo slot s (and its column list) is written.
+enum {
+  B_QFULL = 0,
+  B_KFULL = 1,    // +2
+  B_KEMPTY = 3,   // +2
+  B_VFULL = 5,    // +2
+  B_VEMPTY = 7,   // +2
+  B_SFULL = 9,    // +2
+  B_PFULL = 11,   // +2
+  B_ODONE = 13,
+  B_DRAIN = 14,
+  B_INFO = 15     // +NINFO
+};
 
 // One lane waits, the whole warp learns the outcome (keeps warp-collective
 // tcgen05 and shuffle instructions converged even when a wait runs out).
@@ -169,8 +178,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint32_t* bits1 = bits0 + a.nwords;
   StageInfo* info = reinterpret_cast<StageInfo*>(sm + L::INFO_OFF);
   int* colsm = reinterpret_cast<int*>(sm + L::COL_OFF);
-  uint8_t* ksm = sm + L::K_OFF;
-  uint8_t* vsm = sm + L::V_OFF;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -186,8 +193,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   // ---------------------------------------------------------------- set-up
   if (tid == 0) {
-    for (int i = 0; i < L::NBAR; ++i)
-      mbar_init(&bars[i], (i == B_PFULL || i == B_PMAX || i == B_PMAX + 1 || i == B_LSUM) ? 8u : 1u);
+    for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1) ? 4u : 1u);
     fence_barrier_init();
     misc[2] = 0;
     misc[3] = 0;
@@ -266,8 +272,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     misc[4] = c0; misc[5] = c1; misc[6] = b0; misc[7] = b1; misc[8] = shared_qb ? 1 : 0;
   }
   __syncthreads();
-  const int n_units = misc[3];
-  const int T_u = (n_units + 1) >> 1;
+  const int T_u = misc[3];  // one tile per unit
   const int ccount[2] = {max(0, misc[4]), max(0, misc[5])};
   const int cbase[2] = {misc[6], misc[7]};
   const int cflags[2] = {misc[8] ? 3 : 1, 2};
@@ -276,53 +281,40 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 
   const uint32_t tmem_base = static_cast<uint32_t>(misc[0]);
   const uint32_t tmem_O = tmem_base;
-  const uint32_t tmem_S = tmem_base + S_COL;
   const uint64_t limit = a.wait_limit_ns;
 
   if (warp == 0 || warp == 2 || warp == 3) {
     // ------------------------------------------------------------ loaders
     const int ltid = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
     if (warp == 0 && lane == 0) {
-      mbar_arrive_expect_tx(&bars[B_QFULL], DS * SLAB);
-      for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * SLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
+      mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
+      for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
       int w = 0;
       uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
-      auto next_unit = [&](int& fl) -> int {
-        while (pend == 0u) {
-          if (++w >= a.nwords) return -1;
+      for (int t = 0; t < T_u; ++t) {
+        const int b = t & 1;
+        const uint32_t use = (t >> 1) & 1;
+        if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
+        while (pend == 0u && w + 1 < a.nwords) {
+          ++w;
           pend = bits0[w] | bits1[w];
         }
-        const int b = __ffs(pend) - 1;
+        const int bit = __ffs(pend) - 1;  // T_u counts exactly the set bits
         pend &= pend - 1u;
-        fl = (int)((bits0[w] >> b) & 1u) | ((int)((bits1[w] >> b) & 1u) << 1);
-        return w * 32 + b;
-      };
-      for (int t = 0; t < T_u; ++t) {
-        if (!mbar_wait(&bars[B_KEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
-        int f0 = 0, f1 = 0;
-        const int u0 = next_unit(f0);
-        int u1 = next_unit(f1);
-        if (u1 < 0) f1 = 0;
-        StageInfo& si = info[t & 1];
+        const int u = w * 32 + bit;
+        StageInfo& si = info[t % NINFO];
         si.type = 0;
-        si.u0 = u0;
-        si.u1 = u1;
-        si.flags0 = f0;
-        si.flags1 = f1;
+        si.u = u;
+        si.flags = (int)((bits0[w] >> bit) & 1u) | ((int)((bits1[w] >> bit) & 1u) << 1);
         si.ncols = 0;
-        mbar_arrive(&bars[B_INFO + (t & 1)]);
-        const int ul = (u1 < 0) ? u0 : u1;
-        mbar_arrive_expect_tx(&bars[B_KFULL], DS * SLAB);
-        for (int c = 0; c < DS; ++c) {
-          tma_load_3d(ksm + c * SLAB, &tmK, &bars[B_KFULL], c * 64, u0 * UNIT, kvh);
-          tma_load_3d(ksm + c * SLAB + SLAB / 2, &tmK, &bars[B_KFULL], c * 64, ul * UNIT, kvh);
-        }
-        if (!mbar_wait(&bars[B_VEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[B_VFULL], DS * SLAB);
-        for (int c = 0; c < DS; ++c) {
-          tma_load_3d(vsm + c * SLAB, &tmV, &bars[B_VFULL], c * 64, u0 * UNIT, kvh);
-          tma_load_3d(vsm + c * SLAB + SLAB / 2, &tmV, &bars[B_VFULL], c * 64, ul * UNIT, kvh);
-        }
+        mbar_arrive(&bars[B_INFO + t % NINFO]);
+        uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+        uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
+        mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
+        for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, kvh);
+        if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
+        mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
+        for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, kvh);
       }
     }
     __syncwarp();
@@ -332,16 +324,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     for (int hh = 0; go && hh < 2; ++hh) {
       const int nt = hh ? T_c1 : T_c0;
       for (int ct = 0; ct < nt; ++ct, ++t) {
+        const int b = t & 1;
+        const uint32_t use = (t >> 1) & 1;
         if (ltid == 0) {
-          bool ok = mbar_wait(&bars[B_KEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
-          ok = ok && mbar_wait(&bars[B_VEMPTY], (t & 1) ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
+          bool ok = mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
+          ok = ok && mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
           misc[9] = ok ? 1 : 0;
         }
         named_barrier(1, 96);
         if (misc[9] == 0) { go = false; break; }
         const int first = cbase[hh] + ct * BN;
         const int nc = min(BN, ccount[hh] - ct * BN);
-        int* cj = colsm + (t & 1) * BN;
+        int* cj = colsm + (t % NINFO) * BN;
+        uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+        uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
         constexpr int CH = D / 8;  // 16-byte chunks per row
         for (int i = ltid; i < BN * CH; i += 96) {
           const int slot = i / CH;
@@ -365,23 +361,21 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const int jr = j < 0 ? 0 : j;
           const uint4 kv = __ldg(reinterpret_cast<const uint4*>(a.K + kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
           const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.V + kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
-          const uint32_t off = (ch >> 3) * SLAB + swz(slot, ch & 7);
-          *reinterpret_cast<uint4*>(ksm + off) = kv;
-          *reinterpret_cast<uint4*>(vsm + off) = vv;
+          const uint32_t off = (ch >> 3) * KSLAB + swz(slot, ch & 7);
+          *reinterpret_cast<uint4*>(kst + off) = kv;
+          *reinterpret_cast<uint4*>(vst + off) = vv;
         }
         fence_proxy_async_smem();
         named_barrier(1, 96);
         if (ltid == 0) {
-          StageInfo& si = info[t & 1];
+          StageInfo& si = info[t % NINFO];
           si.type = 1;
-          si.u0 = -1;
-          si.u1 = -1;
-          si.flags0 = cflags[hh];
-          si.flags1 = 0;
+          si.u = -1;
+          si.flags = cflags[hh];
           si.ncols = nc;
-          mbar_arrive(&bars[B_INFO + (t & 1)]);
-          mbar_arrive(&bars[B_KFULL]);
-          mbar_arrive(&bars[B_VFULL]);
+          mbar_arrive(&bars[B_INFO + t % NINFO]);
+          mbar_arrive(&bars[B_KFULL + b]);
+          mbar_arrive(&bars[B_VFULL + b]);
         }
       }
     }
@@ -392,34 +386,45 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
       const uint32_t q_addr = smem_u32(sm + L::Q_OFF);
-      const uint32_t k_addr = smem_u32(ksm);
-      const uint32_t v_addr = smem_u32(vsm);
       bool ok = mbar_wait(&bars[B_QFULL], 0, limit, a.status, DETAIL_WAIT_Q, abort_flag);
-      for (int t = 0; ok && t < T; ++t) {
-        const uint32_t ph = t & 1;
-        if (!mbar_wait(&bars[B_KFULL], ph, limit, a.status, DETAIL_WAIT_K, abort_flag)) break;
-        // P of the previous tile lives where S is about to be written
-        if (t > 0 && !mbar_wait(&bars[B_ODONE], ph ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) break;
-        tc_fence_after();
+      for (int t = 0; ok && t <= T; ++t) {
+        if (t < T) {
+          // S(t) = Q K(t)^T into S buffer t & 1
+          const int b = t & 1;
+          const uint32_t use = (t >> 1) & 1;
+          if (!mbar_wait(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag)) break;
+          // the buffer still holds P(t-2) until that P.V has finished
+          if (t >= 2 && !mbar_wait(&bars[B_ODONE], t & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(sm + L::K_OFF + b * DS * KSLAB);
+          const uint32_t s_tmem = tmem_base + S_COL + 64 * b;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc(q_addr + (kk >> 2) * SLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-          const uint64_t bd = smem_desc(k_addr + (kk >> 2) * SLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-          tc_mma_f16(tmem_S, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t ad = smem_desc(q_addr + (kk >> 2) * QSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
+            const uint64_t bd = smem_desc(k_addr + (kk >> 2) * KSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
+            tc_mma_f16(s_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+          }
+          tc_commit(&bars[B_SFULL + b]);
+          tc_commit(&bars[B_KEMPTY + b]);
         }
-        tc_commit(&bars[B_SFULL]);
-        tc_commit(&bars[B_KEMPTY]);
-        if (!mbar_wait(&bars[B_PFULL], ph, limit, a.status, DETAIL_WAIT_P, abort_flag)) break;
-        if (!mbar_wait(&bars[B_VFULL], ph, limit, a.status, DETAIL_WAIT_V, abort_flag)) break;
-        tc_fence_after();
+        if (t >= 1) {
+          // O += P(t-1) V(t-1)
+          const int u = t - 1;
+          const int b = u & 1;
+          const uint32_t use = (u >> 1) & 1;
+          if (!mbar_wait(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag)) break;
+          if (!mbar_wait(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag)) break;
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(sm + L::V_OFF + b * DS * KSLAB);
+          const uint32_t p_tmem = tmem_base + S_COL + 64 * b;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk) {
-          const uint64_t bd = smem_desc(v_addr + kk * 2048, SLAB, 1024, SWZ_128B);
-          // P of keys 0-63 sits in S columns 0-31, of keys 64-127 in columns 64-95
-          tc_mma_ts(tmem_O, tmem_S + (kk >> 2) * 64 + (kk & 3) * 8, bd, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BN / 16; ++kk) {
+            const uint64_t bd = smem_desc(v_addr + kk * 2048, KSLAB, 1024, SWZ_128B);
+            tc_mma_ts(tmem_O, p_tmem + kk * 8, bd, IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(&bars[B_ODONE]);
+          tc_commit(&bars[B_VEMPTY + b]);
         }
-        tc_commit(&bars[B_ODONE]);
-        tc_commit(&bars[B_VEMPTY]);
       }
       // drain every MMA this thread issued before TMEM is released
       tc_commit(&bars[B_DRAIN]);
@@ -428,82 +433,66 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    // Warps 4..11, two threads per row: ch selects the 64 key columns of the tile
-    // (and the half of O's columns) this thread owns.  The two halves agree on the
-    // row max through shared memory before any exponent is taken, so every P of a
-    // row uses the same running max.
     const int q4 = warp & 3;           // TMEM lane quadrant of this warp
-    const int ch = (warp - 4) >> 2;    // column half
     const int r = q4 * 32 + lane;      // row within the tile == TMEM lane
     const int row = row0 + r;
     const int half = r >> 6;
     const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    const uint32_t s_t = tmem_S + lane_off + ch * 64;  // this thread's 64 score columns
-    float* pmax = reinterpret_cast<float*>(sm + L::RED_OFF);  // [2 tiles][2 halves][BM rows]
-    float* lpart = pmax + 4 * BM;                              // [2 halves][BM rows]
-    constexpr int OC = D / 2;                                  // O columns per thread
-    const uint32_t o_t = tmem_O + lane_off + ch * OC;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int t = 0; t < T; ++t) {
-      const uint32_t ph = t & 1;
-      if (!warp_wait(&bars[B_INFO + (t & 1)], (t >> 1) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
+      const int b = t & 1;
+      const uint32_t use = (t >> 1) & 1;
+      const int slot = t % NINFO;
+      if (!warp_wait(&bars[B_INFO + slot], (t / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
         ok = false;
         break;
       }
-      const StageInfo si = info[t & 1];
-      // allowed-key bits of this thread's 64 columns, 32 per word
+      const StageInfo si = info[slot];
+      // allowed-key bits of this row, 32 columns per word
       uint32_t mw[2];
       if (si.type == 0) {
-        const int u = ch ? si.u1 : si.u0;  // columns 64ch.. are exactly unit slot ch
-        const bool oks = ch ? ((si.u1 >= 0) && (si.flags1 & hbit)) : ((si.flags0 & hbit) != 0);
+        const bool oks = (si.flags & hbit) != 0;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
-          const int j0 = u * UNIT + k * 32;
+          const int j0 = si.u * UNIT + k * 32;
           uint32_t bits = oks ? low_bits(row - j0 + 1) : 0u;
           if (kind == DSA_KIND_ASHAPE) bits &= low_bits(sink - j0) | ~low_bits(row - window + 1 - j0);
           mw[k] = bits;
         }
       } else {
-        const int* cj = colsm + (t & 1) * BN + ch * 64;
-        const bool okh = (si.flags0 & hbit) != 0;
+        const int* cj = colsm + slot * BN;
+        const bool okh = (si.flags & hbit) != 0;
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           uint32_t bits = 0u;
 #pragma unroll 8
           for (int i = 0; i < 32; ++i) {
             const int v = cj[k * 32 + i];
-            const bool al = okh && (ch * 64 + k * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
+            const bool al = okh && (k * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
                             ((v & 0xFFFFFF) <= row);
             bits |= (al ? 1u : 0u) << i;
           }
           mw[k] = bits;
         }
       }
-      if (!warp_wait(&bars[B_SFULL], ph, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
+      if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      // pass 1: max of the allowed raw scores over this thread's columns
+      const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
+      float s[64];
+      tmem_ld32(s_t, s);
+      tmem_ld32(s_t + 32, s + 32);
+      tmem_wait_ld();
+      // tile max of the allowed raw scores (independent partial maxima)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        float s[32];
-        tmem_ld32(s_t + k * 32, s);
-        tmem_wait_ld();
         const uint32_t bits = mw[k];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[i] : -INFINITY);
+        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[k * 32 + i] : -INFINITY);
       }
-      float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      // exchange with the other half of the row
-      pmax[((t & 1) * 2 + ch) * BM + r] = mt;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PMAX + (t & 1)]);
-      if (!warp_wait(&bars[B_PMAX + (t & 1)], (t >> 1) & 1, limit, a.status, DETAIL_WAIT_S, abort_flag)) {
-        ok = false;
-        break;
-      }
-      mt = fmaxf(mt, pmax[((t & 1) * 2 + (ch ^ 1)) * BM + r]);
+      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m, mt * a.scale_log2);
       const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
       float alpha = 1.f;
@@ -512,38 +501,33 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         l *= alpha;
         m = m_new;
       }
-      if (t > 0) {
-        // P.V of the previous tile must be done before O is rescaled
-        if (!warp_wait(&bars[B_ODONE], ph ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
+      if (t > 0 && __any_sync(0xffffffffu, need)) {
+        // O must hold every P.V so far before it is rescaled: wait for P(t-1) V(t-1)
+        if (!warp_wait(&bars[B_ODONE], (t - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, need)) {
+        const uint32_t o_t = tmem_O + lane_off;
 #pragma unroll 1
-          for (int c = 0; c < OC / 32; ++c) {
-            float o[32];
-            tmem_ld32(o_t + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          float o[32];
+          tmem_ld32(o_t + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] *= alpha;
-            tmem_st32(o_t + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] *= alpha;
+          tmem_st32(o_t + c * 32, o);
         }
       }
-      // pass 2: P = exp2(s * scale - m) as bf16 pairs, written into the first 32
-      // of this thread's 64 columns (already read), keys 64ch .. 64ch+63
+      // P = exp2(s * scale - m) as bf16 pairs over the first 32 columns of the buffer
       const bool dead = (m == -INFINITY);
       const float negm = dead ? 0.f : -m;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int k = 0; k < 2; ++k) {
-        float s[32];
-        tmem_ld32(s_t + k * 32, s);
-        tmem_wait_ld();
         const uint32_t bits = dead ? 0u : mw[k];
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           float x0, x1;
-          fma2(s[2 * i], s[2 * i + 1], a.scale_log2, negm, x0, x1);
+          fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
           const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(x0) : 0.f;
           const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(x1) : 0.f;
           ls[i & 3] += p0 + p1;
@@ -556,27 +540,23 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PFULL]);
+      if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
     }
-    // epilogue: the two halves of a row add their sums, then each writes its
-    // half of O's columns
+    // epilogue.  The softmax does not follow every P.V, so the P.V-done barrier
+    // may be a phase behind here; the drain barrier, committed by the MMA thread
+    // after its last MMA, is the one that says O is final.
     const bool have = ok && T > 0;
     if (have) {
-      if (!warp_wait(&bars[B_ODONE], (T - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) ok = false;
+      if (!warp_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag)) ok = false;
       tc_fence_after();
     }
-    lpart[ch * BM + r] = l;
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[B_LSUM]);
-    if (!warp_wait(&bars[B_LSUM], 0, limit, a.status, DETAIL_WAIT_S, abort_flag)) ok = false;
-    const float lt = l + lpart[(ch ^ 1) * BM + r];
-    const float inv = (lt > 0.f) ? 1.f / lt : 0.f;
-    __nv_bfloat16* orow = a.O + h * a.o_hs + (int64_t)row * a.o_ts + ch * OC;
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    __nv_bfloat16* orow = a.O + h * a.o_hs + (int64_t)row * a.o_ts;
 #pragma unroll 1
-    for (int c = 0; c < OC / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
       float o[32];
       if (have && ok) {
-        tmem_ld32(o_t + c * 32, o);
+        tmem_ld32(tmem_O + lane_off + c * 32, o);
         tmem_wait_ld();
       } else {
 #pragma unroll
@@ -595,8 +575,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         }
       }
     }
-    if (ch == 0 && a.lse != nullptr && row < a.N)
-      a.lse[(int64_t)h * a.N + row] = (lt > 0.f) ? (m + log2f(lt)) * 0.69314718055994531f : -INFINITY;
+    if (a.lse != nullptr && row < a.N)
+      a.lse[(int64_t)h * a.N + row] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     __syncwarp();
   }
 

@@ -121,3 +121,21 @@ def test_tiny_and_single_block(dsa):
         heads = orc.build_indices(to64(Q), to64(K), [dict(kind="block_topk", topk=2),
                                                      dict(kind="ashape", sink=3, window=5)], 64)
         run_case(dsa, Q, K, V, heads, 64)
+
+
+def test_repeat_runs_are_bit_identical(dsa):
+    """The kernel has a fixed order of MMAs and softmax steps, so two runs on the
+    same inputs must agree bit for bit; a difference means a race (for example a
+    barrier phase read too early)."""
+    w = synth.workload(2, N=4000, Hq=8, Hkv=2)
+    Q, K, V, _ = synth.make_inputs(w, device="cuda")
+    pats = synth.head_patterns(w)
+    idx = dsa.build_indices(Q, K, pats, w["B"])
+    outs = []
+    for _ in range(3):
+        O, lse = dsa.sparse_prefill(Q, K, V, idx, want_lse=True)
+        torch.cuda.synchronize()
+        outs.append((O.clone(), lse.clone()))
+    for O, lse in outs[1:]:
+        assert torch.equal(O, outs[0][0])
+        assert torch.equal(lse, outs[0][1])
