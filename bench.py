@@ -110,6 +110,20 @@ def algorithmic_index_bytes(w, pats):
     return byt, nqb
 
 
+def reduce_max_over_ranks(values, device="cpu"):
+    """Max over all ranks of each value (timings: the slowest rank sets the pace).
+    Identity when torch.distributed is not initialised."""
+    t = torch.tensor(values, dtype=torch.float64, device=device)
+    if torch.distributed.is_available() and torch.distributed.is_initialized():
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tokens_per_s(N, world, ms_per_step):
+    """Every rank processes its own N-token layer per step (weak scaling)."""
+    return N * world / (ms_per_step * 1e-3)
+
+
 def build_workload(w, device, seed_offset=0):
     w = dict(w)
     w["seed"] = w["seed"] + seed_offset
@@ -282,12 +296,10 @@ def main():
     t_build = [e[0].elapsed_time(e[1]) for e in evs]
     t_attn = [e[1].elapsed_time(e[2]) for e in evs]
     t_step = [a + b for a, b in zip(t_build, t_attn)]
-    tot = torch.tensor([sum(t_step), sum(t_build), sum(t_attn)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(tot, op=torch.distributed.ReduceOp.MAX)
-    ms_step = tot[0].item() / args.steps
-    ms_build = tot[1].item() / args.steps
-    ms_attn = tot[2].item() / args.steps
+    tot = reduce_max_over_ranks([sum(t_step), sum(t_build), sum(t_attn)], device=dev)
+    ms_step = tot[0] / args.steps
+    ms_build = tot[1] / args.steps
+    ms_attn = tot[2] / args.steps
     st, det = dsa.device_status()
     if st != 0:
         raise RuntimeError(f"device status {st} detail {det}")
@@ -317,10 +329,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = torch.tensor([e0.elapsed_time(e1) / args.e2e_steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_ms, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = e2e_ms.item()
+    e2e_ms = reduce_max_over_ranks([e0.elapsed_time(e1) / args.e2e_steps], device=dev)[0]
 
     pk, pk_src = peaks()
     tflops = f_sel / (ms_attn * 1e-3) / 1e12
@@ -335,7 +344,7 @@ def main():
             traffic = tr.get("dram_bytes_per_launch")
 
     line = {
-        "metric": METRIC, "value": N * world / (ms_step * 1e-3), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": whole_job_tokens_per_s(N, world, ms_step), "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
@@ -350,7 +359,7 @@ def main():
                       "density_vs_causal": pairs / causal_pairs},
         "index_build": {"ms": ms_build, "algorithmic_bytes": idx_bytes, "gbs": idx_gbs,
                         "frac_hbm": idx_gbs / pk["hbm_gbs"], "hbm_peak_source": pk_src},
-        "e2e": {"value": N * world / (e2e_ms * 1e-3), "unit": "tokens/s",
+        "e2e": {"value": whole_job_tokens_per_s(N, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * 2,
                 "d2h_bytes_per_step": O.numel() * 2, "ms_per_step": e2e_ms},
         "gpu_launches": kernel_launches_per_step(pats) * args.steps,

@@ -1,0 +1,133 @@
+"""GPU parity at the full sizes of the five workloads, in the launch configuration
+bench.py times: index sets of sampled heads against the oracle (tie-aware), and
+attention outputs of sampled rows against the oracle evaluating the GPU's own
+indices.  The million-token workload is also run as the 4-head x 65536-token
+slice (KV head 0) as a standalone problem."""
+import numpy as np
+import pytest
+import torch
+
+import synth
+from oracle import dsa_oracle as orc
+from tests._parity import assert_close_outputs, assert_lse_close, gpu_lists_to_oracle_heads, to64
+from tests.test_gpu_index import check_indices
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a GPU")
+    import dynamic_sparse_attention_build_b200 as m
+    return m
+
+
+def run_workload(dsa, w, index_heads, row_blocks, rows_per_block=64, seed=0):
+    """Builds indices and attention on the GPU for workload w; checks the index
+    sets of `index_heads` and the outputs of sampled rows of every head."""
+    Q, K, V, planted = synth.make_inputs(w, device="cuda")
+    pats = synth.head_patterns(w)
+    convs = synth.conv_weights(w, device="cuda")
+    G = w["Hq"] // w["Hkv"]
+    dpats = [dict(p, conv=convs[h // G]) if (convs is not None and p["kind"] == "moba") else p
+             for h, p in enumerate(pats)]
+    bufs = dsa.build_indices(Q, K, dpats, w["B"])
+    O, lse = dsa.sparse_prefill(Q, K, V, bufs, want_lse=True)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == (0, 0)
+    N, B = w["N"], w["B"]
+    # index parity for the sampled heads
+    qh = [to64(Q[h]) for h in index_heads]
+    kh = [to64(K[h // G]) for h in index_heads]
+    ref = []
+    for i, h in enumerate(index_heads):
+        conv = None
+        if convs is not None and pats[h]["kind"] == "moba":
+            conv = (convs[h // G][0].double().cpu().numpy(), convs[h // G][1].double().cpu().numpy())
+        ref.append(orc.build_head_index(qh[i], kh[i], pats[h], B, conv))
+
+    class Sub:  # the sampled heads' lists, shaped like IndexBuffers.host_lists()
+        def __init__(self, lists):
+            self.lists = lists
+
+        def host_lists(self):
+            return self.lists
+
+    all_lists = bufs.host_lists()
+    check_indices(Sub([all_lists[h] for h in index_heads]), ref, [pats[h] for h in index_heads], N, B)
+    # attention on sampled rows, every head, with the GPU's own indices
+    rng = np.random.default_rng(seed)
+    nqb = (N + B - 1) // B
+    qbs = sorted(set([nqb - 1] + list(rng.choice(nqb, size=min(nqb, row_blocks - 1), replace=False))))
+    rows = np.concatenate([np.arange(qb * B, min(N, qb * B + B))[:rows_per_block] for qb in qbs])
+    heads = gpu_lists_to_oracle_heads(bufs, N, B)
+    Qc, Kc, Vc = to64(Q), to64(K), to64(V)
+    O_ref, lse_ref = orc.sparse_attention(Qc, Kc, Vc, heads, rows)
+    assert_close_outputs(to64(O)[:, rows], O_ref, w["name"])
+    assert_lse_close(lse.cpu().double().numpy()[:, rows], lse_ref, w["name"])
+    return bufs, planted
+
+
+def test_workload2_llama3_mixed_32k(dsa):
+    w = synth.workload(2)
+    pats = synth.head_patterns(w)
+    kinds = [p["kind"] for p in pats]
+    idx_heads = [kinds.index("vs"), kinds.index("ashape"), kinds.index("block_topk")]
+    bufs, planted = run_workload(dsa, w, idx_heads, row_blocks=3, rows_per_block=16)
+    # planted verticals are found by the VS heads
+    hv = idx_heads[0]
+    G = w["Hq"] // w["Hkv"]
+    assert set(planted["vert"][hv // G].tolist()) <= set(bufs.host_lists()[hv]["vert"].tolist())
+
+
+def test_workload3_flashprefill_threshold_128k(dsa):
+    w = synth.workload(3)
+    bufs, planted = run_workload(dsa, w, [0, 17], row_blocks=4, rows_per_block=16)
+    # kept blocks beyond sink and local share the query block's topic
+    topic = planted["topic"][0].numpy()
+    lists = bufs.host_lists()[0]["blocks"]
+    same = np.mean([all(topic[J] == topic[I] for J in lists[I] if J not in (0, I)) for I in range(len(lists))])
+    assert same > 0.9
+
+
+@pytest.mark.parametrize("B,conv", [(512, 0), (128, 0), (512, 4), (128, 4)])
+def test_workload4_moba_64k(dsa, B, conv):
+    w = synth.workload(4, B=B, conv_width=conv)
+    run_workload(dsa, w, [0, 9], row_blocks=3, rows_per_block=16)
+
+
+def test_workload5_slice_4heads_64k(dsa):
+    """The million-token workload's slice: q-heads 0-3 (KV head 0), tokens 0-65535."""
+    w = synth.workload(5, N=65536, Hq=4, Hkv=1)
+    run_workload(dsa, w, [0, 3], row_blocks=4, rows_per_block=8)
+
+
+def test_workload5_vs_1m(dsa):
+    """Full million-token layer: VS top-k of 2 heads against the oracle and 4 heads'
+    outputs on one sampled row of each of 16 seeded query blocks."""
+    w = synth.workload(5)
+    Q, K, V, planted = synth.make_inputs(w, device="cuda")
+    pats = synth.head_patterns(w)
+    bufs = dsa.build_indices(Q, K, pats, w["B"])
+    O, lse = dsa.sparse_prefill(Q, K, V, bufs, want_lse=True)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == (0, 0)
+    N, B, G = w["N"], w["B"], w["Hq"] // w["Hkv"]
+    lists = bufs.host_lists()
+    from tests._parity import topk_set_ok
+    for h in (0, 5):
+        v, s = orc.vs_estimate(to64(Q[h]), to64(K[h // G]), pats[h]["last_q"])
+        ok, msg = topk_set_ok(lists[h]["vert"], orc.topk_indices(v, pats[h]["n_vert"]), v, pats[h]["n_vert"])
+        assert ok, msg
+        ok, msg = topk_set_ok(lists[h]["slash"], orc.topk_indices(s, pats[h]["n_slash"]), s, pats[h]["n_slash"])
+        assert ok, msg
+        assert set(planted["vert"][h // G].tolist()) <= set(lists[h]["vert"].tolist())
+    heads = gpu_lists_to_oracle_heads(bufs, N, B)
+    rng = np.random.default_rng(5)
+    nqb = N // B
+    rows = np.sort(np.concatenate([[N - 1], rng.choice(nqb, 15, replace=False) * B + rng.integers(0, B, 15)]))
+    for h in (0, 1, 2, 3):
+        Oh, lh = orc.attention_rows(to64(Q[h]), to64(K[h // G]), to64(V[h // G]), heads[h], rows)
+        assert_close_outputs(to64(O[h])[rows], Oh, f"head {h}")
+        assert_lse_close(lse[h].cpu().double().numpy()[rows], lh, f"head {h}")
