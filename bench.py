@@ -339,8 +339,13 @@ def main():
     traffic = None
     tp = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if os.path.exists(tp):
+        # DRAM bytes per launch from an ncu capture; only valid for the kernel
+        # source it was taken on and for this workload
+        import hashlib
         tr = json.load(open(tp))
-        if tr.get("workload") == w["name"]:
+        src = os.path.join(ROOT, "dynamic_sparse_attention_build_b200", "csrc", "dsa_attn.cu")
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        if tr.get("workload") == w["name"] and tr.get("kernel_source_sha256_16") == sha and w["N"] == 32768:
             traffic = tr.get("dram_bytes_per_launch")
 
     line = {

@@ -27,7 +27,7 @@ Sources (page title, section):
         picked by a router) and "2. キーに対する畳み込み適用" (short key conv with
         SiLU and a residual before routing).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * score scale tau = 1/sqrt(d) everywhere;
 * block score s_IJ = tau * mean(q_I) . mean(k_J)  (equal, by bilinearity, to the
@@ -45,9 +45,9 @@ Readings where the pages are silent (each is listed in the design doc):
 * a row with no allowed key has O = 0 and LSE = -inf.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against brute force, closed forms or a library routine, except the two readings
-named "parity unpinned" in the design doc (the VS aggregation rule and the per-config
-forced blocks), which rest on the readings above rather than on the pages.
+against brute force, closed forms or a library routine.  Parity unpinned: the VS
+aggregation rule and the forced blocks of each kind rest on the readings above,
+not on anything the pages fix.
 """
 from __future__ import annotations
 
