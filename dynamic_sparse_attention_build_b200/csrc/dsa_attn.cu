@@ -47,6 +47,9 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t S_COL = 128;    // S buffer b at S_COL + 64 b
 constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after its softmax ended)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+#ifndef DSA_POLY_PERIOD
+#define DSA_POLY_PERIOD 4  // one exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe
+#endif
 
 struct StageInfo {
   int type;   // 0 = key unit, 1 = column tile
@@ -135,6 +138,37 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float
   asm("mov.b64 %0, {%1, %2};" : "=l"(cv) : "f"(c), "f"(c));
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(bv), "l"(cv));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(r));
+}
+
+// 2^x for two values on the FMA and integer pipes instead of the XU pipe:
+// x = j + f with j = round(x) (taken from the low mantissa bits after adding
+// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted for this
+// library to minimise the relative error on [-1/2, 1/2] (max 7.5e-5, far below the
+// bf16 rounding of P); 2^j is added to the exponent field.  x is clamped at -125 so
+// that the exponent field stays normal; 2^-125 is negligible next to the row max.
+__device__ __forceinline__ void poly_ex2x2(float x0, float x1, float& y0, float& y1) {
+  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.99992807f, c1 = 0.693261f, c2 = 0.24261112f, c3 = 0.05517161f;
+  x0 = fmaxf(x0, -125.f);
+  x1 = fmaxf(x1, -125.f);
+  uint64_t xv, sh, yv, jv, fv, pv, cv;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(sh) : "f"(kShift));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(yv) : "l"(xv), "l"(sh));   // y = x + shift
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(jv) : "l"(yv), "l"(sh));   // j = round(x)
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(fv) : "l"(xv), "l"(jv));   // f = x - j
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c3));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(pv) : "f"(c2));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(cv), "l"(fv), "l"(pv));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c1));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(pv), "l"(fv), "l"(cv));
+  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c0));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(pv), "l"(fv), "l"(cv));
+  uint32_t p0, p1, j0, j1;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(pv));
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(yv));
+  y0 = __uint_as_float(p0 + (j0 << 23));
+  y1 = __uint_as_float(p1 + (j1 << 23));
 }
 
 __device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
@@ -484,13 +518,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tmem_ld32(s_t, s);
       tmem_ld32(s_t + 32, s + 32);
       tmem_wait_ld();
+      // fully visible tile for the whole warp: no per-element masking
+      const bool full = __all_sync(0xffffffffu, (mw[0] & mw[1]) == 0xffffffffu);
       // tile max of the allowed raw scores (independent partial maxima)
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+      if (full) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t bits = mw[k];
+        for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+      } else {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[k * 32 + i] : -INFINITY);
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t bits = mw[k];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[k * 32 + i] : -INFINITY);
+        }
       }
       const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       const float m_new = fmaxf(m, mt * a.scale_log2);
@@ -520,21 +561,43 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const bool dead = (m == -INFINITY);
       const float negm = dead ? 0.f : -m;
       float ls[4] = {0.f, 0.f, 0.f, 0.f};
+      if (full && !dead) {
 #pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const uint32_t bits = dead ? 0u : mw[k];
-        uint32_t pk[16];
+        for (int k = 0; k < 2; ++k) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          float x0, x1;
-          fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
-          const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(x0) : 0.f;
-          const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(x1) : 0.f;
-          ls[i & 3] += p0 + p1;
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-          pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1, p0, p1;
+            fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
+            if (i % DSA_POLY_PERIOD == DSA_POLY_PERIOD - 1) {
+              poly_ex2x2(x0, x1, p0, p1);  // part of the pairs on the FMA pipe
+            } else {
+              p0 = fast_ex2(x0);
+              p1 = fast_ex2(x1);
+            }
+            ls[i & 3] += p0 + p1;
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+            pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          tmem_st16(s_t + k * 16, pk);
         }
-        tmem_st16(s_t + k * 16, pk);
+      } else {
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+          const uint32_t bits = dead ? 0u : mw[k];
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            float x0, x1;
+            fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
+            const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(x0) : 0.f;
+            const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(x1) : 0.f;
+            ls[i & 3] += p0 + p1;
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
+            pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          tmem_st16(s_t + k * 16, pk);
+        }
       }
       l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
       tmem_wait_st();
