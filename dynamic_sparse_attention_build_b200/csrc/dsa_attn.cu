@@ -48,7 +48,7 @@ constexpr uint32_t S_COL = 128;    // S buffer b at S_COL + 64 b
 constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after its softmax ended)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
 #ifndef DSA_POLY_PERIOD
-#define DSA_POLY_PERIOD 4  // one exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe
+#define DSA_POLY_PERIOD 8  // one exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe
 #endif
 
 struct StageInfo {
