@@ -72,30 +72,6 @@ __device__ __forceinline__ uint32_t fkey(float f) {
 // ---------------------------------------------------------------------------
 // CTA-wide helpers (blockDim.x threads, multiple of 32, <= 1024)
 // ---------------------------------------------------------------------------
-__device__ int block_sum_int(int v, int* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  v = warp_sum_int(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  int t = 0;
-  for (int i = 0; i < nw; ++i) t += red[i];
-  __syncthreads();
-  return t;
-}
-
-__device__ float block_max_f(float v, float* red) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  v = warp_max(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  float t = -INFINITY;
-  for (int i = 0; i < nw; ++i) t = fmaxf(t, red[i]);
-  __syncthreads();
-  return t;
-}
-
 // Exact top-k of vals[0..n) (ties to the lower index), n > k >= 1.  Finds the
 // k-th largest key T by 4 radix passes of 8 bits, and how many keys equal to T
 // to take.  hist: shared int[256 * nwarps]; red: shared int[64].
@@ -263,13 +239,33 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  for (int r = r_beg + rg; r < r_end; r += RG) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(X + (int64_t)r * ts + c0);
-    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-    float x[8];
+  if (W == 0) {
+    // plain mean: eight independent row loads in flight per thread
+    int r = r_beg + rg;
+    for (; r + 7 * RG < r_end; r += 8 * RG) {
+      uint4 raw[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(e[i]);
-    if (W > 0) {
+      for (int u = 0; u < 8; ++u) raw[u] = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r + u * RG) * ts + c0));
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
+      }
+    }
+    for (; r < r_end; r += RG) {
+      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * ts + c0));
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
+    }
+  } else {
+    for (int r = r_beg + rg; r < r_end; r += RG) {
+      const uint4 raw = *reinterpret_cast<const uint4*>(X + (int64_t)r * ts + c0);
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+      float x[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(e[i]);
       float conv[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) conv[i] = cb[c0 + i];
@@ -281,10 +277,8 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
         for (int i = 0; i < 8; ++i) conv[i] = fmaf(cw[(c0 + i) * W + t], __bfloat162float(ee[i]), conv[i]);
       }
 #pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] += conv[i] / (1.f + expf(-conv[i]));
+      for (int i = 0; i < 8; ++i) acc[i] += x[i] + conv[i] / (1.f + expf(-conv[i]));
     }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += x[i];
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) part[rg][c0 + i] = acc[i];
@@ -297,76 +291,184 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
 }
 
 // ---------------------------------------------------------------------------
-// block scores + selection: one CTA (256 threads) per (block slot, query block I)
+// block scores + selection.  One CTA (256 threads) per (block slot, SEL_RI
+// consecutive query blocks).  The scores of those rows against every candidate
+// key block are an fp32 tile product q̄_tile x K̄^T computed through shared
+// memory (K̄ is read once per SEL_RI rows, not once per row); thread t owns the
+// 2 x 4 block of rows 2 (t / 32) + {0, 1} and key blocks t % 32 + 32 m.  Then one warp per row selects: a max and a compare for
+// the threshold, an exact radix select for top-k; the selection bitmap is built
+// one 32-block word at a time from warp ballots.
 // ---------------------------------------------------------------------------
+constexpr int SEL_RI = 16;  // query blocks per CTA
+constexpr int SEL_RJ = 128;  // key blocks per shared-memory chunk
+
+// Warp-level exact top-k of vals[0..n) (ties to the lower index), 0 < k < n.
+// hist: this warp's shared int[256].  Returns the k-th largest key and how many
+// keys equal to it to take.
+__device__ void warp_radix_kth(const float* vals, int n, int k, int* hist, uint32_t* T_out, int* take_eq) {
+  const int lane = threadIdx.x & 31;
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int b = lane; b < 256; b += 32) hist[b] = 0;
+    __syncwarp();
+    for (int i = lane; i < n; i += 32) {
+      const uint32_t key = fkey(vals[i]);
+      if ((key & mask) == prefix) atomicAdd(&hist[(key >> shift) & 255u], 1);
+    }
+    __syncwarp();
+    // lane L owns bins 255-8L .. 248-8L (descending); find the bin where the
+    // running count from the top reaches `need`
+    int c[8], own = 0;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      c[q] = hist[255 - 8 * lane - q];
+      own += c[q];
+    }
+    int incl = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int excl = incl - own;
+    const bool here = excl < need && incl >= need;
+    const unsigned who = __ballot_sync(0xffffffffu, here);
+    const int src = __ffs(who) - 1;
+    int digit = 0, above = 0;
+    if (here) {
+      int run = excl;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (run + c[q] >= need) { digit = 255 - 8 * lane - q; break; }
+        run += c[q];
+      }
+      above = run;
+    }
+    digit = __shfl_sync(0xffffffffu, digit, src);
+    above = __shfl_sync(0xffffffffu, above, src);
+    prefix |= (uint32_t)digit << shift;
+    mask |= 255u << shift;
+    need -= above;
+    __syncwarp();
+  }
+  *T_out = prefix;
+  *take_eq = need;
+}
+
+static_assert((256 / 32) * 2 == SEL_RI && 32 * 4 == SEL_RJ, "score tile mapping of k_block_select");
+
 template <int D>
 __global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                       int32_t* blk_ptr) {
-  extern __shared__ float sc[];  // [nkb] scores
-  __shared__ float qv[D];
-  __shared__ int hist[256 * 8];
-  __shared__ int red[64];
-  __shared__ float redf[32];
-  const int I = blockIdx.x;
+  extern __shared__ float smf[];
+  constexpr int KS = D + 4;                  // padded K̄ row (floats)
+  float* qs = smf;                           // [SEL_RI][D]
+  float* ks = qs + SEL_RI * D;               // [SEL_RJ][KS]
+  float* sc = ks + SEL_RJ * KS;              // [SEL_RI][npad]
+  __shared__ int hist[8][256];
+  const int npad = L.nkw * 32;
   const int slot = blockIdx.y;
+  const int I0 = blockIdx.x * SEL_RI;
+  const int nI = min(SEL_RI, L.nqb - I0);
   const int h = ht.bhead[slot];
   const int kind = ht.kind[h];
   const int kvh = h / L.G;
   const float tau = rsqrtf((float)D);
-  const float* qbar = reinterpret_cast<const float*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I) * D;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* qbar = reinterpret_cast<const float*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I0) * D;
   const float* kbar = reinterpret_cast<const float*>(ws + L.off_kbar) + (int64_t)kvh * L.nqb * D;
-  uint32_t* sel = reinterpret_cast<uint32_t*>(ws + L.off_sel) + ((int64_t)slot * L.nqb + I) * L.nkw;
-  for (int c = threadIdx.x; c < D; c += blockDim.x) qv[c] = qbar[c];
-  for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) sel[w] = 0u;
-  __syncthreads();
-  // candidates: J <= I (MoBA: J < I)
-  const int ncand = (kind == DSA_KIND_MOBA) ? I : I + 1;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int J = warp; J < ncand; J += 8) {
-    const float* kr = kbar + (int64_t)J * D;
-    float s = 0.f;
-    for (int c = lane; c < D; c += 32) s = fmaf(qv[c], kr[c], s);
-    s = warp_sum(s);
-    if (lane == 0) sc[J] = s * tau;
+  for (int i = tid; i < SEL_RI * D; i += 256) qs[i] = (i < nI * D) ? qbar[i] : 0.f;
+  // scores for J < I0 + nI (the candidates of the group's last row)
+  const int Jend = I0 + nI;
+  const int rp = tid >> 5;   // rows 2 rp, 2 rp + 1 (rp < 8, so rows < SEL_RI)
+  const int jq = tid & 31;   // key blocks jq + 32 m, m < 4 (so < SEL_RJ)
+  for (int J0 = 0; J0 < Jend; J0 += SEL_RJ) {
+    __syncthreads();
+    const int nj = min(SEL_RJ, Jend - J0);
+    for (int i = tid; i < SEL_RJ * (D / 4); i += 256) {
+      const int j = i / (D / 4), c = (i % (D / 4)) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < nj) v = *reinterpret_cast<const float4*>(kbar + (int64_t)(J0 + j) * D + c);
+      *reinterpret_cast<float4*>(ks + j * KS + c) = v;
+    }
+    __syncthreads();
+    float acc[2][4];
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) acc[a][m] = 0.f;
+#pragma unroll 4
+    for (int c = 0; c < D; c += 4) {
+      const float4 q0 = *reinterpret_cast<const float4*>(qs + (2 * rp) * D + c);
+      const float4 q1 = *reinterpret_cast<const float4*>(qs + (2 * rp + 1) * D + c);
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const float4 k4 = *reinterpret_cast<const float4*>(ks + (jq + 32 * m) * KS + c);
+        acc[0][m] = fmaf(q0.x, k4.x, fmaf(q0.y, k4.y, fmaf(q0.z, k4.z, fmaf(q0.w, k4.w, acc[0][m]))));
+        acc[1][m] = fmaf(q1.x, k4.x, fmaf(q1.y, k4.y, fmaf(q1.z, k4.z, fmaf(q1.w, k4.w, acc[1][m]))));
+      }
+    }
+#pragma unroll
+    for (int a = 0; a < 2; ++a)
+#pragma unroll
+      for (int m = 0; m < 4; ++m) {
+        const int j = jq + 32 * m;
+        if (j < nj) sc[(2 * rp + a) * npad + J0 + j] = acc[a][m] * tau;
+      }
   }
   __syncthreads();
-  int count = 0;
-  if (kind == DSA_KIND_BLOCK_THRESHOLD) {
-    float mx = -INFINITY;
-    for (int J = threadIdx.x; J < ncand; J += blockDim.x) mx = fmaxf(mx, sc[J]);
-    mx = block_max_f(mx, redf);
-    const float thr = mx + ht.lnalpha[h];
-    for (int J = threadIdx.x; J < ncand; J += blockDim.x)
-      if (sc[J] >= thr) atomicOr(&sel[J >> 5], 1u << (J & 31));
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      if (ht.keep_sink[h]) atomicOr(&sel[0], 1u);
-      if (ht.keep_local[h]) atomicOr(&sel[I >> 5], 1u << (I & 31));
+  // selection: warp w handles rows w and w + 8
+  for (int rr = warp; rr < nI; rr += 8) {
+    const int I = I0 + rr;
+    const float* row = sc + rr * npad;
+    uint32_t* sel = reinterpret_cast<uint32_t*>(ws + L.off_sel) + ((int64_t)slot * L.nqb + I) * L.nkw;
+    const int ncand = (kind == DSA_KIND_MOBA) ? I : I + 1;
+    int count = 0;
+    if (kind == DSA_KIND_BLOCK_THRESHOLD) {
+      float mx = -INFINITY;
+      for (int J = lane; J < ncand; J += 32) mx = fmaxf(mx, row[J]);
+      mx = warp_max(mx);
+      const float thr = mx + ht.lnalpha[h];
+      for (int w0 = 0; w0 < L.nkw; ++w0) {
+        const int J = w0 * 32 + lane;
+        bool keep = J < ncand && row[J] >= thr;
+        if (J == 0 && ht.keep_sink[h]) keep = true;
+        if (J == I && ht.keep_local[h]) keep = true;
+        const unsigned bits = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) sel[w0] = bits;
+        count += __popc(bits);
+      }
+    } else {
+      const int k = ht.topk[h];
+      uint32_t T = 0;
+      int take_eq = 0;
+      const bool all = ncand <= k;
+      if (!all && k > 0) warp_radix_kth(row, ncand, k, hist[warp], &T, &take_eq);
+      int eq_run = 0;
+      for (int w0 = 0; w0 < L.nkw; ++w0) {
+        const int J = w0 * 32 + lane;
+        bool keep = false, iseq = false;
+        if (J < ncand && k > 0) {
+          if (all) {
+            keep = true;
+          } else {
+            const uint32_t key = fkey(row[J]);
+            keep = key > T;
+            iseq = key == T;
+          }
+        }
+        const unsigned eqm = __ballot_sync(0xffffffffu, iseq);
+        if (iseq && eq_run + __popc(eqm & ((1u << lane) - 1u)) < take_eq) keep = true;
+        eq_run += __popc(eqm);
+        if (kind == DSA_KIND_MOBA && J == I) keep = true;
+        const unsigned bits = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) sel[w0] = bits;
+        count += __popc(bits);
+      }
     }
-    __syncthreads();
-    int c = 0;
-    for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) c += __popc(sel[w]);
-    count = block_sum_int(c, red);
-  } else {
-    const int k = ht.topk[h];
-    if (ncand <= k) {
-      for (int J = threadIdx.x; J < ncand; J += blockDim.x) atomicOr(&sel[J >> 5], 1u << (J & 31));
-      count = ncand;
-    } else if (k > 0) {
-      uint32_t T;
-      int take_eq;
-      auto load = [&](int i) { return sc[i]; };
-      radix_kth(load, ncand, k, hist, red, &T, &take_eq);
-      ordered_select(load, ncand, T, take_eq, red, [&](int i, int) { atomicOr(&sel[i >> 5], 1u << (i & 31)); });
-      count = k;
-    }
-    __syncthreads();
-    if (kind == DSA_KIND_MOBA) {
-      if (threadIdx.x == 0) atomicOr(&sel[I >> 5], 1u << (I & 31));
-      count += 1;
-    }
+    if (lane == 0) blk_ptr[1 + h * L.nqb + I] = count;
   }
-  if (threadIdx.x == 0) blk_ptr[1 + h * L.nqb + I] = count;
 }
 
 // ---------------------------------------------------------------------------
@@ -1011,7 +1113,7 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
     }
   }
   if (blk > INT32_MAX || ccap > INT32_MAX || (int64_t)p.Hq * nqb + 1 > INT32_MAX) return DSA_ERR_UNSUPPORTED;
-  if (L->nbh > 0 && L->nqb > 16384) return DSA_ERR_UNSUPPORTED;  // block scores live in shared memory
+  if (L->nbh > 0 && L->nqb > 2048) return DSA_ERR_UNSUPPORTED;  // block scores of 16 rows live in shared memory
   const int64_t d = p.d;
   int64_t off = 0;
   L->off_qbar = off; off = align256(off + (int64_t)L->nbh * nqb * d * 4);
@@ -1108,17 +1210,18 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   if (L.nbh > 0) {
-    const size_t sel_smem = (size_t)L.nqb * 4;
     if (p.d == 128) {
       k_pool<128><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
                                                              p.k_head_stride, p.k_token_stride, ws);
+      const size_t sel_smem = (size_t)(SEL_RI * 128 + SEL_RJ * (128 + 4) + SEL_RI * L.nkw * 32) * 4;
       DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<128><<<dim3(L.nqb, L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<128><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
     } else {
       k_pool<64><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
                                                             p.k_head_stride, p.k_token_stride, ws);
+      const size_t sel_smem = (size_t)(SEL_RI * 64 + SEL_RJ * (64 + 4) + SEL_RI * L.nkw * 32) * 4;
       DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<64><<<dim3(L.nqb, L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<64><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
     }
   }
   if (L.nvs > 0) {

@@ -92,6 +92,8 @@ typedef struct dsa_problem {
  *   BLOCK_TOPK:      topk >= 1 (blocks per query block among J <= I).
  *   BLOCK_THRESHOLD: 0 < alpha <= 1, in probability space; keep_sink / keep_local
  *                    force blocks 0 and I.
+ *   Block kinds (BLOCK_TOPK, BLOCK_THRESHOLD, MOBA) need nqb = ceil(N / block) <= 2048
+ *   (DSA_ERR_UNSUPPORTED otherwise).
  *   MOBA:            topk >= 0 past blocks (J < I) plus the own block I.  Optional
  *                    causal depthwise key conv for routing: conv_width in [0, 8]
  *                    (0 = off); conv_weight: device float [d][conv_width] (tap t
