@@ -198,7 +198,8 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                   const __grid_constant__ AttnArgs a) {
   using L = Smem<D>;
   constexpr int DS = L::DS;
   extern __shared__ uint8_t smem_raw[];
@@ -231,15 +232,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     fence_barrier_init();
     misc[2] = 0;
     misc[3] = 0;
+    // Q does not depend on the index lists: start its load before reading them
+    tma_prefetch_desc(&tmQ);
+    mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
+    for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
   }
   if (warp == 1) {
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), TMEM_COLS);
     tc_fence_before();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmO);
   }
   for (int i = tid; i < 2 * a.nwords; i += NTHREADS) bits0[i] = 0u;
   __syncthreads();
@@ -321,8 +326,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // ------------------------------------------------------------ loaders
     const int ltid = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
     if (warp == 0 && lane == 0) {
-      mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
-      for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
       int w = 0;
       uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
       for (int t = 0; t < T_u; ++t) {
@@ -614,7 +617,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       tc_fence_after();
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
-    __nv_bfloat16* orow = a.O + h * a.o_hs + (int64_t)row * a.o_ts;
+    // O / l as bf16 into shared memory (the K buffers, idle once every MMA has
+    // finished) in the 128-byte-swizzled layout of the O tensor map, then one TMA
+    // store per 64 columns; rows past N are clipped by the map
+    uint8_t* ost = sm + L::K_OFF;
 #pragma unroll 1
     for (int c = 0; c < D / 32; ++c) {
       float o[32];
@@ -625,18 +631,24 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
 #pragma unroll
         for (int i = 0; i < 32; ++i) o[i] = 0.f;
       }
-      if (row < a.N) {
 #pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          uint32_t pk[4];
+      for (int v = 0; v < 4; ++v) {
+        uint32_t pk[4];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(o[v * 8 + 2 * i] * inv, o[v * 8 + 2 * i + 1] * inv);
-            pk[i] = *reinterpret_cast<uint32_t*>(&v2);
-          }
-          *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int i = 0; i < 4; ++i) {
+          __nv_bfloat162 v2 = __floats2bfloat162_rn(o[v * 8 + 2 * i] * inv, o[v * 8 + 2 * i + 1] * inv);
+          pk[i] = *reinterpret_cast<uint32_t*>(&v2);
         }
+        *reinterpret_cast<uint4*>(ost + (c >> 1) * QSLAB + swz(r, (c & 1) * 4 + v)) =
+            make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
+    }
+    fence_proxy_async_smem();
+    named_barrier(2, 128);  // the four softmax warps
+    if (r == 0) {
+      for (int c = 0; c < DS; ++c) tma_store_3d(&tmO, ost + c * QSLAB, c * 64, row0, h);
+      tma_store_commit();
+      tma_store_wait_read();
     }
     if (a.lse != nullptr && row < a.N)
       a.lse[(int64_t)h * a.N + row] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
@@ -686,8 +698,9 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int H, int64_t t
 template <int D>
 dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const void* V, const dsa_indices& idx,
                     void* O, float* lse, cudaStream_t stream, unsigned* status) {
-  CUtensorMap mq, mk, mv;
-  if (!make_map(&mq, Q, D, p.N, p.Hq, p.q_token_stride, p.q_head_stride, BM) ||
+  CUtensorMap mq, mk, mv, mo;
+  if (!make_map(&mo, O, D, p.N, p.Hq, p.o_token_stride, p.o_head_stride, BM) ||
+      !make_map(&mq, Q, D, p.N, p.Hq, p.q_token_stride, p.q_head_stride, BM) ||
       !make_map(&mk, K, D, p.N, p.Hkv, p.k_token_stride, p.k_head_stride, UNIT) ||
       !make_map(&mv, V, D, p.N, p.Hkv, p.v_token_stride, p.v_head_stride, UNIT))
     return DSA_ERR_CUDA;
@@ -727,7 +740,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = a.n_qtiles * p.Hq;
   if (grid == 0) return DSA_OK;
-  sparse_attn_kernel<D><<<grid, NTHREADS, smem, stream>>>(mq, mk, mv, a);
+  sparse_attn_kernel<D><<<grid, NTHREADS, smem, stream>>>(mq, mk, mv, mo, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;
