@@ -215,7 +215,7 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
   if (!isq && !ct.need[kvh]) return;
   const __nv_bfloat16* X;
   int64_t ts;
-  float* out;
+  __nv_bfloat16* out;  // the pooled row as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
   int W = 0;
   const float* cw = nullptr;
   const float* cb = nullptr;
@@ -223,11 +223,11 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
     const int h = ht.bhead[item];
     X = Q + h * q_hs;
     ts = q_ts;
-    out = reinterpret_cast<float*>(ws + L.off_qbar) + ((int64_t)item * L.nqb + b) * D;
+    out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_qbar) + ((int64_t)item * L.nqb + b) * 2 * D;
   } else {
     X = K + kvh * k_hs;
     ts = k_ts;
-    out = reinterpret_cast<float*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * D;
+    out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * 2 * D;
     W = ct.width[kvh];
     cw = ct.w[kvh];
     cb = ct.b[kvh];
@@ -286,21 +286,43 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht
   if (threadIdx.x < D) {
     float s = 0.f;
     for (int g = 0; g < RG; ++g) s += part[g][threadIdx.x];
-    out[threadIdx.x] = s / (float)(r_end - r_beg);
+    const float x = s / (float)(r_end - r_beg);
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    out[threadIdx.x] = hi;
+    out[D + threadIdx.x] = __float2bfloat16_rn(x - __bfloat162float(hi));
   }
 }
 
 // ---------------------------------------------------------------------------
-// block scores + selection.  One CTA (256 threads) per (block slot, SEL_RI
+// block scores + selection.  One CTA (SEL_NT threads) per (block slot, SEL_RI
 // consecutive query blocks).  The scores of those rows against every candidate
-// key block are an fp32 tile product q̄_tile x K̄^T computed through shared
-// memory (K̄ is read once per SEL_RI rows, not once per row); thread t owns the
-// 2 x 4 block of rows 2 (t / 32) + {0, 1} and key blocks t % 32 + 32 m.  Then one warp per row selects: a max and a compare for
-// the threshold, an exact radix select for top-k; the selection bitmap is built
-// one 32-block word at a time from warp ballots.
+// key block are one 16-row tile product q̄_tile x K̄^T on the tensor cores
+// (mma.sync m16n8k16, bf16 operands, fp32 accumulation).  The pooled rows are
+// stored as bf16 hi + lo pairs and the product keeps hi.hi + hi.lo + lo.hi, so a
+// score carries about 16 mantissa bits of each operand (the fp32 means have 24).
+// K̄ is read once per SEL_RI rows; each warp takes 8-key-block column tiles in
+// turn.  Then one warp per row selects: a max and a compare for the threshold,
+// an exact radix select for top-k; the selection bitmap is built one 32-block
+// word at a time from warp ballots (only the words up to row I's own block are
+// written; the list fill reads no further).
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
 constexpr int SEL_RI = 16;  // query blocks per CTA
-constexpr int SEL_RJ = 128;  // key blocks per shared-memory chunk
+#ifndef DSA_SEL_NT
+#define DSA_SEL_NT 512
+#endif
+constexpr int SEL_NT = DSA_SEL_NT;  // threads per CTA
+constexpr int SEL_NW = SEL_NT / 32;
+// score row stride in floats: 8 past a multiple of 32 so the 8-byte stores of
+// one half-warp (rows g..g+3, columns 2 t4) hit 16 distinct bank pairs
+__host__ __device__ constexpr int SEL_RS(int npad) { return npad + 8; }
 
 // Warp-level exact top-k of vals[0..n) (ties to the lower index), 0 < k < n.
 // hist: this warp's shared int[256].  Returns the k-th largest key and how many
@@ -356,17 +378,11 @@ __device__ void warp_radix_kth(const float* vals, int n, int k, int* hist, uint3
   *take_eq = need;
 }
 
-static_assert((256 / 32) * 2 == SEL_RI && 32 * 4 == SEL_RJ, "score tile mapping of k_block_select");
-
 template <int D>
-__global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+__global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                       int32_t* blk_ptr) {
-  extern __shared__ float smf[];
-  constexpr int KS = D + 4;                  // padded K̄ row (floats)
-  float* qs = smf;                           // [SEL_RI][D]
-  float* ks = qs + SEL_RI * D;               // [SEL_RJ][KS]
-  float* sc = ks + SEL_RJ * KS;              // [SEL_RI][npad]
-  __shared__ int hist[8][256];
+  extern __shared__ float sc[];  // [SEL_RI][SEL_RS(npad)] scores of the group's rows
+  __shared__ int hist[SEL_NW][256];
   const int npad = L.nkw * 32;
   const int slot = blockIdx.y;
   const int I0 = blockIdx.x * SEL_RI;
@@ -376,52 +392,67 @@ __global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ He
   const int kvh = h / L.G;
   const float tau = rsqrtf((float)D);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const float* qbar = reinterpret_cast<const float*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I0) * D;
-  const float* kbar = reinterpret_cast<const float*>(ws + L.off_kbar) + (int64_t)kvh * L.nqb * D;
-  for (int i = tid; i < SEL_RI * D; i += 256) qs[i] = (i < nI * D) ? qbar[i] : 0.f;
-  // scores for J < I0 + nI (the candidates of the group's last row)
-  const int Jend = I0 + nI;
-  const int rp = tid >> 5;   // rows 2 rp, 2 rp + 1 (rp < 8, so rows < SEL_RI)
-  const int jq = tid & 31;   // key blocks jq + 32 m, m < 4 (so < SEL_RJ)
-  for (int J0 = 0; J0 < Jend; J0 += SEL_RJ) {
-    __syncthreads();
-    const int nj = min(SEL_RJ, Jend - J0);
-    for (int i = tid; i < SEL_RJ * (D / 4); i += 256) {
-      const int j = i / (D / 4), c = (i % (D / 4)) * 4;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < nj) v = *reinterpret_cast<const float4*>(kbar + (int64_t)(J0 + j) * D + c);
-      *reinterpret_cast<float4*>(ks + j * KS + c) = v;
-    }
-    __syncthreads();
-    float acc[2][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) acc[a][m] = 0.f;
-#pragma unroll 4
-    for (int c = 0; c < D; c += 4) {
-      const float4 q0 = *reinterpret_cast<const float4*>(qs + (2 * rp) * D + c);
-      const float4 q1 = *reinterpret_cast<const float4*>(qs + (2 * rp + 1) * D + c);
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const float4 k4 = *reinterpret_cast<const float4*>(ks + (jq + 32 * m) * KS + c);
-        acc[0][m] = fmaf(q0.x, k4.x, fmaf(q0.y, k4.y, fmaf(q0.z, k4.z, fmaf(q0.w, k4.w, acc[0][m]))));
-        acc[1][m] = fmaf(q1.x, k4.x, fmaf(q1.y, k4.y, fmaf(q1.z, k4.z, fmaf(q1.w, k4.w, acc[1][m]))));
-      }
-    }
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int m = 0; m < 4; ++m) {
-        const int j = jq + 32 * m;
-        if (j < nj) sc[(2 * rp + a) * npad + J0 + j] = acc[a][m] * tau;
-      }
+  const __nv_bfloat16* qhl = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I0) * 2 * D;
+  const __nv_bfloat16* khl = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_kbar) + (int64_t)kvh * L.nqb * 2 * D;
+  const int g = lane >> 2, t4 = lane & 3;
+  // The contraction runs over the channels in a permuted order (the same on
+  // both operands, so the dot products are unchanged): the 16-byte run of
+  // channels 32m + 8 t4 .. +7 of a row feeds k-steps 2m and 2m + 1, so every
+  // fragment register pair comes from one vector load.
+  auto ld16 = [](const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint4*>(p)); };
+  // the group's 16 pooled query rows (hi then lo) staged in shared memory; the
+  // row pitch is 64 bytes past a multiple of 128 so that the 16-byte fragment
+  // loads of rows g and g + 1 fall in different banks
+  constexpr int QP = 2 * D + 32;
+  __shared__ __align__(16) __nv_bfloat16 qs[SEL_RI][QP];
+  for (int i = tid; i < SEL_RI * (2 * D / 8); i += SEL_NT) {
+    const int r = i / (2 * D / 8), c = (i % (2 * D / 8)) * 8;
+    *reinterpret_cast<uint4*>(&qs[r][c]) = r < nI ? ld16(qhl + (int64_t)r * 2 * D + c) : make_uint4(0u, 0u, 0u, 0u);
   }
   __syncthreads();
-  // selection: warp w handles rows w and w + 8
-  for (int rr = warp; rr < nI; rr += 8) {
+  // s = tau (qhi khi + qhi klo + qlo khi): bf16 tensor-core products with fp32
+  // accumulation; the dropped qlo klo term is below 2^-16 of |q| |k| per channel.
+  // Each warp takes 8-key-block column tiles in turn.
+  const int Jend = I0 + nI;  // candidates of the group's last row are J < Jend
+  const int ntiles = ceil_div(Jend, 8);
+  for (int nt = warp; nt < ntiles; nt += SEL_NW) {
+    const int J0 = nt * 8;
+    const int Jb = J0 + g;
+    const __nv_bfloat16* kp = khl + (int64_t)min(Jb, L.nqb - 1) * 2 * D + 8 * t4;
+    uint4 bh[D / 32], bl[D / 32];
+#pragma unroll
+    for (int m = 0; m < D / 32; ++m) {
+      bh[m] = ld16(kp + 32 * m);
+      bl[m] = ld16(kp + D + 32 * m);
+    }
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int m = 0; m < D / 32; ++m) {
+      const int cq = 32 * m + 8 * t4;
+      const uint4 h0 = *reinterpret_cast<const uint4*>(&qs[g][cq]);
+      const uint4 h1 = *reinterpret_cast<const uint4*>(&qs[g + 8][cq]);
+      const uint4 l0 = *reinterpret_cast<const uint4*>(&qs[g][D + cq]);
+      const uint4 l1 = *reinterpret_cast<const uint4*>(&qs[g + 8][D + cq]);
+      const uint32_t ah0[4] = {h0.x, h1.x, h0.y, h1.y}, ah1[4] = {h0.z, h1.z, h0.w, h1.w};
+      const uint32_t al0[4] = {l0.x, l1.x, l0.y, l1.y}, al1[4] = {l0.z, l1.z, l0.w, l1.w};
+      mma_bf16_16816(c, ah0, bh[m].x, bh[m].y);
+      mma_bf16_16816(c, ah0, bl[m].x, bl[m].y);
+      mma_bf16_16816(c, al0, bh[m].x, bh[m].y);
+      mma_bf16_16816(c, ah1, bh[m].z, bh[m].w);
+      mma_bf16_16816(c, ah1, bl[m].z, bl[m].w);
+      mma_bf16_16816(c, al1, bh[m].z, bh[m].w);
+    }
+    // columns J0 + 2 t4, +1 of rows g and g + 8; key blocks past the last
+    // real one (clamped loads above) land in columns no row reads
+    const int J = J0 + 2 * t4;
+    if (g < nI) *reinterpret_cast<float2*>(sc + g * SEL_RS(npad) + J) = make_float2(c[0] * tau, c[1] * tau);
+    if (g + 8 < nI) *reinterpret_cast<float2*>(sc + (g + 8) * SEL_RS(npad) + J) = make_float2(c[2] * tau, c[3] * tau);
+  }
+  __syncthreads();
+  // selection: warp w handles rows w, w + SEL_NW, ...
+  for (int rr = warp; rr < nI; rr += SEL_NW) {
     const int I = I0 + rr;
-    const float* row = sc + rr * npad;
+    const float* row = sc + rr * SEL_RS(npad);
     uint32_t* sel = reinterpret_cast<uint32_t*>(ws + L.off_sel) + ((int64_t)slot * L.nqb + I) * L.nkw;
     const int ncand = (kind == DSA_KIND_MOBA) ? I : I + 1;
     int count = 0;
@@ -430,7 +461,7 @@ __global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ He
       for (int J = lane; J < ncand; J += 32) mx = fmaxf(mx, row[J]);
       mx = warp_max(mx);
       const float thr = mx + ht.lnalpha[h];
-      for (int w0 = 0; w0 < L.nkw; ++w0) {
+      for (int w0 = 0; w0 <= (I >> 5); ++w0) {
         const int J = w0 * 32 + lane;
         bool keep = J < ncand && row[J] >= thr;
         if (J == 0 && ht.keep_sink[h]) keep = true;
@@ -446,7 +477,7 @@ __global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ He
       const bool all = ncand <= k;
       if (!all && k > 0) warp_radix_kth(row, ncand, k, hist[warp], &T, &take_eq);
       int eq_run = 0;
-      for (int w0 = 0; w0 < L.nkw; ++w0) {
+      for (int w0 = 0; w0 <= (I >> 5); ++w0) {
         const int J = w0 * 32 + lane;
         bool keep = false, iseq = false;
         if (J < ncand && k > 0) {
@@ -479,13 +510,6 @@ __global__ void __launch_bounds__(256) k_block_select(const __grid_constant__ He
 //           s[o] (diagonal sums, global atomics at the chunk edges)
 // Rows padded to LP = 16 * RT; warps: RT row tiles x (8 / RT) key groups.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-      "{%0,%1,%2,%3};"
-      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
 
 template <int D, int RT, int PASS>
 __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, Layout L, const __nv_bfloat16* Q,
@@ -866,9 +890,10 @@ __global__ void k_blk_fill(const __grid_constant__ HeadTab ht, Layout L, const u
   }
   const uint32_t* sel = reinterpret_cast<const uint32_t*>(ws + L.off_sel) + ((int64_t)ht.bslot[h] * L.nqb + qb) * L.nkw;
   int pos = beg;
-  for (int w0 = 0; w0 < L.nkw; w0 += 32) {
+  const int nw = (qb >> 5) + 1;  // selected blocks satisfy J <= qb; later words are never written
+  for (int w0 = 0; w0 < nw; w0 += 32) {
     const int w = w0 + lane;
-    const uint32_t bits = (w < L.nkw) ? sel[w] : 0u;
+    const uint32_t bits = (w < nw) ? sel[w] : 0u;
     const int c = __popc(bits);
     int incl = c;
 #pragma unroll
@@ -1213,15 +1238,15 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
     if (p.d == 128) {
       k_pool<128><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
                                                              p.k_head_stride, p.k_token_stride, ws);
-      const size_t sel_smem = (size_t)(SEL_RI * 128 + SEL_RJ * (128 + 4) + SEL_RI * L.nkw * 32) * 4;
+      const size_t sel_smem = (size_t)SEL_RI * SEL_RS(L.nkw * 32) * 4;
       DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<128><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<128><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), SEL_NT, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
     } else {
       k_pool<64><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
                                                             p.k_head_stride, p.k_token_stride, ws);
-      const size_t sel_smem = (size_t)(SEL_RI * 64 + SEL_RJ * (64 + 4) + SEL_RI * L.nkw * 32) * 4;
+      const size_t sel_smem = (size_t)SEL_RI * SEL_RS(L.nkw * 32) * 4;
       DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<64><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), 256, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<64><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), SEL_NT, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
     }
   }
   if (L.nvs > 0) {
