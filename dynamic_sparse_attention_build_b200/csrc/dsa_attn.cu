@@ -8,7 +8,8 @@
 // (CSR blocks, or qb - delta for the VS distances), plus its listed columns, and
 // for A-shape heads only those with j < sink or i - j < window.
 //
-// Design (one CTA = 128 query rows of one head, two CTAs per SM):
+// Design (persistent: two CTAs per SM; a work item = 128 query rows of one head,
+// items dealt round-robin over the CTAs, latest (heaviest) query tiles first):
 //   * the tile's two 64-row halves each belong to one query block (two different
 //     blocks when B = 64, the same block otherwise).  Their key lists become two
 //     bitmaps over 64-key units in shared memory; the union is walked in
@@ -16,9 +17,13 @@
 //     halves that listed it (the other half masks it out);
 //   * column lists are gathered into dense 64-key tiles (gather-and-densify); a
 //     column inside a block the half already keeps is masked out;
-//   * warp 0 issues TMA loads (SWIZZLE_128B boxes of 64 x 64) into two K and two V
-//     buffers, warps 0,2,3 gather column rows, warp 1 issues tcgen05.mma, warps
-//     4-7 run the online softmax (one thread per row) and the epilogue;
+//   * warps 0,2,3 build the bitmaps, issue TMA loads (SWIZZLE_128B boxes of
+//     64 x 64) into two K and two V buffers and gather column rows; warp 1 issues
+//     tcgen05.mma; warps 4-7 run the online softmax (one thread per row) and the
+//     epilogue.  The loaders read the next item's lists and load its Q while the
+//     other warps finish the current item, so an item's set-up is off the
+//     critical path; tile and item counters run across items, so every barrier
+//     keeps its phase from one item to the next;
 //   * TMEM (256 columns per CTA): O at [0, 128), two S buffers of 64 columns at
 //     128 and 192.  S(t+1) = Q K(t+1)^T is computed while the softmax works on
 //     S(t); the softmax writes P(t) as bf16 pairs over the first 32 columns of its
@@ -30,6 +35,8 @@
 //     SM, so one CTA's softmax also overlaps the other's tensor-core work.
 // No cluster, no multicast; every wait is bounded (status word + early exit).
 #include <cudaTypedefs.h>
+
+#include <atomic>
 
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
@@ -47,6 +54,17 @@ constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t S_COL = 128;    // S buffer b at S_COL + 64 b
 constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after its softmax ended)
 constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+#ifndef DSA_LOADER_SUSPEND
+#define DSA_LOADER_SUSPEND 1
+#endif
+#ifndef DSA_MMA_SUSPEND
+#define DSA_MMA_SUSPEND 1
+#endif
+// Waits of the TMA producer / MMA thread block in try_wait (the warp then takes
+// no issue slots from the softmax warp that shares its scheduler) instead of
+// polling.
+constexpr bool kLoaderSuspend = DSA_LOADER_SUSPEND != 0;
+constexpr bool kMmaSuspend = DSA_MMA_SUSPEND != 0;
 #ifndef DSA_POLY_PERIOD
 #define DSA_POLY_PERIOD 8  // one exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe
 #endif
@@ -56,6 +74,10 @@ struct StageInfo {
   int u;      // unit id (type 0)
   int flags;  // bit h: half h of the rows uses this tile
   int ncols;  // valid columns (type 1)
+};
+
+struct ItemInfo {
+  int h, qt, kind, sink, window, T;  // T: KV tiles of the item
 };
 
 struct AttnArgs {
@@ -74,6 +96,7 @@ struct AttnArgs {
   int64_t o_hs, o_ts;
   float* lse;
   float scale_log2;
+  unsigned* sched;  // [0] items handed out past the first wave, [1] CTAs finished
   unsigned* status;
   uint64_t wait_limit_ns;
 };
@@ -86,28 +109,35 @@ struct Smem {
   static constexpr int V_OFF = K_OFF + 2 * DS * KSLAB;
   static constexpr int COL_OFF = V_OFF + 2 * DS * KSLAB;   // int [NINFO][BN]
   static constexpr int INFO_OFF = COL_OFF + NINFO * BN * 4;
-  static constexpr int BAR_OFF = INFO_OFF + NINFO * (int)sizeof(StageInfo);
-  static constexpr int NBAR = 20;
+  static constexpr int ITEM_OFF = INFO_OFF + NINFO * (int)sizeof(StageInfo);
+  static constexpr int BAR_OFF = (ITEM_OFF + 2 * (int)sizeof(ItemInfo) + 7) & ~7;
+  static constexpr int NBAR = 25;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BITS_OFF = MISC_OFF + 64;
   static int bytes(int nwords) { return BITS_OFF + 2 * nwords * 4 + 1024; }
 };
 
 // Barrier slots.  Per-buffer barriers (K, V, S, P) complete once per use of their
-// buffer, i.e. once per two tiles; B_ODONE completes once per P.V in order.
-// B_INFO + s completes when StageInfo slot s (and its column list) is written.
+// buffer, i.e. once per two tiles; B_ODONE completes once per P.V in order; Q
+// and O barriers once per item; B_INFO + s when StageInfo slot s (and its column
+// list) is written; B_ITEMFULL / B_ITEMFREE + s guard ItemInfo slot s.
 enum {
   B_QFULL = 0,
-  B_KFULL = 1,    // +2
-  B_KEMPTY = 3,   // +2
-  B_VFULL = 5,    // +2
-  B_VEMPTY = 7,   // +2
-  B_SFULL = 9,    // +2
-  B_PFULL = 11,   // +2
-  B_ODONE = 13,
-  B_DRAIN = 14,
-  B_INFO = 15     // +NINFO
+  B_QEMPTY = 1,
+  B_KFULL = 2,     // +2
+  B_KEMPTY = 4,    // +2
+  B_VFULL = 6,     // +2
+  B_VEMPTY = 8,    // +2
+  B_SFULL = 10,    // +2
+  B_PFULL = 12,    // +2
+  B_ODONE = 14,
+  B_OREADY = 15,
+  B_DRAIN = 16,
+  B_ITEMFULL = 17,  // +2
+  B_ITEMFREE = 19,  // +2
+  B_INFO = 21       // +NINFO
 };
+static_assert(B_INFO + NINFO <= 25, "barrier slots");
 
 // One lane waits, the whole warp learns the outcome (keeps warp-collective
 // tcgen05 and shuffle instructions converged even when a wait runs out).
@@ -145,14 +175,15 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float
 // 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted for this
 // library to minimise the relative error on [-1/2, 1/2] (max 7.5e-5, far below the
 // bf16 rounding of P); 2^j is added to the exponent field.  x is clamped at -125 so
-// that the exponent field stays normal; 2^-125 is negligible next to the row max.
+// that the exponent field stays normal, and inputs below -125 (masked keys are
+// -inf) give exactly 0, like ex2.approx.ftz.
 __device__ __forceinline__ void poly_ex2x2(float x0, float x1, float& y0, float& y1) {
   constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 0.99992807f, c1 = 0.693261f, c2 = 0.24261112f, c3 = 0.05517161f;
-  x0 = fmaxf(x0, -125.f);
-  x1 = fmaxf(x1, -125.f);
+  const float c0x = fmaxf(x0, -125.f);
+  const float c1x = fmaxf(x1, -125.f);
   uint64_t xv, sh, yv, jv, fv, pv, cv;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(x0), "f"(x1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(c0x), "f"(c1x));
   asm("mov.b64 %0, {%1, %1};" : "=l"(sh) : "f"(kShift));
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(yv) : "l"(xv), "l"(sh));   // y = x + shift
   asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(jv) : "l"(yv), "l"(sh));   // j = round(x)
@@ -167,8 +198,8 @@ __device__ __forceinline__ void poly_ex2x2(float x0, float x1, float& y0, float&
   uint32_t p0, p1, j0, j1;
   asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(pv));
   asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(yv));
-  y0 = __uint_as_float(p0 + (j0 << 23));
-  y1 = __uint_as_float(p1 + (j1 << 23));
+  y0 = x0 > -125.f ? __uint_as_float(p0 + (j0 << 23)) : 0.f;
+  y1 = x1 > -125.f ? __uint_as_float(p1 + (j1 << 23)) : 0.f;
 }
 
 __device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
@@ -198,8 +229,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-                   const __grid_constant__ AttnArgs a) {
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
   using L = Smem<D>;
   constexpr int DS = L::DS;
   extern __shared__ uint8_t smem_raw[];
@@ -207,364 +237,456 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
   int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
   // misc: [0] tmem base, [2] abort, [3] unit count, [4] col count half0, [5] col count half1,
-  //       [6] col base half0, [7] col base half1, [8] shared-list flag, [9] loader go flag
+  //       [6] col base half0, [7] col base half1, [9] loader go flag, [10] current item
   volatile int* abort_flag = misc + 2;
   uint32_t* bits0 = reinterpret_cast<uint32_t*>(sm + L::BITS_OFF);
   uint32_t* bits1 = bits0 + a.nwords;
   StageInfo* info = reinterpret_cast<StageInfo*>(sm + L::INFO_OFF);
+  ItemInfo* items = reinterpret_cast<ItemInfo*>(sm + L::ITEM_OFF);
   int* colsm = reinterpret_cast<int*>(sm + L::COL_OFF);
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int bid = blockIdx.x;
-  const int h = bid % a.Hq;
-  const int qt = a.n_qtiles - 1 - bid / a.Hq;  // heaviest (latest) tiles first
-  const int kvh = h / a.G;
-  const int kind = a.head_info[h * 4 + 0];
-  const int sink = a.head_info[h * 4 + 1];
-  const int window = a.head_info[h * 4 + 2];
-  const int row0 = qt * BM;
+  const int n_items = a.n_qtiles * a.Hq;
 
-  // ---------------------------------------------------------------- set-up
+  // ---------------------------------------------------------------- set-up (once per CTA)
   if (tid == 0) {
-    for (int i = 0; i < L::NBAR; ++i) mbar_init(&bars[i], (i == B_PFULL || i == B_PFULL + 1) ? 4u : 1u);
+    for (int i = 0; i < L::NBAR; ++i) {
+      uint32_t cnt = 1;
+      if (i == B_PFULL || i == B_PFULL + 1) cnt = 4;
+      if (i == B_ITEMFREE || i == B_ITEMFREE + 1) cnt = 5;
+      mbar_init(&bars[i], cnt);
+    }
     fence_barrier_init();
     misc[2] = 0;
-    misc[3] = 0;
-    // Q does not depend on the index lists: start its load before reading them
-    tma_prefetch_desc(&tmQ);
-    mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
-    for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
   }
   if (warp == 1) {
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), TMEM_COLS);
     tc_fence_before();
   }
   if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
-    tma_prefetch_desc(&tmO);
   }
-  for (int i = tid; i < 2 * a.nwords; i += NTHREADS) bits0[i] = 0u;
   __syncthreads();
   tc_fence_after();
-
-  // query block and last row of each half
-  int qbh[2], r1h[2];
-  bool live[2];
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    const int r0 = row0 + hh * 64;
-    live[hh] = r0 < a.N;
-    qbh[hh] = r0 / a.B;
-    r1h[hh] = min(a.N - 1, r0 + 63);
-  }
-  const int upb = a.B / UNIT;  // units per block
-  const bool shared_qb = live[1] && (qbh[0] == qbh[1]);
-#pragma unroll
-  for (int hh = 0; hh < 2; ++hh) {
-    if (!live[hh]) continue;
-    uint32_t* bits = hh ? bits1 : bits0;
-    const int qb = qbh[hh];
-    const int r1 = r1h[hh];
-    if (kind == DSA_KIND_VS) {
-      const int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
-      for (int e = beg + tid; e < end; e += NTHREADS) {
-        const int delta = a.dist[e];
-        if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
-        if (delta > qb) continue;
-        const int kb = qb - delta;
-        for (int u = kb * upb; u < kb * upb + upb; ++u)
-          if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
-      }
-    } else {
-      const int r = h * a.nqb + qb;
-      const int beg = a.blk_ptr[r], end = a.blk_ptr[r + 1];
-      for (int e = beg + tid; e < end; e += NTHREADS) {
-        const int kb = a.blk_idx[e];
-        if (kb < 0 || kb >= a.nqb) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_BLOCK); continue; }
-        for (int u = kb * upb; u < kb * upb + upb; ++u)
-          if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
-      }
-    }
-  }
-  __syncthreads();
-  {
-    int cnt = 0;
-    for (int w = tid; w < a.nwords; w += NTHREADS) cnt += __popc(bits0[w] | bits1[w]);
-    cnt = warp_sum_int(cnt);
-    if (lane == 0 && cnt) atomicAdd(&misc[3], cnt);
-  }
-  if (tid == 0) {
-    int c0 = 0, c1 = 0, b0 = 0, b1 = 0;
-    if (live[0]) {
-      const int r = h * a.nqb + qbh[0];
-      b0 = a.col_ptr[r];
-      c0 = a.col_ptr[r + 1] - b0;
-    }
-    if (live[1] && !shared_qb) {
-      const int r = h * a.nqb + qbh[1];
-      b1 = a.col_ptr[r];
-      c1 = a.col_ptr[r + 1] - b1;
-    }
-    misc[4] = c0; misc[5] = c1; misc[6] = b0; misc[7] = b1; misc[8] = shared_qb ? 1 : 0;
-  }
-  __syncthreads();
-  const int T_u = misc[3];  // one tile per unit
-  const int ccount[2] = {max(0, misc[4]), max(0, misc[5])};
-  const int cbase[2] = {misc[6], misc[7]};
-  const int cflags[2] = {misc[8] ? 3 : 1, 2};
-  const int T_c0 = ceil_div(ccount[0], BN), T_c1 = ceil_div(ccount[1], BN);
-  const int T = T_u + T_c0 + T_c1;
 
   const uint32_t tmem_base = static_cast<uint32_t>(misc[0]);
   const uint32_t tmem_O = tmem_base;
   const uint64_t limit = a.wait_limit_ns;
+  const int upb = a.B / UNIT;  // units per block
 
   if (warp == 0 || warp == 2 || warp == 3) {
     // ------------------------------------------------------------ loaders
+    // Work items (query tile, head) are dealt round-robin over the CTAs, latest
+    // (heaviest) tiles first.  While the MMA and softmax warps still work on one
+    // item, these warps already read the next item's lists and start its loads.
     const int ltid = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
-    if (warp == 0 && lane == 0) {
-      int w = 0;
-      uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
-      for (int t = 0; t < T_u; ++t) {
-        const int b = t & 1;
-        const uint32_t use = (t >> 1) & 1;
-        if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
-        while (pend == 0u && w + 1 < a.nwords) {
-          ++w;
-          pend = bits0[w] | bits1[w];
-        }
-        const int bit = __ffs(pend) - 1;  // T_u counts exactly the set bits
-        pend &= pend - 1u;
-        const int u = w * 32 + bit;
-        StageInfo& si = info[t % NINFO];
-        si.type = 0;
-        si.u = u;
-        si.flags = (int)((bits0[w] >> bit) & 1u) | ((int)((bits1[w] >> bit) & 1u) << 1);
-        si.ncols = 0;
-        mbar_arrive(&bars[B_INFO + t % NINFO]);
-        uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
-        uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
-        mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
-        for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, kvh);
-        if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
-        for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, kvh);
-      }
-    }
-    __syncwarp();
-    // column tiles: all 96 loader threads gather rows into the swizzled layout
-    int t = T_u;
+    // The first item of a CTA is its block index; later ones come from a global
+    // counter (dynamic: items differ a lot in cost), fetched one item ahead.
+    int tg = 0;     // tiles of earlier items
+    int kc = 0;     // items of this CTA so far
     bool go = true;
-    for (int hh = 0; go && hh < 2; ++hh) {
-      const int nt = hh ? T_c1 : T_c0;
-      for (int ct = 0; ct < nt; ++ct, ++t) {
-        const int b = t & 1;
-        const uint32_t use = (t >> 1) & 1;
+    int next_item = 0;
+    for (;; ++kc) {
+      if (ltid == 0) {
+        misc[10] = kc == 0 ? (int)blockIdx.x : next_item;
+        next_item = (int)gridDim.x + (int)atomicAdd(a.sched, 1u);
+      }
+      // every loader thread is done with the previous item's bitmaps and counts
+      named_barrier(1, 96);
+      const int item = misc[10];
+      if (!go || item >= n_items) {
+        // no more work: tell the MMA and softmax warps (ItemInfo with T = -1)
         if (ltid == 0) {
-          bool ok = mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
-          ok = ok && mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag);
-          misc[9] = ok ? 1 : 0;
-        }
-        named_barrier(1, 96);
-        if (misc[9] == 0) { go = false; break; }
-        const int first = cbase[hh] + ct * BN;
-        const int nc = min(BN, ccount[hh] - ct * BN);
-        int* cj = colsm + (t % NINFO) * BN;
-        uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
-        uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
-        constexpr int CH = D / 8;  // 16-byte chunks per row
-        for (int i = ltid; i < BN * CH; i += 96) {
-          const int slot = i / CH;
-          const int ch = i % CH;
-          int j = (slot < nc) ? a.col_idx[first + slot] : -1;
-          if (slot < nc && (j < 0 || j >= a.N)) {
-            report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_COL);
-            j = -1;
+          const int slot = kc & 1;
+          if (kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
+                                  DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
+            items[slot].T = -1;
+            mbar_arrive(&bars[B_ITEMFULL + slot]);
           }
-          if (ch == 0) {
-            // bit 24 / 25: the column's block is already kept for half 0 / half 1,
-            // so that half must not count the key a second time
-            int v = j;
-            if (j >= 0) {
-              const int u = j / UNIT;
-              const int cov = (int)((bits0[u >> 5] >> (u & 31)) & 1u) | ((int)((bits1[u >> 5] >> (u & 31)) & 1u) << 1);
-              v = j | (cov << 24);
-            }
-            cj[slot] = v;
-          }
-          const int jr = j < 0 ? 0 : j;
-          const uint4 kv = __ldg(reinterpret_cast<const uint4*>(a.K + kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
-          const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.V + kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
-          const uint32_t off = (ch >> 3) * KSLAB + swz(slot, ch & 7);
-          *reinterpret_cast<uint4*>(kst + off) = kv;
-          *reinterpret_cast<uint4*>(vst + off) = vv;
         }
-        fence_proxy_async_smem();
-        named_barrier(1, 96);
-        if (ltid == 0) {
-          StageInfo& si = info[t % NINFO];
-          si.type = 1;
-          si.u = -1;
-          si.flags = cflags[hh];
-          si.ncols = nc;
-          mbar_arrive(&bars[B_INFO + t % NINFO]);
-          mbar_arrive(&bars[B_KFULL + b]);
-          mbar_arrive(&bars[B_VFULL + b]);
+        break;
+      }
+      const int h = item % a.Hq;
+      const int qt = a.n_qtiles - 1 - item / a.Hq;
+      const int kvh = h / a.G;
+      const int row0 = qt * BM;
+      const int kind = a.head_info[h * 4 + 0];
+      for (int i = ltid; i < 2 * a.nwords; i += 96) bits0[i] = 0u;
+      if (ltid == 0) misc[3] = 0;
+      int qbh[2], r1h[2];
+      bool live[2];
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int r0 = row0 + hh * 64;
+        live[hh] = r0 < a.N;
+        qbh[hh] = r0 / a.B;
+        r1h[hh] = min(a.N - 1, r0 + 63);
+      }
+      const bool shared_qb = live[1] && (qbh[0] == qbh[1]);
+      named_barrier(1, 96);
+      if (ltid == 32) {
+        // column lists: independent of the block lists, read in parallel with them
+        int c0 = 0, c1 = 0, b0 = 0, b1 = 0;
+        if (live[0]) {
+          const int r = h * a.nqb + qbh[0];
+          b0 = a.col_ptr[r];
+          c0 = a.col_ptr[r + 1] - b0;
+        }
+        if (live[1] && !shared_qb) {
+          const int r = h * a.nqb + qbh[1];
+          b1 = a.col_ptr[r];
+          c1 = a.col_ptr[r + 1] - b1;
+        }
+        misc[4] = c0; misc[5] = c1; misc[6] = b0; misc[7] = b1;
+      }
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        if (!live[hh]) continue;
+        uint32_t* bits = hh ? bits1 : bits0;
+        const int qb = qbh[hh];
+        const int r1 = r1h[hh];
+        if (kind == DSA_KIND_VS) {
+          const int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
+          for (int e = beg + ltid; e < end; e += 96) {
+            const int delta = a.dist[e];
+            if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
+            if (delta > qb) continue;
+            const int kb = qb - delta;
+            for (int u = kb * upb; u < kb * upb + upb; ++u)
+              if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
+          }
+        } else {
+          const int r = h * a.nqb + qb;
+          const int beg = a.blk_ptr[r], end = a.blk_ptr[r + 1];
+          for (int e = beg + ltid; e < end; e += 96) {
+            const int kb = a.blk_idx[e];
+            if (kb < 0 || kb >= a.nqb) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_BLOCK); continue; }
+            for (int u = kb * upb; u < kb * upb + upb; ++u)
+              if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
+          }
         }
       }
+      named_barrier(1, 96);
+      {
+        int cnt = 0;
+        for (int w = ltid; w < a.nwords; w += 96) cnt += __popc(bits0[w] | bits1[w]);
+        cnt = warp_sum_int(cnt);
+        if (lane == 0 && cnt) atomicAdd(&misc[3], cnt);
+      }
+      named_barrier(1, 96);
+      const int T_u = misc[3];  // one tile per unit
+      const int ccount[2] = {max(0, misc[4]), max(0, misc[5])};
+      const int cbase[2] = {misc[6], misc[7]};
+      const int cflags[2] = {shared_qb ? 3 : 1, 2};
+      const int T_c0 = ceil_div(ccount[0], BN), T_c1 = ceil_div(ccount[1], BN);
+      const int T = T_u + T_c0 + T_c1;
+      if (ltid == 0) {
+        // publish the item (its slot is free once both consumers read item kc - 2),
+        // then load its Q once every Q K^T of the previous item has finished
+        const int slot = kc & 1;
+        bool ok = kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
+                                      DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+        if (ok) {
+          ItemInfo& it = items[slot];
+          it.h = h;
+          it.qt = qt;
+          it.kind = kind;
+          it.sink = a.head_info[h * 4 + 1];
+          it.window = a.head_info[h * 4 + 2];
+          it.T = T;
+          mbar_arrive(&bars[B_ITEMFULL + slot]);
+        }
+        ok = ok && (kc == 0 || mbar_wait(&bars[B_QEMPTY], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kLoaderSuspend));
+        if (ok) {
+          mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
+          for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
+        }
+        misc[9] = ok ? 1 : 0;
+      }
+      named_barrier(1, 96);
+      if (misc[9] == 0) { go = false; continue; }
+      if (warp == 0 && lane == 0) {
+        int w = 0;
+        uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
+        for (int t = 0; t < T_u; ++t) {
+          const int g = tg + t;
+          const int b = g & 1;
+          const uint32_t use = (g >> 1) & 1;
+          if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) break;
+          while (pend == 0u && w + 1 < a.nwords) {
+            ++w;
+            pend = bits0[w] | bits1[w];
+          }
+          const int bit = __ffs(pend) - 1;  // T_u counts exactly the set bits
+          pend &= pend - 1u;
+          const int u = w * 32 + bit;
+          StageInfo& si = info[g % NINFO];
+          si.type = 0;
+          si.u = u;
+          si.flags = (int)((bits0[w] >> bit) & 1u) | ((int)((bits1[w] >> bit) & 1u) << 1);
+          si.ncols = 0;
+          mbar_arrive(&bars[B_INFO + g % NINFO]);
+          uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+          uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
+          mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
+          for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, kvh);
+          if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) break;
+          mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
+          for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, kvh);
+        }
+      }
+      __syncwarp();
+      // column tiles: all 96 loader threads gather rows into the swizzled layout
+      int t = T_u;
+      for (int hh = 0; go && hh < 2; ++hh) {
+        const int nt = hh ? T_c1 : T_c0;
+        for (int ct = 0; ct < nt; ++ct, ++t) {
+          const int g = tg + t;
+          const int b = g & 1;
+          const uint32_t use = (g >> 1) & 1;
+          if (ltid == 0) {
+            bool ok = mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+            ok = ok && mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+            misc[9] = ok ? 1 : 0;
+          }
+          named_barrier(1, 96);
+          if (misc[9] == 0) { go = false; break; }
+          const int first = cbase[hh] + ct * BN;
+          const int nc = min(BN, ccount[hh] - ct * BN);
+          int* cj = colsm + (g % NINFO) * BN;
+          uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+          uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
+          constexpr int CH = D / 8;  // 16-byte chunks per row
+          for (int i = ltid; i < BN * CH; i += 96) {
+            const int slot = i / CH;
+            const int ch = i % CH;
+            int j = (slot < nc) ? a.col_idx[first + slot] : -1;
+            if (slot < nc && (j < 0 || j >= a.N)) {
+              report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_COL);
+              j = -1;
+            }
+            if (ch == 0) {
+              // bit 24 / 25: the column's block is already kept for half 0 / half 1,
+              // so that half must not count the key a second time
+              int v = j;
+              if (j >= 0) {
+                const int u = j / UNIT;
+                const int cov =
+                    (int)((bits0[u >> 5] >> (u & 31)) & 1u) | ((int)((bits1[u >> 5] >> (u & 31)) & 1u) << 1);
+                v = j | (cov << 24);
+              }
+              cj[slot] = v;
+            }
+            const int jr = j < 0 ? 0 : j;
+            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(a.K + kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
+            const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.V + kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
+            const uint32_t off = (ch >> 3) * KSLAB + swz(slot, ch & 7);
+            *reinterpret_cast<uint4*>(kst + off) = kv;
+            *reinterpret_cast<uint4*>(vst + off) = vv;
+          }
+          fence_proxy_async_smem();
+          named_barrier(1, 96);
+          if (ltid == 0) {
+            StageInfo& si = info[g % NINFO];
+            si.type = 1;
+            si.u = -1;
+            si.flags = cflags[hh];
+            si.ncols = nc;
+            mbar_arrive(&bars[B_INFO + g % NINFO]);
+            mbar_arrive(&bars[B_KFULL + b]);
+            mbar_arrive(&bars[B_VFULL + b]);
+          }
+        }
+      }
+      __syncwarp();
+      tg += T;
     }
-    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
       const uint32_t q_addr = smem_u32(sm + L::Q_OFF);
-      bool ok = mbar_wait(&bars[B_QFULL], 0, limit, a.status, DETAIL_WAIT_Q, abort_flag);
-      for (int t = 0; ok && t <= T; ++t) {
-        if (t < T) {
-          // S(t) = Q K(t)^T into S buffer t & 1
-          const int b = t & 1;
-          const uint32_t use = (t >> 1) & 1;
-          if (!mbar_wait(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag)) break;
-          // the buffer still holds P(t-2) until that P.V has finished
-          if (t >= 2 && !mbar_wait(&bars[B_ODONE], t & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(sm + L::K_OFF + b * DS * KSLAB);
-          const uint32_t s_tmem = tmem_base + S_COL + 64 * b;
+      bool ok = true;
+      int tg = 0;
+      for (int kc = 0; ok; ++kc) {
+        const int slot = kc & 1;
+        if (!mbar_wait(&bars[B_ITEMFULL + slot], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
+        const int T = items[slot].T;
+        mbar_arrive(&bars[B_ITEMFREE + slot]);
+        if (T < 0) break;  // no more items
+        if (!mbar_wait(&bars[B_QFULL], kc & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
+        if (T == 0) tc_commit(&bars[B_QEMPTY]);
+        for (int t = 0; t <= T; ++t) {
+          if (t < T) {
+            // S(g) = Q K(g)^T into S buffer g & 1
+            const int g = tg + t;
+            const int b = g & 1;
+            const uint32_t use = (g >> 1) & 1;
+            if (!mbar_wait(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag, kMmaSuspend)) { ok = false; break; }
+            // the buffer still holds P(g-2) until that P.V has finished; its
+            // V-empty commit says so (a per-buffer barrier: at an item boundary
+            // P(g-1) V(g-1) has been issued too, so B_ODONE could be two phases on)
+            if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t k_addr = smem_u32(sm + L::K_OFF + b * DS * KSLAB);
+            const uint32_t s_tmem = tmem_base + S_COL + 64 * b;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t ad = smem_desc(q_addr + (kk >> 2) * QSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            const uint64_t bd = smem_desc(k_addr + (kk >> 2) * KSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-            tc_mma_f16(s_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint64_t ad = smem_desc(q_addr + (kk >> 2) * QSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
+              const uint64_t bd = smem_desc(k_addr + (kk >> 2) * KSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
+              tc_mma_f16(s_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
+            }
+            tc_commit(&bars[B_SFULL + b]);
+            tc_commit(&bars[B_KEMPTY + b]);
+            if (t == T - 1) tc_commit(&bars[B_QEMPTY]);  // Q may be replaced by the next item's
           }
-          tc_commit(&bars[B_SFULL + b]);
-          tc_commit(&bars[B_KEMPTY + b]);
-        }
-        if (t >= 1) {
-          // O += P(t-1) V(t-1)
-          const int u = t - 1;
-          const int b = u & 1;
-          const uint32_t use = (u >> 1) & 1;
-          if (!mbar_wait(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag)) break;
-          if (!mbar_wait(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag)) break;
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(sm + L::V_OFF + b * DS * KSLAB);
-          const uint32_t p_tmem = tmem_base + S_COL + 64 * b;
+          if (t >= 1) {
+            // O += P(g-1) V(g-1); the item's first P.V overwrites O
+            const int u = t - 1;
+            const int g = tg + u;
+            const int b = g & 1;
+            const uint32_t use = (g >> 1) & 1;
+            if (!mbar_wait(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag, kMmaSuspend)) { ok = false; break; }
+            if (!mbar_wait(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag, kMmaSuspend)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t v_addr = smem_u32(sm + L::V_OFF + b * DS * KSLAB);
+            const uint32_t p_tmem = tmem_base + S_COL + 64 * b;
 #pragma unroll
-          for (int kk = 0; kk < BN / 16; ++kk) {
-            const uint64_t bd = smem_desc(v_addr + kk * 2048, KSLAB, 1024, SWZ_128B);
-            tc_mma_ts(tmem_O, p_tmem + kk * 8, bd, IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < BN / 16; ++kk) {
+              const uint64_t bd = smem_desc(v_addr + kk * 2048, KSLAB, 1024, SWZ_128B);
+              tc_mma_ts(tmem_O, p_tmem + kk * 8, bd, IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
+            }
+            tc_commit(&bars[B_ODONE]);
+            tc_commit(&bars[B_VEMPTY + b]);
           }
-          tc_commit(&bars[B_ODONE]);
-          tc_commit(&bars[B_VEMPTY + b]);
         }
+        if (ok && T > 0) tc_commit(&bars[B_OREADY]);  // the item's O is final once this completes
+        tg += T;
       }
       // drain every MMA this thread issued before TMEM is released
       tc_commit(&bars[B_DRAIN]);
-      mbar_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag);
+      mbar_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
     const int q4 = warp & 3;           // TMEM lane quadrant of this warp
     const int r = q4 * 32 + lane;      // row within the tile == TMEM lane
-    const int row = row0 + r;
     const int half = r >> 6;
     const int hbit = 1 << half;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
-    float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int t = 0; t < T; ++t) {
-      const int b = t & 1;
-      const uint32_t use = (t >> 1) & 1;
-      const int slot = t % NINFO;
-      if (!warp_wait(&bars[B_INFO + slot], (t / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
-        ok = false;
-        break;
-      }
-      const StageInfo si = info[slot];
-      // allowed-key bits of this row, 32 columns per word
-      uint32_t mw[2];
-      if (si.type == 0) {
-        const bool oks = (si.flags & hbit) != 0;
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const int j0 = si.u * UNIT + k * 32;
-          uint32_t bits = oks ? low_bits(row - j0 + 1) : 0u;
-          if (kind == DSA_KIND_ASHAPE) bits &= low_bits(sink - j0) | ~low_bits(row - window + 1 - j0);
-          mw[k] = bits;
+    int tg = 0, nready = 0;
+    for (int kc = 0; ok; ++kc) {
+      const int islot = kc & 1;
+      if (!warp_wait(&bars[B_ITEMFULL + islot], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag)) break;
+      const ItemInfo it = items[islot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[B_ITEMFREE + islot]);
+      if (it.T < 0) break;  // no more items
+      const int T = it.T;
+      const int kind = it.kind;
+      const int sink = it.sink;
+      const int window = it.window;
+      const int row = it.qt * BM + r;
+      float m = -INFINITY, l = 0.f;
+      for (int t = 0; t < T; ++t) {
+        const int g = tg + t;
+        const int b = g & 1;
+        const uint32_t use = (g >> 1) & 1;
+        const int slot = g % NINFO;
+        if (!warp_wait(&bars[B_INFO + slot], (g / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
+          ok = false;
+          break;
         }
-      } else {
-        const int* cj = colsm + slot * BN;
-        const bool okh = (si.flags & hbit) != 0;
+        const StageInfo si = info[slot];
+        // allowed-key bits of this row, 32 columns per word
+        uint32_t mw[2];
+        if (si.type == 0) {
+          const bool oks = (si.flags & hbit) != 0;
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          uint32_t bits = 0u;
-#pragma unroll 8
-          for (int i = 0; i < 32; ++i) {
-            const int v = cj[k * 32 + i];
-            const bool al = okh && (k * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
-                            ((v & 0xFFFFFF) <= row);
-            bits |= (al ? 1u : 0u) << i;
+          for (int k = 0; k < 2; ++k) {
+            const int j0 = si.u * UNIT + k * 32;
+            uint32_t bits = oks ? low_bits(row - j0 + 1) : 0u;
+            if (kind == DSA_KIND_ASHAPE) bits &= low_bits(sink - j0) | ~low_bits(row - window + 1 - j0);
+            mw[k] = bits;
           }
-          mw[k] = bits;
+        } else {
+          const int* cj = colsm + slot * BN;
+          const bool okh = (si.flags & hbit) != 0;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            uint32_t bits = 0u;
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+              const int v = cj[k * 32 + i];
+              const bool al = okh && (k * 32 + i < si.ncols) && (v >= 0) && !((v >> (24 + half)) & 1) &&
+                              ((v & 0xFFFFFF) <= row);
+              bits |= (al ? 1u : 0u) << i;
+            }
+            mw[k] = bits;
+          }
         }
-      }
-      if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
-      float s[64];
-      tmem_ld32(s_t, s);
-      tmem_ld32(s_t + 32, s + 32);
-      tmem_wait_ld();
-      // fully visible tile for the whole warp: no per-element masking
-      const bool full = __all_sync(0xffffffffu, (mw[0] & mw[1]) == 0xffffffffu);
-      // tile max of the allowed raw scores (independent partial maxima)
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      if (full) {
+        if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
+        float s[64];
+        tmem_ld32(s_t, s);
+        tmem_ld32(s_t + 32, s + 32);
+        tmem_wait_ld();
+        // masked keys become -inf, so one code path serves every tile (exp2 of
+        // -inf is 0); a tile the whole warp sees fully skips even that
+        if (!__all_sync(0xffffffffu, (mw[0] & mw[1]) == 0xffffffffu)) {
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) s[k * 32 + i] = ((mw[k] >> i) & 1u) ? s[k * 32 + i] : -INFINITY;
+          }
+        }
+        // tile max of the allowed raw scores (independent partial maxima)
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const uint32_t bits = mw[k];
-#pragma unroll
-          for (int i = 0; i < 32; ++i) mx[i & 3] = fmaxf(mx[i & 3], ((bits >> i) & 1u) ? s[k * 32 + i] : -INFINITY);
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+        const float m_new = fmaxf(m, mt * a.scale_log2);
+        const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
+        float alpha = 1.f;
+        if (need) {
+          alpha = fast_ex2(m - m_new);
+          l *= alpha;
+          m = m_new;
         }
-      }
-      const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
-      const float m_new = fmaxf(m, mt * a.scale_log2);
-      const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
-      float alpha = 1.f;
-      if (need) {
-        alpha = fast_ex2(m - m_new);
-        l *= alpha;
-        m = m_new;
-      }
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
-        // O must hold every P.V so far before it is rescaled: wait for P(t-1) V(t-1)
-        if (!warp_wait(&bars[B_ODONE], (t - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t o_t = tmem_O + lane_off;
+        if (t > 0 && __any_sync(0xffffffffu, need)) {
+          // O must hold every P.V of the item so far before it is rescaled: wait
+          // for P(g-1) V(g-1)
+          if (!warp_wait(&bars[B_ODONE], (g - 1) & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t o_t = tmem_O + lane_off;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          float o[32];
-          tmem_ld32(o_t + c * 32, o);
-          tmem_wait_ld();
+          for (int c = 0; c < D / 32; ++c) {
+            float o[32];
+            tmem_ld32(o_t + c * 32, o);
+            tmem_wait_ld();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] *= alpha;
-          tmem_st32(o_t + c * 32, o);
+            for (int i = 0; i < 32; ++i) o[i] *= alpha;
+            tmem_st32(o_t + c * 32, o);
+          }
         }
-      }
-      // P = exp2(s * scale - m) as bf16 pairs over the first 32 columns of the buffer
-      const bool dead = (m == -INFINITY);
-      const float negm = dead ? 0.f : -m;
-      float ls[4] = {0.f, 0.f, 0.f, 0.f};
-      if (full && !dead) {
+        // P = exp2(s * scale - m) as bf16 pairs over the first 32 columns of the
+        // buffer.  A row with no allowed key so far (m = -inf) keeps x = -inf.
+        const float negm = (m == -INFINITY) ? 0.f : -m;
+        float ls[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
           uint32_t pk[16];
@@ -584,75 +706,54 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
           tmem_st16(s_t + k * 16, pk);
         }
-      } else {
+        l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+      }
+      // epilogue.  The MMA thread commits B_OREADY once per item with tiles,
+      // after the item's last P.V; O is read out of TMEM before this warp
+      // produces the next item's first P, which is what lets that item's first
+      // P.V overwrite it.
+      const bool have = ok && T > 0;
+      if (have) {
+        if (!warp_wait(&bars[B_OREADY], nready & 1, limit, a.status, DETAIL_WAIT_O, abort_flag)) ok = false;
+        ++nready;
+        tc_fence_after();
+      }
+      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      const bool in = row < a.N;
+      __nv_bfloat16* orow = a.O + (int64_t)it.h * a.o_hs + (int64_t)(in ? row : 0) * a.o_ts;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        float o[32];
+        if (have && ok) {
+          tmem_ld32(tmem_O + lane_off + c * 32, o);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int k = 0; k < 2; ++k) {
-          const uint32_t bits = dead ? 0u : mw[k];
-          uint32_t pk[16];
+          for (int i = 0; i < 32; ++i) o[i] = 0.f;
+        }
+        if (in) {
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float x0, x1;
-            fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
-            const float p0 = ((bits >> (2 * i)) & 1u) ? fast_ex2(x0) : 0.f;
-            const float p1 = ((bits >> (2 * i + 1)) & 1u) ? fast_ex2(x1) : 0.f;
-            ls[i & 3] += p0 + p1;
-            __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
-            pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+          for (int v = 0; v < 4; ++v) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              __nv_bfloat162 v2 = __floats2bfloat162_rn(o[v * 8 + 2 * i] * inv, o[v * 8 + 2 * i + 1] * inv);
+              pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+            }
+            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           }
-          tmem_st16(s_t + k * 16, pk);
         }
       }
-      l += (ls[0] + ls[1]) + (ls[2] + ls[3]);
-      tmem_wait_st();
+      if (a.lse != nullptr && in)
+        a.lse[(int64_t)it.h * a.N + row] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[B_PFULL + b]);
+      tg += T;
     }
-    // epilogue.  The softmax does not follow every P.V, so the P.V-done barrier
-    // may be a phase behind here; the drain barrier, committed by the MMA thread
-    // after its last MMA, is the one that says O is final.
-    const bool have = ok && T > 0;
-    if (have) {
-      if (!warp_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag)) ok = false;
-      tc_fence_after();
-    }
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
-    // O / l as bf16 into shared memory (the K buffers, idle once every MMA has
-    // finished) in the 128-byte-swizzled layout of the O tensor map, then one TMA
-    // store per 64 columns; rows past N are clipped by the map
-    uint8_t* ost = sm + L::K_OFF;
-#pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
-      float o[32];
-      if (have && ok) {
-        tmem_ld32(tmem_O + lane_off + c * 32, o);
-        tmem_wait_ld();
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0.f;
-      }
-#pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        uint32_t pk[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          __nv_bfloat162 v2 = __floats2bfloat162_rn(o[v * 8 + 2 * i] * inv, o[v * 8 + 2 * i + 1] * inv);
-          pk[i] = *reinterpret_cast<uint32_t*>(&v2);
-        }
-        *reinterpret_cast<uint4*>(ost + (c >> 1) * QSLAB + swz(r, (c & 1) * 4 + v)) =
-            make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      }
-    }
-    fence_proxy_async_smem();
-    named_barrier(2, 128);  // the four softmax warps
-    if (r == 0) {
-      for (int c = 0; c < DS; ++c) tma_store_3d(&tmO, ost + c * QSLAB, c * 64, row0, h);
-      tma_store_commit();
-      tma_store_wait_read();
-    }
-    if (a.lse != nullptr && row < a.N)
-      a.lse[(int64_t)h * a.N + row] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-    __syncwarp();
   }
 
   // ---------------------------------------------------------------- teardown
@@ -662,11 +763,40 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  if (tid == 0) {
+    // the last CTA out zeroes the item counter for the next launch that uses it
+    __threadfence();
+    if (atomicAdd(a.sched + 1, 1u) == gridDim.x - 1) {
+      a.sched[0] = 0u;
+      a.sched[1] = 0u;
+      __threadfence();
+    }
+  }
 }
 
 // --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
+// Item counters of the persistent attention kernel: one pair per launch, taken
+// round-robin from a pool so that launches in flight on different streams do not
+// share one (up to kSchedSlots of them); each launch leaves its pair at zero.
+constexpr int kSchedSlots = 64;
+__device__ unsigned g_sched[2 * kSchedSlots];
+
+unsigned* sched_slot() {
+  constexpr int kMaxDev = 64;
+  static unsigned* base[kMaxDev] = {};
+  static std::atomic<unsigned> next{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+  if (base[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_sched) != cudaSuccess) return nullptr;
+    base[dev] = static_cast<unsigned*>(p);
+  }
+  return base[dev] + 2 * (next.fetch_add(1u) % kSchedSlots);
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (fn == nullptr) {
@@ -698,9 +828,8 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int H, int64_t t
 template <int D>
 dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const void* V, const dsa_indices& idx,
                     void* O, float* lse, cudaStream_t stream, unsigned* status) {
-  CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mo, O, D, p.N, p.Hq, p.o_token_stride, p.o_head_stride, BM) ||
-      !make_map(&mq, Q, D, p.N, p.Hq, p.q_token_stride, p.q_head_stride, BM) ||
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, D, p.N, p.Hq, p.q_token_stride, p.q_head_stride, BM) ||
       !make_map(&mk, K, D, p.N, p.Hkv, p.k_token_stride, p.k_head_stride, UNIT) ||
       !make_map(&mv, V, D, p.N, p.Hkv, p.v_token_stride, p.v_head_stride, UNIT))
     return DSA_ERR_CUDA;
@@ -732,15 +861,23 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   a.lse = lse;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   a.status = status;
+  a.sched = sched_slot();
+  if (a.sched == nullptr) return DSA_ERR_CUDA;
   a.wait_limit_ns = kWaitLimitNs;
   int smem = Smem<D>::bytes(a.nwords);
   // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
   cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
-  const int grid = a.n_qtiles * p.Hq;
-  if (grid == 0) return DSA_OK;
-  sparse_attn_kernel<D><<<grid, NTHREADS, smem, stream>>>(mq, mk, mv, mo, a);
+  const int n_items = a.n_qtiles * p.Hq;
+  if (n_items == 0) return DSA_OK;
+  // persistent: two CTAs per SM, items dealt round-robin
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const int grid = n_items < 2 * sms ? n_items : 2 * sms;
+  sparse_attn_kernel<D><<<grid, NTHREADS, smem, stream>>>(mq, mk, mv, a);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;

@@ -76,18 +76,34 @@ __device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Blocking probe: the hardware may suspend the thread for a while until the
+// phase completes, so a waiting warp takes no issue slots from the warps that
+// share its scheduler.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_ns` nanoseconds of global time, records DSA_ERR_TIMEOUT with `detail`
 // in the status word, sets *abort (shared flag) and returns false.  Also returns
 // false early if another thread of the block has already set *abort.
+// With `suspend`, the loop blocks in try_wait instead of polling test_wait.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
                                           unsigned* status, unsigned detail,
-                                          volatile int* abort_flag) {
+                                          volatile int* abort_flag, bool suspend = false) {
   if (mbar_test_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t spins = 0;
   while (true) {
-    if (mbar_test_wait(bar, parity)) return true;
+    if (suspend ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
     if (((++spins) & 63u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
