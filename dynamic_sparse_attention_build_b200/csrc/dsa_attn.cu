@@ -9,7 +9,7 @@
 // for A-shape heads only those with j < sink or i - j < window.
 //
 // Design (persistent: two CTAs per SM; a work item = 128 query rows of one head,
-// items dealt round-robin over the CTAs, latest (heaviest) query tiles first):
+// items handed out by a global counter, latest (heaviest) query tiles first):
 //   * the tile's two 64-row halves each belong to one query block (two different
 //     blocks when B = 64, the same block otherwise).  Their key lists become two
 //     bitmaps over 64-key units in shared memory; the union is walked in
@@ -94,6 +94,7 @@ struct AttnArgs {
   int64_t k_hs, k_ts, v_hs, v_ts;
   __nv_bfloat16* O;
   int64_t o_hs, o_ts;
+  int o_v8;  // O rows are 32-byte aligned: 256-bit stores
   float* lse;
   float scale_log2;
   unsigned* sched;  // [0] items handed out past the first wave, [1] CTAs finished
@@ -200,6 +201,27 @@ __device__ __forceinline__ void poly_ex2x2(float x0, float x1, float& y0, float&
   asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(yv));
   y0 = x0 > -125.f ? __uint_as_float(p0 + (j0 << 23)) : 0.f;
   y1 = x1 > -125.f ? __uint_as_float(p1 + (j1 << 23)) : 0.f;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (s0, s1) += (a, b) as one packed f32x2 add
+__device__ __forceinline__ void add2(float& s0, float& s1, float a, float b) {
+  uint64_t sv, av;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(sv) : "f"(s0), "f"(s1));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a), "f"(b));
+  asm("add.rn.f32x2 %0, %0, %1;" : "+l"(sv) : "l"(av));
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(s0), "=f"(s1) : "l"(sv));
+}
+
+// 32 bytes to global memory in one store (address 32-byte aligned)
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+               "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
 }
 
 __device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
@@ -411,7 +433,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (misc[9] == 0) { go = false; continue; }
       if (warp == 0 && lane == 0) {
         int w = 0;
-        uint32_t pend = (a.nwords > 0) ? (bits0[0] | bits1[0]) : 0u;
+        uint32_t pend = bits0[0] | bits1[0];
         for (int t = 0; t < T_u; ++t) {
           const int g = tg + t;
           const int b = g & 1;
@@ -654,14 +676,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // tile max of the allowed raw scores (independent partial maxima)
         float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-        for (int i = 0; i < 64; ++i) mx[i & 3] = fmaxf(mx[i & 3], s[i]);
+        for (int i = 0; i < 32; ++i) mx[i & 3] = max3f(mx[i & 3], s[2 * i], s[2 * i + 1]);
         const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
         const float m_new = fmaxf(m, mt * a.scale_log2);
-        const bool need = m_new > m + RESCALE_THRESHOLD;  // also true for the first finite max
+        // the max moves when it grows by more than the threshold or becomes finite
+        // for the first time; O and l only need rescaling in the first case (a
+        // row without a finite max so far has O = 0 and l = 0)
         float alpha = 1.f;
-        if (need) {
-          alpha = fast_ex2(m - m_new);
-          l *= alpha;
+        bool need = false;
+        if (m_new > m + RESCALE_THRESHOLD) {
+          if (m != -INFINITY) {
+            alpha = fast_ex2(m - m_new);
+            l *= alpha;
+            need = true;
+          }
           m = m_new;
         }
         if (t > 0 && __any_sync(0xffffffffu, need)) {
@@ -700,7 +728,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               p0 = fast_ex2(x0);
               p1 = fast_ex2(x1);
             }
-            ls[i & 3] += p0 + p1;
+            add2(ls[(i & 1) * 2], ls[(i & 1) * 2 + 1], p0, p1);
             __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
             pk[i] = *reinterpret_cast<uint32_t*>(&v2);
           }
@@ -736,15 +764,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           for (int i = 0; i < 32; ++i) o[i] = 0.f;
         }
         if (in) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint32_t pk[4];
+          for (int i = 0; i < 16; ++i) {
+            __nv_bfloat162 v2 = __floats2bfloat162_rn(o[2 * i] * inv, o[2 * i + 1] * inv);
+            pk[i] = *reinterpret_cast<uint32_t*>(&v2);
+          }
+          if (a.o_v8) {
+            st_global_v8(orow + c * 32, pk);
+            st_global_v8(orow + c * 32 + 16, pk + 8);
+          } else {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              __nv_bfloat162 v2 = __floats2bfloat162_rn(o[v * 8 + 2 * i] * inv, o[v * 8 + 2 * i + 1] * inv);
-              pk[i] = *reinterpret_cast<uint32_t*>(&v2);
-            }
-            *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            for (int v = 0; v < 4; ++v)
+              *reinterpret_cast<uint4*>(orow + c * 32 + v * 8) = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
       }
@@ -858,6 +890,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   a.O = static_cast<__nv_bfloat16*>(O);
   a.o_hs = p.o_head_stride;
   a.o_ts = p.o_token_stride;
+  a.o_v8 = ((reinterpret_cast<uintptr_t>(O) & 31u) == 0 && p.o_token_stride % 16 == 0 && p.o_head_stride % 16 == 0) ? 1 : 0;
   a.lse = lse;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   a.status = status;
