@@ -203,6 +203,15 @@ def oracle_sample(w, Q, K, V, pats, target_s=15.0):
 
 
 # --------------------------------------------------------------------------- main
+# what each workload's heads do (synth.head_patterns)
+PATTERN_TEXT = {
+    "vs": "all heads Vertical-Slash (last_q 64, n_vert/n_slash per workload)",
+    "mixed": "seeded per head: 20% A-shape 128/1024, 60% VS 64/1000/6096, 20% block top-100",
+    "threshold": "all heads block threshold, alpha 0.5 in probability space, sink and local block kept",
+    "moba": "all heads MoBA top-8 over earlier blocks plus the diagonal block",
+}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -353,7 +362,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
-                   "patterns": "seeded per head: 20% A-shape 128/1024, 60% VS 64/1000/6096, 20% block top-100",
+                   "patterns": PATTERN_TEXT.get(w["mix"], w["mix"]),
                    "l2": "flushed by a 256 MiB write before every timed step (outside its events)",
                    "parallelism": f"independent layer per rank x{world}"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
