@@ -58,7 +58,7 @@ struct ConvTab {
 
 struct Layout {
   int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_nchunks, vs_lmax;
-  int64_t off_qbar, off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, total;
+  int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
@@ -197,41 +197,26 @@ __global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int
 }
 
 // ---------------------------------------------------------------------------
-// mean pooling (+ optional causal depthwise key conv with SiLU and residual)
+// key mean pooling (+ optional causal depthwise key conv with SiLU and residual)
 // ---------------------------------------------------------------------------
-// grid: (nqb, nbh + Hkv); item < nbh pools Q of block slot `item`, else K of KV
-// head item - nbh (skipped unless some block head reads it).
+// grid: (nqb, Hkv); KV heads that no block head reads are skipped.  Queries are
+// pooled inside k_block_select.
 template <int D>
-__global__ void __launch_bounds__(256) k_pool(const __grid_constant__ HeadTab ht, const __grid_constant__ ConvTab ct,
-                                              Layout L, const __nv_bfloat16* Q, int64_t q_hs, int64_t q_ts,
+__global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct, Layout L,
                                               const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws) {
   constexpr int TPR = D / 8;          // threads per row, 8 channels each
   constexpr int RG = 256 / TPR;       // rows in flight
   __shared__ float part[RG][D];
   const int b = blockIdx.x;
-  const int item = blockIdx.y;
-  const bool isq = item < L.nbh;
-  const int kvh = isq ? 0 : item - L.nbh;
-  if (!isq && !ct.need[kvh]) return;
-  const __nv_bfloat16* X;
-  int64_t ts;
-  __nv_bfloat16* out;  // the pooled row as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
-  int W = 0;
-  const float* cw = nullptr;
-  const float* cb = nullptr;
-  if (isq) {
-    const int h = ht.bhead[item];
-    X = Q + h * q_hs;
-    ts = q_ts;
-    out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_qbar) + ((int64_t)item * L.nqb + b) * 2 * D;
-  } else {
-    X = K + kvh * k_hs;
-    ts = k_ts;
-    out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * 2 * D;
-    W = ct.width[kvh];
-    cw = ct.w[kvh];
-    cb = ct.b[kvh];
-  }
+  const int kvh = blockIdx.y;
+  if (!ct.need[kvh]) return;
+  const __nv_bfloat16* X = K + kvh * k_hs;
+  const int64_t ts = k_ts;
+  // the pooled row as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * 2 * D;
+  const int W = ct.width[kvh];
+  const float* cw = ct.w[kvh];
+  const float* cb = ct.b[kvh];
   const int rg = threadIdx.x / TPR;
   const int c0 = (threadIdx.x % TPR) * 8;
   const int r_beg = b * L.B;
@@ -323,6 +308,18 @@ constexpr int SEL_NW = SEL_NT / 32;
 // score row stride in floats: 8 past a multiple of 32 so the 8-byte stores of
 // one half-warp (rows g..g+3, columns 2 t4) hit 16 distinct bank pairs
 __host__ __device__ constexpr int SEL_RS(int npad) { return npad + 8; }
+// query blocks per select CTA: up to 2048 query rows to pool, at most SEL_RI
+inline int sel_blocks_per_cta(int B) {
+  int ri = SEL_RI;
+  while (ri > 1 && ri * B > 2048) ri >>= 1;
+  return ri;
+}
+// dynamic shared memory: the score tile, which first holds the pooling partials
+inline size_t sel_smem_bytes(int D, int nkw) {
+  const size_t scores = (size_t)SEL_RI * SEL_RS(nkw * 32) * 4;
+  const size_t partials = (size_t)(SEL_NT / (D / 8)) * D * 4;
+  return scores > partials ? scores : partials;
+}
 
 // Warp-level exact top-k of vals[0..n) (ties to the lower index), 0 < k < n.
 // hist: this warp's shared int[256].  Returns the k-th largest key and how many
@@ -378,21 +375,25 @@ __device__ void warp_radix_kth(const float* vals, int n, int k, int* hist, uint3
   *take_eq = need;
 }
 
+// ri query blocks per CTA (a power of two, at most SEL_RI): their rows are
+// mean-pooled here, straight from Q (Q-bar never goes to memory), then scored
+// and selected.  Streaming Q is most of the index build's HBM traffic; doing it
+// in the CTAs that also score lets one CTA's selection overlap another's loads.
 template <int D>
-__global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
-                                                      int32_t* blk_ptr) {
+__global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__ HeadTab ht, Layout L,
+                                                      const __nv_bfloat16* Q, int64_t q_hs, int64_t q_ts,
+                                                      uint8_t* ws, int32_t* blk_ptr, int ri) {
   extern __shared__ float sc[];  // [SEL_RI][SEL_RS(npad)] scores of the group's rows
   __shared__ int hist[SEL_NW][256];
   const int npad = L.nkw * 32;
   const int slot = blockIdx.y;
-  const int I0 = blockIdx.x * SEL_RI;
-  const int nI = min(SEL_RI, L.nqb - I0);
+  const int I0 = blockIdx.x * ri;
+  const int nI = min(ri, L.nqb - I0);
   const int h = ht.bhead[slot];
   const int kind = ht.kind[h];
   const int kvh = h / L.G;
   const float tau = rsqrtf((float)D);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const __nv_bfloat16* qhl = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_qbar) + ((int64_t)slot * L.nqb + I0) * 2 * D;
   const __nv_bfloat16* khl = reinterpret_cast<const __nv_bfloat16*>(ws + L.off_kbar) + (int64_t)kvh * L.nqb * 2 * D;
   const int g = lane >> 2, t4 = lane & 3;
   // The contraction runs over the channels in a permuted order (the same on
@@ -405,11 +406,61 @@ __global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__
   // loads of rows g and g + 1 fall in different banks
   constexpr int QP = 2 * D + 32;
   __shared__ __align__(16) __nv_bfloat16 qs[SEL_RI][QP];
-  for (int i = tid; i < SEL_RI * (2 * D / 8); i += SEL_NT) {
-    const int r = i / (2 * D / 8), c = (i % (2 * D / 8)) * 8;
-    *reinterpret_cast<uint4*>(&qs[r][c]) = r < nI ? ld16(qhl + (int64_t)r * 2 * D + c) : make_uint4(0u, 0u, 0u, 0u);
+  {
+    // mean pooling: thread (row group rg, 8-channel chunk c0); row group rg
+    // serves block rg / gpb and takes every gpb-th row of it, eight loads in
+    // flight; partial sums meet in shared memory (aliasing the score tile)
+    constexpr int CPR = D / 8;         // 16-byte chunks per row
+    constexpr int RGS = SEL_NT / CPR;  // row groups
+    static_assert(RGS % SEL_RI == 0, "row groups per block");
+    const int gpb = RGS / ri;
+    const int rg = tid / CPR, c0 = (tid % CPR) * 8;
+    const int b = rg / gpb, sub = rg % gpb;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    if (b < nI) {
+      const int r_beg = (I0 + b) * L.B, r_end = min(L.N, r_beg + L.B);
+      const __nv_bfloat16* X = Q + (int64_t)h * q_hs + c0;
+      int r = r_beg + sub;
+      for (; r + 7 * gpb < r_end; r += 8 * gpb) {
+        uint4 raw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) raw[u] = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r + u * gpb) * q_ts));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) acc[j] += __bfloat162float(e[j]);
+        }
+      }
+      for (; r < r_end; r += gpb) {
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)r * q_ts));
+        const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += __bfloat162float(e[j]);
+      }
+    }
+    float* part = sc;  // [RGS][D]
+#pragma unroll
+    for (int j = 0; j < 8; ++j) part[rg * D + c0 + j] = acc[j];
+    __syncthreads();
+    for (int i = tid; i < SEL_RI * D; i += SEL_NT) {
+      const int bb = i / D, ch = i % D;
+      __nv_bfloat16 hi = __float2bfloat16_rn(0.f), lo = hi;
+      if (bb < nI) {
+        float sum = 0.f;
+        for (int k = 0; k < gpb; ++k) sum += part[(bb * gpb + k) * D + ch];
+        const int r_beg = (I0 + bb) * L.B;
+        const float x = sum / (float)(min(L.N, r_beg + L.B) - r_beg);
+        hi = __float2bfloat16_rn(x);
+        lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+      }
+      qs[bb][ch] = hi;
+      qs[bb][D + ch] = lo;
+    }
+    __syncthreads();  // the score tile may now overwrite the partial sums
   }
-  __syncthreads();
   // s = tau (qhi khi + qhi klo + qlo khi): bf16 tensor-core products with fp32
   // accumulation; the dropped qlo klo term is below 2^-16 of |q| |k| per channel.
   // Each warp takes 8-key-block column tiles in turn.
@@ -1141,7 +1192,6 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   if (L->nbh > 0 && L->nqb > 2048) return DSA_ERR_UNSUPPORTED;  // block scores of 16 rows live in shared memory
   const int64_t d = p.d;
   int64_t off = 0;
-  L->off_qbar = off; off = align256(off + (int64_t)L->nbh * nqb * d * 4);
   L->off_kbar = off; off = align256(off + (L->nbh ? (int64_t)p.Hkv * nqb * d * 4 : 0));
   L->off_sel = off;  off = align256(off + (int64_t)L->nbh * nqb * L->nkw * 4);
   L->off_v = off;    off = align256(off + (int64_t)L->nvs * N * 4);
@@ -1236,17 +1286,19 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   if (L.nbh > 0) {
     if (p.d == 128) {
-      k_pool<128><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
-                                                             p.k_head_stride, p.k_token_stride, ws);
-      const size_t sel_smem = (size_t)SEL_RI * SEL_RS(L.nkw * 32) * 4;
+      k_pool<128><<<dim3(L.nqb, p.Hkv), 256, 0, st>>>(ct, L, k, p.k_head_stride, p.k_token_stride, ws);
+      const int ri = sel_blocks_per_cta(p.block);
+      const size_t sel_smem = sel_smem_bytes(128, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<128><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), SEL_NT, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<128><<<dim3(ceil_div(L.nqb, ri), L.nbh), SEL_NT, sel_smem, st>>>(
+          ht, L, q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri);
     } else {
-      k_pool<64><<<dim3(L.nqb, L.nbh + p.Hkv), 256, 0, st>>>(ht, ct, L, q, p.q_head_stride, p.q_token_stride, k,
-                                                            p.k_head_stride, p.k_token_stride, ws);
-      const size_t sel_smem = (size_t)SEL_RI * SEL_RS(L.nkw * 32) * 4;
+      k_pool<64><<<dim3(L.nqb, p.Hkv), 256, 0, st>>>(ct, L, k, p.k_head_stride, p.k_token_stride, ws);
+      const int ri = sel_blocks_per_cta(p.block);
+      const size_t sel_smem = sel_smem_bytes(64, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<64><<<dim3(ceil_div(L.nqb, SEL_RI), L.nbh), SEL_NT, sel_smem, st>>>(ht, L, ws, out.blk_ptr);
+      k_block_select<64><<<dim3(ceil_div(L.nqb, ri), L.nbh), SEL_NT, sel_smem, st>>>(
+          ht, L, q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri);
     }
   }
   if (L.nvs > 0) {
