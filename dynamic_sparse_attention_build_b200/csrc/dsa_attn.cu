@@ -144,6 +144,8 @@ static_assert(B_INFO + NINFO <= 25, "barrier slots");
 // tcgen05 and shuffle instructions converged even when a wait runs out).
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit, unsigned* status,
                                           unsigned detail, volatile int* abort_flag) {
+  // fast path: every lane probes once, no broadcast needed
+  if (__all_sync(0xffffffffu, mbar_test_wait(bar, parity))) return true;
   int ok = 0;
   if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, limit, status, detail, abort_flag) ? 1 : 0;
   ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -620,16 +622,28 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int window = it.window;
       const int row = it.qt * BM + r;
       float m = -INFINITY, l = 0.f;
-      for (int t = 0; t < T; ++t) {
+      // The StageInfo of tile t + 1 is waited for and read while the S load of
+      // tile t is in flight, and the mask of tile t is built there too, so none
+      // of it sits between one tile's P and the next tile's exponentials.
+      StageInfo si_next{};
+      if (T > 0) {
+        if (warp_wait(&bars[B_INFO + tg % NINFO], (tg / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag))
+          si_next = info[tg % NINFO];
+        else
+          ok = false;
+      }
+      for (int t = 0; ok && t < T; ++t) {
         const int g = tg + t;
         const int b = g & 1;
         const uint32_t use = (g >> 1) & 1;
         const int slot = g % NINFO;
-        if (!warp_wait(&bars[B_INFO + slot], (g / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
-          ok = false;
-          break;
-        }
-        const StageInfo si = info[slot];
+        const StageInfo si = si_next;
+        if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
+        float s[64];
+        tmem_ld32(s_t, s);
+        tmem_ld32(s_t + 32, s + 32);
         // allowed-key bits of this row, 32 columns per word
         uint32_t mw[2];
         if (si.type == 0) {
@@ -657,13 +671,15 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mw[k] = bits;
           }
         }
-        if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
-        float s[64];
-        tmem_ld32(s_t, s);
-        tmem_ld32(s_t + 32, s + 32);
+        if (t + 1 < T) {
+          const int sn = (g + 1) % NINFO;
+          if (warp_wait(&bars[B_INFO + sn], ((g + 1) / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag))
+            si_next = info[sn];
+          else
+            ok = false;
+        }
         tmem_wait_ld();
+        if (!ok) break;
         // masked keys become -inf, so one code path serves every tile (exp2 of
         // -inf is 0); a tile the whole warp sees fully skips even that
         if (!__all_sync(0xffffffffu, (mw[0] & mw[1]) == 0xffffffffu)) {
