@@ -28,7 +28,7 @@
 //     128 and 192.  S(t+1) = Q K(t+1)^T is computed while the softmax works on
 //     S(t); the softmax writes P(t) as bf16 pairs over the first 32 columns of its
 //     S buffer and O += P(t) V(t) reads it from there;
-//   * the running max is only raised when it grows by more than 2^8; only then
+//   * the running max is only raised when it grows by more than 2^32; only then
 //     does the softmax wait for the previous P.V and rescale O, so in the common
 //     case the softmax of one tile overlaps the P.V of the one before;
 //   * ~100 KB of shared memory and 256 TMEM columns per CTA let two CTAs share an
@@ -53,7 +53,11 @@ constexpr int NTHREADS = 256;      // warps 0,2,3 load, warp 1 issues MMAs, warp
 constexpr uint32_t TMEM_COLS = 256;
 constexpr uint32_t S_COL = 128;    // S buffer b at S_COL + 64 b
 constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after its softmax ended)
-constexpr float RESCALE_THRESHOLD = 8.0f;  // log2 units
+// log2 units.  Scaling every P of a row by one power of two changes no rounding
+// (fp32 and bf16 are relative), so a running max that lags the true one is exact
+// after the final division; 2^32 leaves P <= 2^32, l and O <= 2^53 |V| for 2^21
+// keys, far inside fp32 range, and avoids almost every O rescale.
+constexpr float RESCALE_THRESHOLD = 32.0f;
 #ifndef DSA_LOADER_SUSPEND
 #define DSA_LOADER_SUSPEND 1
 #endif
@@ -78,6 +82,17 @@ struct StageInfo {
 
 struct ItemInfo {
   int h, qt, kind, sink, window, T;  // T: KV tiles of the item
+};
+
+// An item as the decoder warps hand it to the TMA producer and to themselves
+// (column gathering): bitmap set item & 1 holds its key units.
+struct DecInfo {
+  int item;    // -1: no more items
+  int h, qt, kvh;
+  int T_u, T;  // unit tiles, all tiles
+  int tg;      // tiles of this CTA's earlier items
+  int flags1;  // halves that use half 0's column tiles (3 when both halves share a query block)
+  int cc[2], cb[2];  // column count / first column of each half
 };
 
 struct AttnArgs {
@@ -111,11 +126,13 @@ struct Smem {
   static constexpr int COL_OFF = V_OFF + 2 * DS * KSLAB;   // int [NINFO][BN]
   static constexpr int INFO_OFF = COL_OFF + NINFO * BN * 4;
   static constexpr int ITEM_OFF = INFO_OFF + NINFO * (int)sizeof(StageInfo);
-  static constexpr int BAR_OFF = (ITEM_OFF + 2 * (int)sizeof(ItemInfo) + 7) & ~7;
-  static constexpr int NBAR = 25;
+  static constexpr int DEC_OFF = ITEM_OFF + 2 * (int)sizeof(ItemInfo);
+  static constexpr int BAR_OFF = (DEC_OFF + 2 * (int)sizeof(DecInfo) + 7) & ~7;
+  static constexpr int NBAR = 29;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int BITS_OFF = MISC_OFF + 64;
-  static int bytes(int nwords) { return BITS_OFF + 2 * nwords * 4 + 1024; }
+  // two bitmap sets (items kc and kc + 1), each two halves of nwords words
+  static int bytes(int nwords) { return BITS_OFF + 4 * nwords * 4 + 1024; }
 };
 
 // Barrier slots.  Per-buffer barriers (K, V, S, P) complete once per use of their
@@ -136,9 +153,12 @@ enum {
   B_DRAIN = 16,
   B_ITEMFULL = 17,  // +2
   B_ITEMFREE = 19,  // +2
-  B_INFO = 21       // +NINFO
+  B_INFO = 21,      // +NINFO
+  B_DECFULL = 25,   // +2: bitmap set s and DecInfo s written
+  B_UNITS = 27,     // once per item: the producer has issued the item's unit tiles
+  B_COLS = 28       // once per item: the gatherers have filled the item's column tiles
 };
-static_assert(B_INFO + NINFO <= 25, "barrier slots");
+static_assert(B_COLS + 1 <= 29, "barrier slots");
 
 // One lane waits, the whole warp learns the outcome (keeps warp-collective
 // tcgen05 and shuffle instructions converged even when a wait runs out).
@@ -241,6 +261,19 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       : "memory");
 }
 
+// 16 consecutive fp32 columns of this thread's TMEM lane (completes at tmem_wait_ld)
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+  uint32_t r[16];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -263,8 +296,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   // misc: [0] tmem base, [2] abort, [3] unit count, [4] col count half0, [5] col count half1,
   //       [6] col base half0, [7] col base half1, [9] loader go flag, [10] current item
   volatile int* abort_flag = misc + 2;
-  uint32_t* bits0 = reinterpret_cast<uint32_t*>(sm + L::BITS_OFF);
-  uint32_t* bits1 = bits0 + a.nwords;
+  uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L::BITS_OFF);  // [set][half][nwords]
+  DecInfo* dec = reinterpret_cast<DecInfo*>(sm + L::DEC_OFF);
   StageInfo* info = reinterpret_cast<StageInfo*>(sm + L::INFO_OFF);
   ItemInfo* items = reinterpret_cast<ItemInfo*>(sm + L::ITEM_OFF);
   int* colsm = reinterpret_cast<int*>(sm + L::COL_OFF);
@@ -302,45 +335,121 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   const uint64_t limit = a.wait_limit_ns;
   const int upb = a.B / UNIT;  // units per block
 
-  if (warp == 0 || warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ loaders
-    // Work items (query tile, head) are dealt round-robin over the CTAs, latest
-    // (heaviest) tiles first.  While the MMA and softmax warps still work on one
-    // item, these warps already read the next item's lists and start its loads.
-    const int ltid = (warp == 0 ? 0 : warp - 1) * 32 + lane;  // 0..95
-    // The first item of a CTA is its block index; later ones come from a global
-    // counter (dynamic: items differ a lot in cost), fetched one item ahead.
-    int tg = 0;     // tiles of earlier items
-    int kc = 0;     // items of this CTA so far
-    bool go = true;
-    int next_item = 0;
-    for (;; ++kc) {
-      if (ltid == 0) {
-        misc[10] = kc == 0 ? (int)blockIdx.x : next_item;
-        next_item = (int)gridDim.x + (int)atomicAdd(a.sched, 1u);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    // Q of every item and the TMA loads of its key units, walking the bitmap set
+    // that the decoder warps filled (up to one item ahead).
+    if (lane == 0) {
+      for (int kc = 0;; ++kc) {
+        const int s = kc & 1;
+        if (!mbar_wait(&bars[B_DECFULL + s], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+                       kLoaderSuspend))
+          break;
+        const DecInfo di = dec[s];
+        if (di.item < 0) break;  // no more items
+        // Q once every Q K^T of the previous item has finished
+        if (kc > 0 && !mbar_wait(&bars[B_QEMPTY], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag,
+                                 kLoaderSuspend))
+          break;
+        mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
+        for (int c = 0; c < DS; ++c)
+          tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, di.qt * BM, di.h);
+        // Tiles are issued in order (units, then columns, item by item): a buffer's
+        // empty barrier is waited on by parity, which is only unambiguous when the
+        // tile two before has been issued.  So the previous item's column tiles
+        // come first.
+        if (kc > 0 && !mbar_wait(&bars[B_COLS], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+                                 kLoaderSuspend))
+          break;
+        const uint32_t* b0 = bits + s * 2 * a.nwords;
+        const uint32_t* b1 = b0 + a.nwords;
+        bool ok = true;
+        int w = 0;
+        uint32_t pend = b0[0] | b1[0];
+        for (int t = 0; t < di.T_u; ++t) {
+          const int g = di.tg + t;
+          const int b = g & 1;
+          const uint32_t use = (g >> 1) & 1;
+          if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
+            ok = false;
+            break;
+          }
+          while (pend == 0u && w + 1 < a.nwords) {
+            ++w;
+            pend = b0[w] | b1[w];
+          }
+          const int bit = __ffs(pend) - 1;  // T_u counts exactly the set bits
+          pend &= pend - 1u;
+          const int u = w * 32 + bit;
+          StageInfo& si = info[g % NINFO];
+          si.type = 0;
+          si.u = u;
+          si.flags = (int)((b0[w] >> bit) & 1u) | ((int)((b1[w] >> bit) & 1u) << 1);
+          si.ncols = 0;
+          mbar_arrive(&bars[B_INFO + g % NINFO]);
+          uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+          uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
+          mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
+          for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, di.kvh);
+          if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
+          for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, di.kvh);
+        }
+        if (!ok) break;
+        mbar_arrive(&bars[B_UNITS]);  // this item's bitmaps are no longer read here
       }
-      // every loader thread is done with the previous item's bitmaps and counts
-      named_barrier(1, 96);
+    }
+    __syncwarp();
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ decoders
+    // Work items (query tile, head) are dealt latest (heaviest) tiles first: the
+    // first item of a CTA is its block index, later ones come from a global
+    // counter (dynamic: items differ a lot in cost).  These two warps turn item
+    // kc + 1's lists into bitmap set (kc + 1) & 1 before they gather item kc's
+    // column tiles, so the lists of an item are read while the item before it
+    // still computes.
+    const int dtid = (warp - 2) * 32 + lane;  // 0..63
+    int next_item = (int)blockIdx.x;          // held by dtid 0
+    int tg_dec = 0;                           // tiles of the items decoded so far
+    bool go = true;
+
+    // Decodes item kc of this CTA into bitmap set kc & 1 and publishes it.
+    // Returns false when there is no such item (end marker published) or on abort.
+    // Set kc & 1 is free: these warps gathered item kc - 2's columns, which they
+    // only start once the producer has issued that item's units.
+    auto decode = [&](int kc) -> bool {
+      const int s = kc & 1;
+      if (dtid == 0) {
+        misc[10] = next_item;
+        next_item = (int)gridDim.x + (int)atomicAdd(a.sched, 1u);  // fetched one item ahead
+        misc[3] = 0;
+      }
+      named_barrier(1, 64);
       const int item = misc[10];
-      if (!go || item >= n_items) {
-        // no more work: tell the MMA and softmax warps (ItemInfo with T = -1)
-        if (ltid == 0) {
+      if (item >= n_items) {
+        // no more work: end markers for the producer, the MMA and the softmax warps
+        if (dtid == 0) {
           const int slot = kc & 1;
           if (kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
                                   DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
             items[slot].T = -1;
             mbar_arrive(&bars[B_ITEMFULL + slot]);
           }
+          dec[s].item = -1;
+          mbar_arrive(&bars[B_DECFULL + s]);
         }
-        break;
+        return false;  // the previous item's column tiles are still gathered
       }
       const int h = item % a.Hq;
       const int qt = a.n_qtiles - 1 - item / a.Hq;
-      const int kvh = h / a.G;
       const int row0 = qt * BM;
       const int kind = a.head_info[h * 4 + 0];
-      for (int i = ltid; i < 2 * a.nwords; i += 96) bits0[i] = 0u;
-      if (ltid == 0) misc[3] = 0;
+      uint32_t* b0 = bits + s * 2 * a.nwords;
+      uint32_t* b1 = b0 + a.nwords;
+      for (int i = dtid; i < 2 * a.nwords; i += 64) b0[i] = 0u;
       int qbh[2], r1h[2];
       bool live[2];
 #pragma unroll
@@ -351,69 +460,74 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         r1h[hh] = min(a.N - 1, r0 + 63);
       }
       const bool shared_qb = live[1] && (qbh[0] == qbh[1]);
-      named_barrier(1, 96);
-      if (ltid == 32) {
+      named_barrier(1, 64);
+      if (dtid == 32) {
         // column lists: independent of the block lists, read in parallel with them
-        int c0 = 0, c1 = 0, b0 = 0, b1 = 0;
+        int c0 = 0, c1 = 0, cb0 = 0, cb1 = 0;
         if (live[0]) {
           const int r = h * a.nqb + qbh[0];
-          b0 = a.col_ptr[r];
-          c0 = a.col_ptr[r + 1] - b0;
+          cb0 = a.col_ptr[r];
+          c0 = a.col_ptr[r + 1] - cb0;
         }
         if (live[1] && !shared_qb) {
           const int r = h * a.nqb + qbh[1];
-          b1 = a.col_ptr[r];
-          c1 = a.col_ptr[r + 1] - b1;
+          cb1 = a.col_ptr[r];
+          c1 = a.col_ptr[r + 1] - cb1;
         }
-        misc[4] = c0; misc[5] = c1; misc[6] = b0; misc[7] = b1;
+        dec[s].cc[0] = max(0, c0);
+        dec[s].cc[1] = max(0, c1);
+        dec[s].cb[0] = cb0;
+        dec[s].cb[1] = cb1;
       }
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         if (!live[hh]) continue;
-        uint32_t* bits = hh ? bits1 : bits0;
+        uint32_t* bb = hh ? b1 : b0;
         const int qb = qbh[hh];
         const int r1 = r1h[hh];
         if (kind == DSA_KIND_VS) {
           const int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
-          for (int e = beg + ltid; e < end; e += 96) {
+          for (int e = beg + dtid; e < end; e += 64) {
             const int delta = a.dist[e];
             if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
             if (delta > qb) continue;
             const int kb = qb - delta;
             for (int u = kb * upb; u < kb * upb + upb; ++u)
-              if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
+              if (u * UNIT <= r1) atomicOr(&bb[u >> 5], 1u << (u & 31));
           }
         } else {
           const int r = h * a.nqb + qb;
           const int beg = a.blk_ptr[r], end = a.blk_ptr[r + 1];
-          for (int e = beg + ltid; e < end; e += 96) {
+          for (int e = beg + dtid; e < end; e += 64) {
             const int kb = a.blk_idx[e];
             if (kb < 0 || kb >= a.nqb) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_BLOCK); continue; }
             for (int u = kb * upb; u < kb * upb + upb; ++u)
-              if (u * UNIT <= r1) atomicOr(&bits[u >> 5], 1u << (u & 31));
+              if (u * UNIT <= r1) atomicOr(&bb[u >> 5], 1u << (u & 31));
           }
         }
       }
-      named_barrier(1, 96);
+      named_barrier(1, 64);
       {
         int cnt = 0;
-        for (int w = ltid; w < a.nwords; w += 96) cnt += __popc(bits0[w] | bits1[w]);
+        for (int w = dtid; w < a.nwords; w += 64) cnt += __popc(b0[w] | b1[w]);
         cnt = warp_sum_int(cnt);
         if (lane == 0 && cnt) atomicAdd(&misc[3], cnt);
       }
-      named_barrier(1, 96);
-      const int T_u = misc[3];  // one tile per unit
-      const int ccount[2] = {max(0, misc[4]), max(0, misc[5])};
-      const int cbase[2] = {misc[6], misc[7]};
-      const int cflags[2] = {shared_qb ? 3 : 1, 2};
-      const int T_c0 = ceil_div(ccount[0], BN), T_c1 = ceil_div(ccount[1], BN);
-      const int T = T_u + T_c0 + T_c1;
-      if (ltid == 0) {
-        // publish the item (its slot is free once both consumers read item kc - 2),
-        // then load its Q once every Q K^T of the previous item has finished
+      named_barrier(1, 64);
+      if (dtid == 0) {
+        DecInfo& di = dec[s];
+        di.item = item;
+        di.h = h;
+        di.qt = qt;
+        di.kvh = h / a.G;
+        di.T_u = misc[3];  // one tile per unit
+        di.flags1 = shared_qb ? 3 : 1;
+        di.T = di.T_u + ceil_div(di.cc[0], BN) + ceil_div(di.cc[1], BN);
+        di.tg = tg_dec;
+        // publish the item (its slot is free once both consumers read item kc - 2)
         const int slot = kc & 1;
-        bool ok = kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
-                                      DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+        const bool ok = kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
+                                            DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
         if (ok) {
           ItemInfo& it = items[slot];
           it.h = h;
@@ -421,104 +535,97 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           it.kind = kind;
           it.sink = a.head_info[h * 4 + 1];
           it.window = a.head_info[h * 4 + 2];
-          it.T = T;
+          it.T = di.T;
           mbar_arrive(&bars[B_ITEMFULL + slot]);
-        }
-        ok = ok && (kc == 0 || mbar_wait(&bars[B_QEMPTY], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kLoaderSuspend));
-        if (ok) {
-          mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
-          for (int c = 0; c < DS; ++c) tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, row0, h);
+          mbar_arrive(&bars[B_DECFULL + s]);
         }
         misc[9] = ok ? 1 : 0;
       }
-      named_barrier(1, 96);
-      if (misc[9] == 0) { go = false; continue; }
-      if (warp == 0 && lane == 0) {
-        int w = 0;
-        uint32_t pend = bits0[0] | bits1[0];
-        for (int t = 0; t < T_u; ++t) {
-          const int g = tg + t;
-          const int b = g & 1;
-          const uint32_t use = (g >> 1) & 1;
-          if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) break;
-          while (pend == 0u && w + 1 < a.nwords) {
-            ++w;
-            pend = bits0[w] | bits1[w];
-          }
-          const int bit = __ffs(pend) - 1;  // T_u counts exactly the set bits
-          pend &= pend - 1u;
-          const int u = w * 32 + bit;
-          StageInfo& si = info[g % NINFO];
-          si.type = 0;
-          si.u = u;
-          si.flags = (int)((bits0[w] >> bit) & 1u) | ((int)((bits1[w] >> bit) & 1u) << 1);
-          si.ncols = 0;
-          mbar_arrive(&bars[B_INFO + g % NINFO]);
-          uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
-          uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
-          mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
-          for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, kvh);
-          if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) break;
-          mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
-          for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, kvh);
-        }
-      }
-      __syncwarp();
-      // column tiles: all 96 loader threads gather rows into the swizzled layout
-      int t = T_u;
+      named_barrier(1, 64);
+      if (misc[9] == 0) { go = false; return false; }
+      tg_dec += dec[s].T;
+      return true;
+    };
+
+    // Gathers the column tiles of item kc (bitmap set kc & 1) into the K/V
+    // buffers: rows loaded into the swizzled layout by all 64 threads.
+    auto gather = [&](int kc) {
+      const int s = kc & 1;
+      const DecInfo di = dec[s];
+      const uint32_t* b0 = bits + s * 2 * a.nwords;
+      const uint32_t* b1 = b0 + a.nwords;
+      // the column tiles follow the item's unit tiles (see the producer)
+      if (dtid == 0)
+        misc[9] = mbar_wait(&bars[B_UNITS], kc & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend) ? 1 : 0;
+      named_barrier(1, 64);
+      if (misc[9] == 0) { go = false; return; }
+      int t = di.T_u;
       for (int hh = 0; go && hh < 2; ++hh) {
-        const int nt = hh ? T_c1 : T_c0;
+        const int nt = ceil_div(di.cc[hh], BN);
+        const int cflags = hh ? 2 : di.flags1;
         for (int ct = 0; ct < nt; ++ct, ++t) {
-          const int g = tg + t;
+          const int g = di.tg + t;
           const int b = g & 1;
           const uint32_t use = (g >> 1) & 1;
-          if (ltid == 0) {
+          if (dtid == 0) {
             bool ok = mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
             ok = ok && mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
             misc[9] = ok ? 1 : 0;
           }
-          named_barrier(1, 96);
+          named_barrier(1, 64);
           if (misc[9] == 0) { go = false; break; }
-          const int first = cbase[hh] + ct * BN;
-          const int nc = min(BN, ccount[hh] - ct * BN);
+          const int first = di.cb[hh] + ct * BN;
+          const int nc = min(BN, di.cc[hh] - ct * BN);
           int* cj = colsm + (g % NINFO) * BN;
           uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
           uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
-          constexpr int CH = D / 8;  // 16-byte chunks per row
-          for (int i = ltid; i < BN * CH; i += 96) {
-            const int slot = i / CH;
-            const int ch = i % CH;
-            int j = (slot < nc) ? a.col_idx[first + slot] : -1;
-            if (slot < nc && (j < 0 || j >= a.N)) {
-              report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_COL);
-              j = -1;
-            }
-            if (ch == 0) {
-              // bit 24 / 25: the column's block is already kept for half 0 / half 1,
-              // so that half must not count the key a second time
-              int v = j;
-              if (j >= 0) {
-                const int u = j / UNIT;
-                const int cov =
-                    (int)((bits0[u >> 5] >> (u & 31)) & 1u) | ((int)((bits1[u >> 5] >> (u & 31)) & 1u) << 1);
-                v = j | (cov << 24);
+          constexpr int CH = D / 8;           // 16-byte chunks per row
+          constexpr int PER = BN * CH / 64;   // chunks per thread
+          constexpr int UNR = 4;
+          static_assert(PER % UNR == 0, "gather unroll");
+#pragma unroll 1
+          for (int i0 = 0; i0 < PER; i0 += UNR) {
+            uint4 kv[UNR], vv[UNR];
+            uint32_t off[UNR];
+#pragma unroll
+            for (int q = 0; q < UNR; ++q) {
+              const int i = (i0 + q) * 64 + dtid;
+              const int slot = i / CH;
+              const int ch = i % CH;
+              int j = (slot < nc) ? a.col_idx[first + slot] : -1;
+              if (slot < nc && (j < 0 || j >= a.N)) {
+                report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_COL);
+                j = -1;
               }
-              cj[slot] = v;
+              if (ch == 0) {
+                // bit 24 / 25: the column's block is already kept for half 0 / half 1,
+                // so that half must not count the key a second time
+                int v = j;
+                if (j >= 0) {
+                  const int u = j / UNIT;
+                  const int cov = (int)((b0[u >> 5] >> (u & 31)) & 1u) | ((int)((b1[u >> 5] >> (u & 31)) & 1u) << 1);
+                  v = j | (cov << 24);
+                }
+                cj[slot] = v;
+              }
+              const int jr = j < 0 ? 0 : j;
+              kv[q] = __ldg(reinterpret_cast<const uint4*>(a.K + di.kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
+              vv[q] = __ldg(reinterpret_cast<const uint4*>(a.V + di.kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
+              off[q] = (ch >> 3) * KSLAB + swz(slot, ch & 7);
             }
-            const int jr = j < 0 ? 0 : j;
-            const uint4 kv = __ldg(reinterpret_cast<const uint4*>(a.K + kvh * a.k_hs + (int64_t)jr * a.k_ts) + ch);
-            const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.V + kvh * a.v_hs + (int64_t)jr * a.v_ts) + ch);
-            const uint32_t off = (ch >> 3) * KSLAB + swz(slot, ch & 7);
-            *reinterpret_cast<uint4*>(kst + off) = kv;
-            *reinterpret_cast<uint4*>(vst + off) = vv;
+#pragma unroll
+            for (int q = 0; q < UNR; ++q) {
+              *reinterpret_cast<uint4*>(kst + off[q]) = kv[q];
+              *reinterpret_cast<uint4*>(vst + off[q]) = vv[q];
+            }
           }
           fence_proxy_async_smem();
-          named_barrier(1, 96);
-          if (ltid == 0) {
+          named_barrier(1, 64);
+          if (dtid == 0) {
             StageInfo& si = info[g % NINFO];
             si.type = 1;
             si.u = -1;
-            si.flags = cflags[hh];
+            si.flags = cflags;
             si.ncols = nc;
             mbar_arrive(&bars[B_INFO + g % NINFO]);
             mbar_arrive(&bars[B_KFULL + b]);
@@ -526,9 +633,16 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         }
       }
-      __syncwarp();
-      tg += T;
+      if (go && dtid == 0) mbar_arrive(&bars[B_COLS]);
+    };
+
+    bool have = decode(0);
+    for (int kc = 0; have && go; ++kc) {
+      const bool have_next = decode(kc + 1);
+      if (go) gather(kc);
+      have = have_next;
     }
+    __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
@@ -622,22 +736,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int window = it.window;
       const int row = it.qt * BM + r;
       float m = -INFINITY, l = 0.f;
-      // The StageInfo of tile t + 1 is waited for and read while the S load of
-      // tile t is in flight, and the mask of tile t is built there too, so none
-      // of it sits between one tile's P and the next tile's exponentials.
-      StageInfo si_next{};
-      if (T > 0) {
-        if (warp_wait(&bars[B_INFO + tg % NINFO], (tg / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag))
-          si_next = info[tg % NINFO];
-        else
-          ok = false;
-      }
       for (int t = 0; ok && t < T; ++t) {
         const int g = tg + t;
         const int b = g & 1;
         const uint32_t use = (g >> 1) & 1;
         const int slot = g % NINFO;
-        const StageInfo si = si_next;
+        // The StageInfo of a tile is published when its K load is issued, before
+        // its S can exist, so this wait ends at the first probe whenever S is not
+        // ready yet either.  The tile's mask is built while its S load is in flight.
+        if (!warp_wait(&bars[B_INFO + slot], (g / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag)) {
+          ok = false;
+          break;
+        }
+        const StageInfo si = info[slot];
         if (!warp_wait(&bars[B_SFULL + b], use, limit, a.status, DETAIL_WAIT_S, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t s_t = tmem_base + lane_off + S_COL + 64 * b;
@@ -671,15 +782,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             mw[k] = bits;
           }
         }
-        if (t + 1 < T) {
-          const int sn = (g + 1) % NINFO;
-          if (warp_wait(&bars[B_INFO + sn], ((g + 1) / NINFO) & 1, limit, a.status, DETAIL_WAIT_K, abort_flag))
-            si_next = info[sn];
-          else
-            ok = false;
-        }
         tmem_wait_ld();
-        if (!ok) break;
         // masked keys become -inf, so one code path serves every tile (exp2 of
         // -inf is 0); a tile the whole warp sees fully skips even that
         if (!__all_sync(0xffffffffu, (mw[0] & mw[1]) == 0xffffffffu)) {
