@@ -70,8 +70,12 @@ constexpr float RESCALE_THRESHOLD = 32.0f;
 constexpr bool kLoaderSuspend = DSA_LOADER_SUSPEND != 0;
 constexpr bool kMmaSuspend = DSA_MMA_SUSPEND != 0;
 #ifndef DSA_POLY_PERIOD
-#define DSA_POLY_PERIOD 8  // one exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe
+// One exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe (0: none).  Off: the
+// exponentials do not saturate the XU pipe in this kernel, and the smaller loop
+// body measured faster.
+#define DSA_POLY_PERIOD 0
 #endif
+constexpr int kPolyPeriod = DSA_POLY_PERIOD > 0 ? DSA_POLY_PERIOD : 1 << 20;
 
 struct StageInfo {
   int type;   // 0 = key unit, 1 = column tile
@@ -259,19 +263,6 @@ __device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
-}
-
-// 16 consecutive fp32 columns of this thread's TMEM lane (completes at tmem_wait_ld)
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-  uint32_t r[16];
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr));
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
@@ -841,7 +832,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           for (int i = 0; i < 16; ++i) {
             float x0, x1, p0, p1;
             fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
-            if (i % DSA_POLY_PERIOD == DSA_POLY_PERIOD - 1) {
+            if (kPolyPeriod > 0 && i % kPolyPeriod == kPolyPeriod - 1) {
               poly_ex2x2(x0, x1, p0, p1);  // part of the pairs on the FMA pipe
             } else {
               p0 = fast_ex2(x0);
