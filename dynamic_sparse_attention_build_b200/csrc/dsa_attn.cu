@@ -333,13 +333,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0) {
       for (int kc = 0;; ++kc) {
         const int s = kc & 1;
-        if (!mbar_wait(&bars[B_DECFULL + s], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+        if (!mbar_wait_ool(&bars[B_DECFULL + s], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
                        kLoaderSuspend))
           break;
         const DecInfo di = dec[s];
         if (di.item < 0) break;  // no more items
         // Q once every Q K^T of the previous item has finished
-        if (kc > 0 && !mbar_wait(&bars[B_QEMPTY], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag,
+        if (kc > 0 && !mbar_wait_ool(&bars[B_QEMPTY], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag,
                                  kLoaderSuspend))
           break;
         mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
@@ -349,7 +349,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // empty barrier is waited on by parity, which is only unambiguous when the
         // tile two before has been issued.  So the previous item's column tiles
         // come first.
-        if (kc > 0 && !mbar_wait(&bars[B_COLS], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+        if (kc > 0 && !mbar_wait_ool(&bars[B_COLS], (kc - 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
                                  kLoaderSuspend))
           break;
         const uint32_t* b0 = bits + s * 2 * a.nwords;
@@ -361,7 +361,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const int g = di.tg + t;
           const int b = g & 1;
           const uint32_t use = (g >> 1) & 1;
-          if (!mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
+          if (!mbar_wait_ool(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
             ok = false;
             break;
           }
@@ -382,7 +382,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
           mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
           for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, di.kvh);
-          if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
+          if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
             ok = false;
             break;
           }
@@ -424,7 +424,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         // no more work: end markers for the producer, the MMA and the softmax warps
         if (dtid == 0) {
           const int slot = kc & 1;
-          if (kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
+          if (kc < 2 || mbar_wait_ool(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
                                   DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
             items[slot].T = -1;
             mbar_arrive(&bars[B_ITEMFULL + slot]);
@@ -517,7 +517,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         di.tg = tg_dec;
         // publish the item (its slot is free once both consumers read item kc - 2)
         const int slot = kc & 1;
-        const bool ok = kc < 2 || mbar_wait(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
+        const bool ok = kc < 2 || mbar_wait_ool(&bars[B_ITEMFREE + slot], ((kc >> 1) - 1) & 1, limit, a.status,
                                             DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
         if (ok) {
           ItemInfo& it = items[slot];
@@ -547,7 +547,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint32_t* b1 = b0 + a.nwords;
       // the column tiles follow the item's unit tiles (see the producer)
       if (dtid == 0)
-        misc[9] = mbar_wait(&bars[B_UNITS], kc & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend) ? 1 : 0;
+        misc[9] = mbar_wait_ool(&bars[B_UNITS], kc & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend) ? 1 : 0;
       named_barrier(1, 64);
       if (misc[9] == 0) { go = false; return; }
       int t = di.T_u;
@@ -559,8 +559,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const int b = g & 1;
           const uint32_t use = (g >> 1) & 1;
           if (dtid == 0) {
-            bool ok = mbar_wait(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
-            ok = ok && mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+            bool ok = mbar_wait_ool(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
+            ok = ok && mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend);
             misc[9] = ok ? 1 : 0;
           }
           named_barrier(1, 64);
@@ -627,11 +627,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (go && dtid == 0) mbar_arrive(&bars[B_COLS]);
     };
 
-    bool have = decode(0);
-    for (int kc = 0; have && go; ++kc) {
-      const bool have_next = decode(kc + 1);
-      if (go) gather(kc);
-      have = have_next;
+    // decode(kc) then gather(kc - 1): one call site each keeps the code small
+    for (int kc = 0; go; ++kc) {
+      const bool have = decode(kc);
+      if (kc > 0 && go) gather(kc - 1);
+      if (!have) break;
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -644,11 +644,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       int tg = 0;
       for (int kc = 0; ok; ++kc) {
         const int slot = kc & 1;
-        if (!mbar_wait(&bars[B_ITEMFULL + slot], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
+        if (!mbar_wait_ool(&bars[B_ITEMFULL + slot], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
         const int T = items[slot].T;
         mbar_arrive(&bars[B_ITEMFREE + slot]);
         if (T < 0) break;  // no more items
-        if (!mbar_wait(&bars[B_QFULL], kc & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
+        if (!mbar_wait_ool(&bars[B_QFULL], kc & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
         if (T == 0) tc_commit(&bars[B_QEMPTY]);
         for (int t = 0; t <= T; ++t) {
           if (t < T) {
@@ -656,11 +656,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int g = tg + t;
             const int b = g & 1;
             const uint32_t use = (g >> 1) & 1;
-            if (!mbar_wait(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag, kMmaSuspend)) { ok = false; break; }
+            if (!mbar_wait_ool(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag, kMmaSuspend)) { ok = false; break; }
             // the buffer still holds P(g-2) until that P.V has finished; its
             // V-empty commit says so (a per-buffer barrier: at an item boundary
             // P(g-1) V(g-1) has been issued too, so B_ODONE could be two phases on)
-            if (!mbar_wait(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend)) {
+            if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend)) {
               ok = false;
               break;
             }
@@ -683,8 +683,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int g = tg + u;
             const int b = g & 1;
             const uint32_t use = (g >> 1) & 1;
-            if (!mbar_wait(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag, kMmaSuspend)) { ok = false; break; }
-            if (!mbar_wait(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag, kMmaSuspend)) { ok = false; break; }
+            if (!mbar_wait_ool(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag, kMmaSuspend)) { ok = false; break; }
+            if (!mbar_wait_ool(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag, kMmaSuspend)) { ok = false; break; }
             tc_fence_after();
             const uint32_t v_addr = smem_u32(sm + L::V_OFF + b * DS * KSLAB);
             const uint32_t p_tmem = tmem_base + S_COL + 64 * b;
@@ -702,7 +702,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       }
       // drain every MMA this thread issued before TMEM is released
       tc_commit(&bars[B_DRAIN]);
-      mbar_wait(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend);
+      mbar_wait_ool(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend);
     }
     __syncwarp();
   } else {

@@ -91,6 +91,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Records a timed-out wait (status word + the CTA's abort flag).  Out of line:
+// it only runs on a timeout, and every wait site would otherwise carry a copy.
+static __device__ __noinline__ void report_timeout(unsigned* status, unsigned detail, volatile int* abort_flag) {
+  report(status, DSA_ERR_TIMEOUT, detail);
+  *abort_flag = 1;
+}
+
 // Waits for the phase with the given parity to complete.  Gives up after
 // `limit_ns` nanoseconds of global time, records DSA_ERR_TIMEOUT with `detail`
 // in the status word, sets *abort (shared flag) and returns false.  Also returns
@@ -107,12 +114,38 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
     if (((++spins) & 63u) == 0u) {
       if (*abort_flag) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
-        report(status, DSA_ERR_TIMEOUT, detail);
-        *abort_flag = 1;
+        report_timeout(status, detail, abort_flag);
         return false;
       }
     }
   }
+}
+
+// mbar_wait with its bounded loop out of line: one copy of the loop serves every
+// wait site that uses it.  For threads with few live registers (a producer or
+// MMA-issuing thread), where a call costs little and a kernel's code would
+// otherwise carry one loop per site.
+static __device__ __noinline__ bool mbar_wait_loop(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                                    unsigned* status, unsigned detail,
+                                                    volatile int* abort_flag, bool suspend) {
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t spins = 0;
+  while (true) {
+    if (suspend ? mbar_try_wait(bar, parity) : mbar_test_wait(bar, parity)) return true;
+    if (((++spins) & 63u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        report_timeout(status, detail, abort_flag);
+        return false;
+      }
+    }
+  }
+}
+__device__ __forceinline__ bool mbar_wait_ool(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                              unsigned* status, unsigned detail,
+                                              volatile int* abort_flag, bool suspend = false) {
+  if (mbar_test_wait(bar, parity)) return true;
+  return mbar_wait_loop(bar, parity, limit_ns, status, detail, abort_flag, suspend);
 }
 
 // ---------------------------------------------------------------------------
