@@ -254,14 +254,61 @@ __device__ __forceinline__ uint32_t low_bits(int n) {  // n clamped to [0, 32]
   return n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
 }
 
-// O[tmem] (+)= P[tmem] * V[smem desc]: A operand read from tensor memory.
-__device__ __forceinline__ void tc_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                          uint32_t accumulate) {
+// The MMAs of one tile, issued from one asm block (predicates set once; the
+// descriptors advance from a base by constant address offsets, the address
+// field being bits 0-13 of the descriptor in 16-byte units, which never carries
+// for shared-memory addresses below 256 KB).
+//   S = Q K^T: NK k-steps of 16 over the head dimension, accumulating after the first.
+template <int NK>
+__device__ __forceinline__ void mma_qk_tile(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc) {
+  static_assert(NK == 4 || NK == 8, "head dimension 64 or 128");
+  // k-step kk: 64-column slab kk >> 2 (QSLAB / KSLAB bytes apart), 32 bytes per step inside it
+  constexpr uint64_t QS = QSLAB >> 4, KS = KSLAB >> 4;
+  const uint32_t zero = 0;
+  if constexpr (NK == 4) {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %9, 0;\n\tsetp.eq.b32 pt, %9, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %5, %10, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %6, %10, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %7, %10, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %8, %10, pt;\n\t}" ::"r"(d_tmem),
+        "l"(a0), "l"(a0 + 2), "l"(a0 + 4), "l"(a0 + 6), "l"(b0), "l"(b0 + 2), "l"(b0 + 4), "l"(b0 + 6),
+        "r"(zero), "r"(idesc)
+        : "memory");
+  } else {
+    asm volatile(
+        "{\n\t.reg .pred pf, pt;\n\t"
+        "setp.ne.b32 pf, %17, 0;\n\tsetp.eq.b32 pt, %17, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %9, %18, pf;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %2, %10, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %11, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %4, %12, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %13, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %6, %14, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %15, %18, pt;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %8, %16, %18, pt;\n\t}" ::"r"(d_tmem),
+        "l"(a0), "l"(a0 + 2), "l"(a0 + 4), "l"(a0 + 6), "l"(a0 + QS), "l"(a0 + QS + 2), "l"(a0 + QS + 4),
+        "l"(a0 + QS + 6), "l"(b0), "l"(b0 + 2), "l"(b0 + 4), "l"(b0 + 6), "l"(b0 + KS), "l"(b0 + KS + 2),
+        "l"(b0 + KS + 4), "l"(b0 + KS + 6), "r"(zero), "r"(idesc)
+        : "memory");
+  }
+}
+//   O (+)= P V: four k-steps of 16 keys, P read from TMEM (8 columns of packed
+//   bf16 per step), V from shared memory (2048 bytes per step); the first step
+//   overwrites O when acc_first is 0.
+__device__ __forceinline__ void mma_pv_tile(uint32_t d_tmem, uint32_t p_tmem, uint64_t b0, uint32_t idesc,
+                                            uint32_t acc_first) {
+  constexpr uint64_t VS = 2048 >> 4;
   asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      "{\n\t.reg .pred pf, pt;\n\t"
+      "setp.ne.b32 pf, %9, 0;\n\tsetp.eq.b32 pt, %9, %9;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %5, %10, pf;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%2], %6, %10, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %7, %10, pt;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%4], %8, %10, pt;\n\t}" ::"r"(d_tmem),
+      "r"(p_tmem), "r"(p_tmem + 8), "r"(p_tmem + 16), "r"(p_tmem + 24), "l"(b0), "l"(b0 + VS), "l"(b0 + 2 * VS),
+      "l"(b0 + 3 * VS), "r"(acc_first), "r"(idesc)
       : "memory");
 }
 
@@ -639,7 +686,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     if (lane == 0) {
       constexpr uint32_t IDESC_QK = idesc_bf16(BM, BN, 0, 0);
       constexpr uint32_t IDESC_PV = idesc_bf16(BM, D, 0, 1);
-      const uint32_t q_addr = smem_u32(sm + L::Q_OFF);
+      static_assert(BN == 64, "P.V issues four k-steps of 16 keys");
+      const uint64_t q_desc = smem_desc(smem_u32(sm + L::Q_OFF), 16, 1024, SWZ_128B);
+      const uint64_t k_desc0 = smem_desc(smem_u32(sm + L::K_OFF), 16, 1024, SWZ_128B);
+      const uint64_t k_desc1 = smem_desc(smem_u32(sm + L::K_OFF + DS * KSLAB), 16, 1024, SWZ_128B);
+      const uint64_t v_desc0 = smem_desc(smem_u32(sm + L::V_OFF), KSLAB, 1024, SWZ_128B);
+      const uint64_t v_desc1 = smem_desc(smem_u32(sm + L::V_OFF + DS * KSLAB), KSLAB, 1024, SWZ_128B);
       bool ok = true;
       int tg = 0;
       for (int kc = 0; ok; ++kc) {
@@ -665,14 +717,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
               break;
             }
             tc_fence_after();
-            const uint32_t k_addr = smem_u32(sm + L::K_OFF + b * DS * KSLAB);
-            const uint32_t s_tmem = tmem_base + S_COL + 64 * b;
-#pragma unroll
-            for (int kk = 0; kk < D / 16; ++kk) {
-              const uint64_t ad = smem_desc(q_addr + (kk >> 2) * QSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-              const uint64_t bd = smem_desc(k_addr + (kk >> 2) * KSLAB + (kk & 3) * 32, 16, 1024, SWZ_128B);
-              tc_mma_f16(s_tmem, ad, bd, IDESC_QK, kk > 0 ? 1u : 0u);
-            }
+            mma_qk_tile<D / 16>(tmem_base + S_COL + 64 * b, q_desc, b ? k_desc1 : k_desc0, IDESC_QK);
             tc_commit(&bars[B_SFULL + b]);
             tc_commit(&bars[B_KEMPTY + b]);
             if (t == T - 1) tc_commit(&bars[B_QEMPTY]);  // Q may be replaced by the next item's
@@ -686,13 +731,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             if (!mbar_wait_ool(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag, kMmaSuspend)) { ok = false; break; }
             if (!mbar_wait_ool(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag, kMmaSuspend)) { ok = false; break; }
             tc_fence_after();
-            const uint32_t v_addr = smem_u32(sm + L::V_OFF + b * DS * KSLAB);
-            const uint32_t p_tmem = tmem_base + S_COL + 64 * b;
-#pragma unroll
-            for (int kk = 0; kk < BN / 16; ++kk) {
-              const uint64_t bd = smem_desc(v_addr + kk * 2048, KSLAB, 1024, SWZ_128B);
-              tc_mma_ts(tmem_O, p_tmem + kk * 8, bd, IDESC_PV, (u > 0 || kk > 0) ? 1u : 0u);
-            }
+            mma_pv_tile(tmem_O, tmem_base + S_COL + 64 * b, b ? v_desc1 : v_desc0, IDESC_PV, u > 0 ? 1u : 0u);
             tc_commit(&bars[B_ODONE]);
             tc_commit(&bars[B_VEMPTY + b]);
           }
