@@ -555,12 +555,33 @@ __global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__
 
 // ---------------------------------------------------------------------------
 // VS estimate: logits of the last Lq rows against one chunk of keys, bf16
-// mma.sync m16n8k16 with fp32 accumulate.
-//   PASS 1: per-row max and sum of exp over the chunk -> partials
-//   PASS 2: p = exp(l - m_i) / l_i; v[j] (column sums, owned by this CTA) and
-//           s[o] (diagonal sums, global atomics at the chunk edges)
+// mma.sync m16n8k16 with fp32 accumulate, in log2 units (x = tau log2(e) q.k,
+// so every exponential is one ex2).
+//   PASS 1: per-row max and sum of 2^(x - max) over the chunk -> partials
+//   PASS 2: p = 2^(x - m_i) / l_i into a shared fp32 tile; v[j] (column sums,
+//           owned by this CTA) and s[o] (diagonal sums: one thread per offset
+//           over the rows that offset meets, global atomics at the chunk edges)
+// K sub-tiles arrive by cp.async (zero-filled past the end) into one buffer,
+// refilled as soon as the sub-tile's MMAs have read it, so the next load
+// overlaps the exponentials and the sums.
 // Rows padded to LP = 16 * RT; warps: RT row tiles x (8 / RT) key groups.
 // ---------------------------------------------------------------------------
+// 16 bytes global -> shared, asynchronously; src_bytes = 0 writes zeros
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
+               "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
 
 template <int D, int RT, int PASS>
 __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, Layout L, const __nv_bfloat16* Q,
@@ -571,9 +592,10 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   constexpr int KPW = VS_SUB / WPR;      // keys per warp per sub-tile
   constexpr int NT = KPW / 8;            // n-tiles per warp
   constexpr int DP = D + 8;              // padded smem row (bf16)
-  constexpr int PP = VS_SUB + 4;         // padded fp32 row of the P tile
+  constexpr int CH = D / 8;              // 16-byte pieces per row
   extern __shared__ uint8_t smraw[];
   __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smraw);          // [LP][DP]
+  constexpr int PP = VS_SUB + 4;         // padded fp32 row of the P tile
   __nv_bfloat16* ks = qs + LP * DP;                                      // [VS_SUB][DP]
   float* ps = reinterpret_cast<float*>(ks + VS_SUB * DP);                // [LP][PP] (pass 2)
   float* sbuf = ps + LP * PP;                                            // [VS_CHUNK + LP]
@@ -591,13 +613,28 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   const int i0 = L.N - Lq;  // first estimate row
   const int j0 = chunk * VS_CHUNK;
   const int j1 = min(L.N, j0 + VS_CHUNK);
-  const float tau = rsqrtf((float)D);
+  const float sc = 1.4426950408889634f * rsqrtf((float)D);  // tau * log2(e)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rt = warp % RT, kg = warp / RT;
+  const int g = lane >> 2, t4 = lane & 3;
+  const __nv_bfloat16* kbase = K + kvh * k_hs;
+
+  auto load_sub = [&](int sub) {
+    __nv_bfloat16* dst = ks;
+#pragma unroll
+    for (int it = 0; it < VS_SUB * CH / 256; ++it) {
+      const int idx = it * 256 + tid;
+      const int r = idx / CH, c = (idx % CH) * 8;
+      const bool in = sub + r < j1;
+      cp_async16(dst + r * DP + c, kbase + (int64_t)(in ? sub + r : j0) * k_ts + c, in ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  load_sub(j0);
 
   // Q rows (padding rows are zero)
-  for (int idx = tid; idx < LP * (D / 8); idx += 256) {
-    const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
+  for (int idx = tid; idx < LP * CH; idx += 256) {
+    const int r = idx / CH, c = (idx % CH) * 8;
     uint4 v = make_uint4(0, 0, 0, 0);
     if (r < Lq) v = *reinterpret_cast<const uint4*>(Q + h * q_hs + (int64_t)(i0 + r) * q_ts + c);
     *reinterpret_cast<uint4*>(qs + r * DP + c) = v;
@@ -617,7 +654,7 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   // A fragments of this warp's row tile, kept in registers
   uint32_t af[D / 16][4];
   {
-    const int g = lane >> 2, q = (lane & 3) * 2;
+    const int q = t4 * 2;
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
       const __nv_bfloat16* base = qs + (rt * 16) * DP + kk * 16;
@@ -627,40 +664,48 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
       af[kk][3] = *reinterpret_cast<const uint32_t*>(base + (g + 8) * DP + q + 8);
     }
   }
+  const int rA = rt * 16 + g;  // this thread's two rows: rA, rA + 8
+  float rm[2] = {0.f, 0.f}, rl[2] = {0.f, 0.f};
+  if (PASS == 2) {
+    rm[0] = rowm[rA];
+    rm[1] = rowm[rA + 8];
+    rl[0] = rowl[rA];
+    rl[1] = rowl[rA + 8];
+  }
   float run_m[2] = {-INFINITY, -INFINITY}, run_l[2] = {0.f, 0.f};
-  const int rA = rt * 16 + (lane >> 2);  // this thread's two rows: rA, rA + 8
-  for (int sub = j0; sub < j1; sub += VS_SUB) {
+  const int obase = i0 - (j0 + VS_CHUNK - 1);  // sbuf index of offset o is o - obase
+  const int nsub = (j1 - j0 + VS_SUB - 1) / VS_SUB;
+  for (int si = 0; si < nsub; ++si) {
+    const int sub = j0 + si * VS_SUB;
+    cp_async_wait<0>();
     __syncthreads();
-    for (int idx = tid; idx < VS_SUB * (D / 8); idx += 256) {
-      const int r = idx / (D / 8), c = (idx % (D / 8)) * 8;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (sub + r < j1) v = *reinterpret_cast<const uint4*>(K + kvh * k_hs + (int64_t)(sub + r) * k_ts + c);
-      *reinterpret_cast<uint4*>(ks + r * DP + c) = v;
-    }
-    __syncthreads();
+    const __nv_bfloat16* kt = ks;
     float acc[NT][4];
 #pragma unroll
     for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
-      const int key = kg * KPW + n * 8 + (lane >> 2);
+      const int key = kg * KPW + n * 8 + g;
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
-        const __nv_bfloat16* kb = ks + key * DP + kk * 16 + (lane & 3) * 2;
+        const __nv_bfloat16* kb = kt + key * DP + kk * 16 + t4 * 2;
         const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
         const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
         mma_bf16_16816(acc[n], af[kk], b0, b1);
       }
     }
-    // logits -> natural units, masked (row < Lq, key <= row, key < N)
+    __syncthreads();  // every warp has read the sub-tile: refill the buffer
+    if (si + 1 < nsub) load_sub(sub + VS_SUB);
+    // logits in log2 units, masked (row < Lq, key <= row, key < N)
+    const int cb = sub + kg * KPW + t4 * 2;  // column of element (n = 0, e = 0)
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int r = rA + ((e >> 1) << 3);
-        const int j = sub + kg * KPW + n * 8 + (lane & 3) * 2 + (e & 1);
+        const int j = cb + n * 8 + (e & 1);
         const bool ok = (r < Lq) && (j < j1) && (j <= i0 + r);
-        acc[n][e] = ok ? acc[n][e] * tau : -INFINITY;
+        acc[n][e] = ok ? acc[n][e] * sc : -INFINITY;
       }
     }
     if (PASS == 1) {
@@ -676,48 +721,49 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
         float s = 0.f;
         if (live) {
 #pragma unroll
-          for (int n = 0; n < NT; ++n) s += expf(acc[n][2 * hr] - mnew) + expf(acc[n][2 * hr + 1] - mnew);
+          for (int n = 0; n < NT; ++n) s += ex2_approx(acc[n][2 * hr] - mnew) + ex2_approx(acc[n][2 * hr + 1] - mnew);
         }
         s += __shfl_xor_sync(0xffffffffu, s, 1);
         s += __shfl_xor_sync(0xffffffffu, s, 2);
         if (live) {
-          run_l[hr] = run_l[hr] * expf(run_m[hr] - mnew) + s;
+          run_l[hr] = run_l[hr] * ex2_approx(run_m[hr] - mnew) + s;
           run_m[hr] = mnew;
         }
       }
     } else {
-      // p into the fp32 tile, then column and diagonal sums
+      // p into the fp32 tile (masked entries are -inf -> 0)
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int r = rA + ((e >> 1) << 3);
-          const int c = kg * KPW + n * 8 + (lane & 3) * 2 + (e & 1);
-          ps[r * PP + c] = (acc[n][e] == -INFINITY) ? 0.f : expf(acc[n][e] - rowm[r]) * rowl[r];
+          const int c = kg * KPW + n * 8 + t4 * 2 + (e & 1);
+          ps[r * PP + c] = ex2_approx(acc[n][e] - rm[e >> 1]) * rl[e >> 1];
         }
       }
       __syncthreads();
       if (tid < VS_SUB) {
         float cs = 0.f;
+#pragma unroll 8
         for (int r = 0; r < LP; ++r) cs += ps[r * PP + tid];
         vbuf[sub - j0 + tid] += cs;
       }
-      // offsets of this sub-tile: o = (i0 + r) - (sub + c); index into sbuf by
-      // t = o - (i0 - (j0 + VS_CHUNK - 1)), c = (i0 + r) - o - sub
-      const int obase = i0 - (j0 + VS_CHUNK - 1);
+      // offset o meets row r at column c = i0 + r - o - sub, i.e. the rows
+      // [o + sub - i0, o + sub - i0 + VS_SUB) of the tile; neighbouring threads
+      // read neighbouring columns of each row
       for (int o = i0 - (sub + VS_SUB - 1) + tid; o <= i0 + LP - 1 - sub; o += 256) {
+        const int base = o + sub - i0;
+        const int rlo = max(0, base), rhi = min(LP, base + VS_SUB);
         float acc_s = 0.f;
-        for (int r = 0; r < LP; ++r) {
-          const int c = i0 + r - o - sub;
-          if (c >= 0 && c < VS_SUB) acc_s += ps[r * PP + c];
-        }
+        for (int r = rlo; r < rhi; ++r) acc_s += ps[r * PP + (r - base)];
         sbuf[o - obase] += acc_s;
       }
     }
+    __syncthreads();  // the P tile and the sums are done before the next sub-tile
   }
   if (PASS == 1) {
     // combine the key-group warps of each row tile
-    if ((lane & 3) == 0) {
+    if (t4 == 0) {
 #pragma unroll
       for (int hr = 0; hr < 2; ++hr) {
         wpart[(kg * LP + rA + 8 * hr) * 2 + 0] = run_m[hr];
@@ -727,12 +773,12 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
     __syncthreads();
     for (int r = tid; r < Lq; r += 256) {
       float m = -INFINITY;
-      for (int g = 0; g < WPR; ++g) m = fmaxf(m, wpart[(g * LP + r) * 2]);
+      for (int gw = 0; gw < WPR; ++gw) m = fmaxf(m, wpart[(gw * LP + r) * 2]);
       float l = 0.f;
       if (m != -INFINITY)
-        for (int g = 0; g < WPR; ++g) {
-          const float gm = wpart[(g * LP + r) * 2];
-          if (gm != -INFINITY) l += wpart[(g * LP + r) * 2 + 1] * expf(gm - m);
+        for (int gw = 0; gw < WPR; ++gw) {
+          const float gm = wpart[(gw * LP + r) * 2];
+          if (gm != -INFINITY) l += wpart[(gw * LP + r) * 2 + 1] * ex2_approx(gm - m);
         }
       float* pp = part + (((int64_t)vslot * L.vs_nchunks + chunk) * VS_MAXL + r) * 2;
       pp[0] = m;
@@ -743,7 +789,6 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
     float* vout = reinterpret_cast<float*>(ws + L.off_v) + (int64_t)vslot * L.N;
     float* sout = reinterpret_cast<float*>(ws + L.off_s) + (int64_t)vslot * L.N;
     for (int j = j0 + tid; j < j1; j += 256) vout[j] = vbuf[j - j0];
-    const int obase = i0 - (j0 + VS_CHUNK - 1);
     for (int t = tid; t < VS_CHUNK + LP; t += 256) {
       const int o = obase + t;
       const float val = sbuf[t];
@@ -752,7 +797,7 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   }
 }
 
-// merge the per-chunk (max, sum) partials into the row softmax statistics
+// merge the per-chunk (max, sum) partials (log2 units) into the row softmax statistics
 __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws) {
   const int vslot = blockIdx.x;
   const int h = ht.vhead[vslot];
@@ -766,7 +811,7 @@ __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint
     float l = 0.f;
     for (int c = 0; c < L.vs_nchunks; ++c) {
       const float* pp = part + (((int64_t)vslot * L.vs_nchunks + c) * VS_MAXL + r) * 2;
-      if (pp[0] != -INFINITY) l += pp[1] * expf(pp[0] - m);
+      if (pp[0] != -INFINITY) l += pp[1] * exp2f(pp[0] - m);
     }
     stat[((int64_t)vslot * VS_MAXL + r) * 2 + 0] = m;
     stat[((int64_t)vslot * VS_MAXL + r) * 2 + 1] = l;
@@ -799,48 +844,60 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
   ordered_select(load, L.N, T, take_eq, red, [&](int i, int pos) { out[pos] = i; });
 }
 
-// block distances D of one VS head: {floor(o/B), ceil(o/B)} for the chosen slashes
-__global__ void k_vs_dist(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws, const int32_t* slash_idx,
-                          int slash_stride, int32_t* dist_ptr) {
+// block distances D of one VS head: {floor(o/B), ceil(o/B)} for the chosen
+// slashes.  One flag byte per key block (plain stores: every writer writes 1),
+// then one bitmap word per 32 blocks from a warp ballot, and the ascending list
+// from a scan of the per-word counts.  Dynamic shared memory: nkw * 32 bytes.
+__global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+                                                  const int32_t* slash_idx, int slash_stride, int32_t* dist_ptr) {
+  extern __shared__ uint8_t flag[];
+  __shared__ int wofs[1025];  // nkw <= 1024 (N <= 2^21, B >= 64)
   const int vslot = blockIdx.x;
   const int h = ht.vhead[vslot];
   uint32_t* dbits = reinterpret_cast<uint32_t*>(ws + L.off_dbits) + (int64_t)vslot * L.nkw;
   int32_t* dtmp = reinterpret_cast<int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.nqb;
-  for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) dbits[w] = 0u;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  for (int i = threadIdx.x; i < L.nkw * 8; i += blockDim.x) reinterpret_cast<uint32_t*>(flag)[i] = 0u;
   __syncthreads();
   const int ns = min(ht.n_slash[h], L.N);
   for (int t = threadIdx.x; t < ns; t += blockDim.x) {
     const int o = slash_idx[(int64_t)h * slash_stride + t];
     if (o < 0) continue;
     const int lo = o / L.B, hi = (o + L.B - 1) / L.B;
-    if (lo < L.nqb) atomicOr(&dbits[lo >> 5], 1u << (lo & 31));
-    if (hi < L.nqb) atomicOr(&dbits[hi >> 5], 1u << (hi & 31));
+    if (lo < L.nqb) flag[lo] = 1;
+    if (hi < L.nqb) flag[hi] = 1;
   }
-  __threadfence_block();
   __syncthreads();
-  // ascending compaction by one warp (word order), counts via popc
-  if (threadIdx.x < 32) {
-    int base = 0;
+  for (int w = warp; w < L.nkw; w += nw) {
+    const unsigned bits = __ballot_sync(0xffffffffu, flag[w * 32 + lane] != 0);
+    if (lane == 0) {
+      dbits[w] = bits;
+      wofs[w] = __popc(bits);
+    }
+  }
+  __syncthreads();
+  if (warp == 0) {
+    // exclusive scan of the per-word counts
+    int carry = 0;
     for (int w0 = 0; w0 < L.nkw; w0 += 32) {
-      const int w = w0 + threadIdx.x;
-      const uint32_t bits = (w < L.nkw) ? dbits[w] : 0u;
-      const int c = __popc(bits);
+      const int w = w0 + lane;
+      const int c = (w < L.nkw) ? wofs[w] : 0;
       int incl = c;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if ((int)threadIdx.x >= o) incl += y;
+        if (lane >= o) incl += y;
       }
-      int pos = base + incl - c;
-      uint32_t b = bits;
-      while (b) {
-        const int bit = __ffs(b) - 1;
-        b &= b - 1u;
-        dtmp[pos++] = w * 32 + bit;
-      }
-      base += __shfl_sync(0xffffffffu, incl, 31);
+      if (w < L.nkw) wofs[w] = carry + incl - c;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
     }
-    if (threadIdx.x == 0) dist_ptr[1 + h] = base;
+    if (lane == 0) dist_ptr[1 + h] = carry;
+  }
+  __syncthreads();
+  for (int w = warp; w < L.nkw; w += nw) {
+    const bool f = flag[w * 32 + lane] != 0;
+    const unsigned bits = __ballot_sync(0xffffffffu, f);
+    if (f) dtmp[wofs[w] + __popc(bits & ((1u << lane) - 1u))] = w * 32 + lane;
   }
 }
 
@@ -1310,7 +1367,7 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
     if (s != DSA_OK) return s;
     k_vs_topk<<<dim3(L.nvs, 2), 1024, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride, out.slash_idx,
                                                 out.slash_stride);
-    k_vs_dist<<<L.nvs, 256, 0, st>>>(ht, L, ws, out.slash_idx, out.slash_stride, out.dist_ptr);
+    k_vs_dist<<<L.nvs, 1024, L.nkw * 32, st>>>(ht, L, ws, out.slash_idx, out.slash_stride, out.dist_ptr);
     k_vs_cols<false><<<dim3(ceil_div(L.nqb, 8), L.nvs), 256, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride,
                                                                       out.col_ptr, out.col_idx, out.col_cap, status);
   }
