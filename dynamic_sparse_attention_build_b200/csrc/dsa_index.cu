@@ -75,19 +75,31 @@ __device__ __forceinline__ uint32_t fkey(float f) {
 // Exact top-k of vals[0..n) (ties to the lower index), n > k >= 1.  Finds the
 // k-th largest key T by 4 radix passes of 8 bits, and how many keys equal to T
 // to take.  hist: shared int[256 * nwarps]; red: shared int[64].
+constexpr int RB = 8;  // keys loaded per thread before use in the CTA-wide select
+
 template <typename Loader>
 __device__ void radix_kth(const Loader& load, int n, int k, int* hist, int* red, uint32_t* T_out,
                           int* take_eq_out) {
   const int nw = blockDim.x >> 5;
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint32_t prefix = 0, mask = 0;
   int need = k;
   for (int shift = 24; shift >= 0; shift -= 8) {
     for (int i = threadIdx.x; i < 256 * nw; i += blockDim.x) hist[i] = 0;
     __syncthreads();
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-      const uint32_t key = fkey(load(i));
-      if ((key & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key >> shift) & 255u)], 1);
+    // RB independent loads in flight per thread before their keys are counted
+    for (int i0 = 0; i0 < n; i0 += RB * blockDim.x) {
+      uint32_t key[RB];
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        const int i = i0 + q * blockDim.x + threadIdx.x;
+        key[q] = (i < n) ? fkey(load(i)) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        const int i = i0 + q * blockDim.x + threadIdx.x;
+        if (i < n && (key[q] & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key[q] >> shift) & 255u)], 1);
+      }
     }
     __syncthreads();
     for (int b = threadIdx.x; b < 256; b += blockDim.x) {
@@ -96,15 +108,41 @@ __device__ void radix_kth(const Loader& load, int n, int k, int* hist, int* red,
       hist[b] = s;
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int above = 0;
-      int digit = 0;
-      for (int b = 255; b >= 0; --b) {
-        if (above + hist[b] >= need) { digit = b; break; }
-        above += hist[b];
+    if (warp == 0) {
+      // the digit whose bin takes the count from the top past `need`: lane l
+      // holds bins 255 - 8l .. 248 - 8l, a warp scan gives the count above them
+      int c[8], tot = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        c[q] = hist[255 - (lane * 8 + q)];
+        tot += c[q];
       }
-      red[0] = digit;
-      red[1] = above;
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int above = incl - tot, digit = -1, ab = 0;
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (digit < 0) {
+          if (above + c[q] >= need) {
+            digit = 255 - (lane * 8 + q);
+            ab = above;
+          } else {
+            above += c[q];
+          }
+        }
+      }
+      const unsigned found = __ballot_sync(0xffffffffu, digit >= 0);
+      const int src = __ffs(found) - 1;  // the candidates always hold `need` keys
+      digit = __shfl_sync(0xffffffffu, digit, src);
+      ab = __shfl_sync(0xffffffffu, ab, src);
+      if (lane == 0) {
+        red[0] = digit;
+        red[1] = ab;
+      }
     }
     __syncthreads();
     prefix |= (uint32_t)red[0] << shift;
@@ -126,10 +164,17 @@ __device__ void ordered_select(const Loader& load, int n, uint32_t T, int take_e
   const int seg = ceil_div(ceil_div(n, nw), 32) * 32;
   const int beg = min(n, warp * seg), end = min(n, beg + seg);
   int gt = 0, eq = 0;
-  for (int i = beg + lane; i < end; i += 32) {
-    const uint32_t key = fkey(load(i));
-    gt += key > T;
-    eq += key == T;
+  for (int i0 = beg + lane; i0 < end; i0 += 32 * RB) {
+    uint32_t key[RB];
+#pragma unroll
+    for (int q = 0; q < RB; ++q) key[q] = (i0 + 32 * q < end) ? fkey(load(i0 + 32 * q)) : 0u;
+#pragma unroll
+    for (int q = 0; q < RB; ++q) {
+      if (i0 + 32 * q < end) {
+        gt += key[q] > T;
+        eq += key[q] == T;
+      }
+    }
   }
   gt = warp_sum_int(gt);
   eq = warp_sum_int(eq);
@@ -148,11 +193,20 @@ __device__ void ordered_select(const Loader& load, int n, uint32_t T, int take_e
   __syncthreads();
   int eq_run = eq_base;
   int pos = out_base;
+  uint32_t kb[RB];
   for (int i0 = beg; i0 < end; i0 += 32) {
     const int i = i0 + lane;
+    const int q = ((i0 - beg) >> 5) % RB;
+    if (q == 0) {
+#pragma unroll
+      for (int u = 0; u < RB; ++u) kb[u] = (i + 32 * u < end) ? fkey(load(i + 32 * u)) : 0u;
+    }
+    uint32_t key = kb[0];
+#pragma unroll
+    for (int u = 1; u < RB; ++u)
+      if (q == u) key = kb[u];
     bool sel = false, iseq = false;
     if (i < end) {
-      const uint32_t key = fkey(load(i));
       iseq = key == T;
       sel = key > T;
     }
@@ -902,40 +956,63 @@ __global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTa
 }
 
 // columns of (VS head, query block): j in V, j <= qb*B+B-1, (qb - j/B) not in D.
-// One warp per query block.  FILL=false writes counts, FILL=true writes lists.
+// One warp per query block, eight per CTA; the CTA stages the D bitmap and a
+// window of the (ascending) vertical list in shared memory once for its warps.
+// FILL=false writes counts, FILL=true writes lists.
 template <bool FILL>
-__global__ void k_vs_cols(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws, const int32_t* vert_idx,
-                          int vert_stride, int32_t* col_ptr, int32_t* col_idx, int64_t col_cap, unsigned* status) {
+__global__ void __launch_bounds__(256) k_vs_cols(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+                                                 const int32_t* vert_idx, int vert_stride, int32_t* col_ptr,
+                                                 int32_t* col_idx, int64_t col_cap, unsigned* status) {
+  constexpr int WIN = 1024;
+  __shared__ int32_t vwin[WIN];
+  __shared__ uint32_t dsh[1024];  // nkw <= 1024
   const int vslot = blockIdx.y;
   const int h = ht.vhead[vslot];
-  const int qb = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (qb >= L.nqb) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = blockIdx.x * 8 + warp;
+  const int qb_last = min(L.nqb - 1, blockIdx.x * 8 + 7);
+  const int lim_cta = qb_last * L.B + L.B - 1;
   const uint32_t* dbits = reinterpret_cast<const uint32_t*>(ws + L.off_dbits) + (int64_t)vslot * L.nkw;
+  for (int w = threadIdx.x; w < L.nkw; w += blockDim.x) dsh[w] = dbits[w];
   const int32_t* V = vert_idx + (int64_t)h * vert_stride;
   const int nv = min(ht.n_vert[h], L.N);
   const int lim = qb * L.B + L.B - 1;
   const int row = h * L.nqb + qb;
-  int pos = FILL ? col_ptr[row] : 0;
-  const int end = FILL ? col_ptr[row + 1] : 0;
-  if (FILL && end > col_cap) {
-    if (lane == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_COL);
-    return;
-  }
-  for (int t0 = 0; t0 < nv; t0 += 32) {
-    const int t = t0 + lane;
-    const int j = (t < nv) ? V[t] : -1;
-    bool take = false;
-    if (j >= 0 && j <= lim) {
-      const int delta = qb - j / L.B;
-      take = !((dbits[delta >> 5] >> (delta & 31)) & 1u);
+  bool active = qb < L.nqb;
+  int pos = 0;
+  if (FILL && active) {
+    pos = col_ptr[row];
+    if (col_ptr[row + 1] > col_cap) {
+      if (lane == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_COL);
+      active = false;
     }
-    const unsigned m = __ballot_sync(0xffffffffu, take);
-    if (FILL && take) col_idx[pos + __popc(m & ((1u << lane) - 1u))] = j;
-    pos += __popc(m);
-    if (__shfl_sync(0xffffffffu, j, 31) > lim) break;  // V is ascending
   }
-  if (!FILL && lane == 0) col_ptr[1 + row] = pos;
+  for (int c0 = 0; c0 < nv; c0 += WIN) {
+    const int cn = min(WIN, nv - c0);
+    __syncthreads();  // the previous window is consumed (and dsh is written)
+    for (int t = threadIdx.x; t < cn; t += blockDim.x) vwin[t] = V[c0 + t];
+    __syncthreads();
+    if (active) {
+      for (int t0 = 0; t0 < cn; t0 += 32) {
+        const int t = t0 + lane;
+        const int j = (t < cn) ? vwin[t] : -1;
+        bool take = false;
+        if (j >= 0 && j <= lim) {
+          const int delta = qb - j / L.B;
+          take = !((dsh[delta >> 5] >> (delta & 31)) & 1u);
+        }
+        const unsigned m = __ballot_sync(0xffffffffu, take);
+        if (FILL && take) col_idx[pos + __popc(m & ((1u << lane) - 1u))] = j;
+        pos += __popc(m);
+        if (__shfl_sync(0xffffffffu, j, 31) > lim) {  // V is ascending
+          active = false;
+          break;
+        }
+      }
+    }
+    if (vwin[cn - 1] > lim_cta) break;  // no query block of this CTA reads further
+  }
+  if (!FILL && lane == 0 && qb < L.nqb) col_ptr[1 + row] = pos;
 }
 
 // in-place inclusive scan of ptr[0..n) (ptr[0] == 0, ptr[r+1] == count of row r)
