@@ -139,3 +139,38 @@ def test_repeat_runs_are_bit_identical(dsa):
     for O, lse in outs[1:]:
         assert torch.equal(O, outs[0][0])
         assert torch.equal(lse, outs[0][1])
+
+
+@pytest.mark.parametrize("kind", ["dense", "vs"])
+def test_large_logit_jumps(dsa, kind):
+    """Keys with very large logits after a row's first tile: the running max of
+    the online softmax then grows by far more than its raise threshold (2^32 in
+    base 2), so O and l are rescaled mid-row (and, for the VS head, columns add
+    keys after the block tiles)."""
+    N, d, B = 640, 128, 64
+    Q, K, V = synth.random_qkv(2, 1, N, d, seed=11)
+    g = torch.Generator().manual_seed(12)
+    u = torch.randn(d, generator=g)
+    u = u / u.norm()
+    Kf = K.float()
+    # keys 200, 333 and 517 point along u with norm 500: logit ~ 44 * (q . u),
+    # i.e. jumps of tens of natural units (x 1.44 in base 2) for many rows
+    for j, a in ((200, 500.0), (333, -300.0), (517, 700.0)):
+        Kf[0, j] = a * u
+    K = Kf.to(torch.bfloat16)
+    nb = (N + B - 1) // B
+    if kind == "dense":
+        pats = [dict(kind="block_topk", topk=nb)] * 2
+    else:
+        pats = [dict(kind="vs", last_q=64, n_vert=40, n_slash=12)] * 2
+    heads = orc.build_indices(to64(Q), to64(K), pats, B)
+    if kind == "vs":
+        # make sure the planted keys are columns of some query blocks
+        for hi in heads:
+            for qb in range(nb):
+                extra = [j for j in (200, 333, 517) if j <= qb * B + B - 1]
+                hi.cols[qb] = np.unique(np.concatenate([hi.cols[qb], np.asarray(extra, np.int64)]))
+    # the oracle's rows really do see such jumps
+    lg = to64(Q)[0] @ to64(K)[0].T / np.sqrt(d)
+    assert (lg[:, 517] - lg[:, :64].max(axis=1) > 32 / np.log2(np.e)).sum() > 20
+    run_case(dsa, Q, K, V, heads, B)
