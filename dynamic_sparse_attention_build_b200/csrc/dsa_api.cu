@@ -17,6 +17,7 @@ constexpr int kMaxDevices = 64;
 unsigned* g_status_addr[kMaxDevices] = {};
 
 __global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns) {
+  pdl_prologue();
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {

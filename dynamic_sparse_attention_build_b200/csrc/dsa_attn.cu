@@ -325,6 +325,7 @@ template <int D>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
+  pdl_prologue();
   using L = Smem<D>;
   constexpr int DS = L::DS;
   extern __shared__ uint8_t smem_raw[];
@@ -1059,8 +1060,8 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = n_items < 2 * sms ? n_items : 2 * sms;
-  sparse_attn_kernel<D><<<grid, NTHREADS, smem, stream>>>(mq, mk, mv, a);
-  e = cudaGetLastError();
+  e = launch_pdl(sparse_attn_kernel<D>, dim3(grid), dim3(NTHREADS), (size_t)smem, stream, mq, mk, mv, a);
+  if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;
 }

@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "dsa.h"
 
 namespace dsa {
@@ -146,6 +148,36 @@ __device__ __forceinline__ bool mbar_wait_ool(uint64_t* bar, uint32_t parity, ui
                                               volatile int* abort_flag, bool suspend = false) {
   if (mbar_test_wait(bar, parity)) return true;
   return mbar_wait_loop(bar, parity, limit_ns, status, detail, abort_flag, suspend);
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  Every kernel of the library is launched with
+// programmatic stream serialization (launch_pdl below) and starts with
+// pdl_prologue(): it waits until the previous grid on the stream has completed
+// and its writes are visible (before touching global memory at all), then lets
+// the next grid be scheduled.  The next grid can only start once every CTA of
+// this one has started, so the waiting never holds resources a running CTA
+// needs; what overlaps is launch latency and the next kernel's set-up.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_prologue() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                              Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ---------------------------------------------------------------------------

@@ -223,9 +223,13 @@ __device__ void ordered_select(const Loader& load, int n, uint32_t T, int take_e
 // ---------------------------------------------------------------------------
 // head info + A-shape / block counts
 // ---------------------------------------------------------------------------
-__global__ void k_head_info(const __grid_constant__ HeadTab ht, int Hq, int32_t* head_info) {
+// also clears the distance-list counts of non-VS heads (and the leading zero)
+__global__ void k_head_info(const __grid_constant__ HeadTab ht, int Hq, int32_t* head_info, int32_t* dist_ptr) {
+  pdl_prologue();
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h >= Hq) return;
+  if (h == 0) dist_ptr[0] = 0;
+  if (ht.kind[h] != DSA_KIND_VS) dist_ptr[1 + h] = 0;
   head_info[h * 4 + 0] = ht.kind[h];
   head_info[h * 4 + 1] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.sink[h] : 0;
   head_info[h * 4 + 2] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.window[h] : 0;
@@ -239,11 +243,22 @@ __device__ __forceinline__ void ashape_range(int qb, int B, int N, int sink, int
   *w = max(0, r0 - window + 1) / B;             // window blocks [w, qb]
 }
 
-__global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int32_t* blk_ptr) {
+// Block-list counts of A-shape heads; zero counts for the rows no later kernel
+// fills (block lists of VS heads, column lists of non-VS heads) and the leading
+// zeros of both pointer arrays.  Block-kind and VS counts are written later.
+__global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int32_t* blk_ptr, int32_t* col_ptr) {
+  pdl_prologue();
   const int h = blockIdx.y;
-  if (ht.kind[h] != DSA_KIND_ASHAPE) return;
   const int qb = blockIdx.x * blockDim.x + threadIdx.x;
   if (qb >= L.nqb) return;
+  const int kind = ht.kind[h];
+  if (h == 0 && qb == 0) {
+    blk_ptr[0] = 0;
+    col_ptr[0] = 0;
+  }
+  if (kind != DSA_KIND_VS) col_ptr[1 + h * L.nqb + qb] = 0;
+  if (kind == DSA_KIND_VS) blk_ptr[1 + h * L.nqb + qb] = 0;
+  if (kind != DSA_KIND_ASHAPE) return;
   int a, w;
   ashape_range(qb, L.B, L.N, ht.sink[h], ht.window[h], &a, &w);
   const int cnt = a + (qb + 1 - max(w, a) > 0 ? qb + 1 - max(w, a) : 0);
@@ -258,6 +273,7 @@ __global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int
 template <int D>
 __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct, Layout L,
                                               const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws) {
+  pdl_prologue();
   constexpr int TPR = D / 8;          // threads per row, 8 channels each
   constexpr int RG = 256 / TPR;       // rows in flight
   __shared__ float part[RG][D];
@@ -437,6 +453,7 @@ template <int D>
 __global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__ HeadTab ht, Layout L,
                                                       const __nv_bfloat16* Q, int64_t q_hs, int64_t q_ts,
                                                       uint8_t* ws, int32_t* blk_ptr, int ri) {
+  pdl_prologue();
   extern __shared__ float sc[];  // [SEL_RI][SEL_RS(npad)] scores of the group's rows
   __shared__ int hist[SEL_NW][256];
   const int npad = L.nkw * 32;
@@ -641,6 +658,7 @@ template <int D, int RT, int PASS>
 __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, Layout L, const __nv_bfloat16* Q,
                                             int64_t q_hs, int64_t q_ts, const __nv_bfloat16* K, int64_t k_hs,
                                             int64_t k_ts, uint8_t* ws) {
+  pdl_prologue();
   constexpr int LP = 16 * RT;
   constexpr int WPR = 8 / RT;            // warps per row tile
   constexpr int KPW = VS_SUB / WPR;      // keys per warp per sub-tile
@@ -695,6 +713,11 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   }
   float* part = reinterpret_cast<float*>(ws + L.off_part);
   float* stat = reinterpret_cast<float*>(ws + L.off_stat);
+  if (PASS == 1) {
+    // pass 2 adds its diagonal sums into s with atomics: clear this chunk of it
+    float* sout = reinterpret_cast<float*>(ws + L.off_s) + (int64_t)vslot * L.N;
+    for (int j = j0 + tid; j < j1; j += 256) sout[j] = 0.f;
+  }
   if (PASS == 2) {
     for (int i = tid; i < VS_CHUNK + LP; i += 256) sbuf[i] = 0.f;
     for (int i = tid; i < VS_CHUNK; i += 256) vbuf[i] = 0.f;
@@ -853,6 +876,7 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
 
 // merge the per-chunk (max, sum) partials (log2 units) into the row softmax statistics
 __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws) {
+  pdl_prologue();
   const int vslot = blockIdx.x;
   const int h = ht.vhead[vslot];
   const int Lq = min(ht.last_q[h], L.N);
@@ -876,6 +900,7 @@ __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint
 __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                   int32_t* vert_idx, int vert_stride, int32_t* slash_idx,
                                                   int slash_stride) {
+  pdl_prologue();
   __shared__ int hist[256 * 32];
   __shared__ int red[80];
   const int vslot = blockIdx.x;
@@ -904,6 +929,7 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
 // from a scan of the per-word counts.  Dynamic shared memory: nkw * 32 bytes.
 __global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                   const int32_t* slash_idx, int slash_stride, int32_t* dist_ptr) {
+  pdl_prologue();
   extern __shared__ uint8_t flag[];
   __shared__ int wofs[1025];  // nkw <= 1024 (N <= 2^21, B >= 64)
   const int vslot = blockIdx.x;
@@ -963,6 +989,7 @@ template <bool FILL>
 __global__ void __launch_bounds__(256) k_vs_cols(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                  const int32_t* vert_idx, int vert_stride, int32_t* col_ptr,
                                                  int32_t* col_idx, int64_t col_cap, unsigned* status) {
+  pdl_prologue();
   constexpr int WIN = 1024;
   __shared__ int32_t vwin[WIN];
   __shared__ uint32_t dsh[1024];  // nkw <= 1024
@@ -1018,6 +1045,7 @@ __global__ void __launch_bounds__(256) k_vs_cols(const __grid_constant__ HeadTab
 // in-place inclusive scan of ptr[0..n) (ptr[0] == 0, ptr[r+1] == count of row r)
 __global__ void __launch_bounds__(1024) k_scan(int32_t* p0, int n0, int64_t cap0, int32_t* p1, int n1, int64_t cap1,
                                                int32_t* p2, int n2, int64_t cap2, unsigned* status) {
+  pdl_prologue();
   __shared__ int wsum[32];
   int32_t* p = blockIdx.x == 0 ? p0 : (blockIdx.x == 1 ? p1 : p2);
   const int n = blockIdx.x == 0 ? n0 : (blockIdx.x == 1 ? n1 : n2);
@@ -1053,6 +1081,7 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* p0, int n0, int64_t cap0
 // fill block lists: A-shape closed form, block kinds from the selection bitmap
 __global__ void k_blk_fill(const __grid_constant__ HeadTab ht, Layout L, const uint8_t* ws, const int32_t* blk_ptr,
                            int32_t* blk_idx, int64_t blk_cap, unsigned* status) {
+  pdl_prologue();
   const int h = blockIdx.y;
   const int kind = ht.kind[h];
   if (kind == DSA_KIND_VS) return;
@@ -1100,6 +1129,7 @@ __global__ void k_blk_fill(const __grid_constant__ HeadTab ht, Layout L, const u
 
 __global__ void k_dist_fill(const __grid_constant__ HeadTab ht, Layout L, const uint8_t* ws, const int32_t* dist_ptr,
                             int32_t* dist, int64_t dist_cap, unsigned* status) {
+  pdl_prologue();
   const int vslot = blockIdx.x;
   const int h = ht.vhead[vslot];
   const int beg = dist_ptr[h], end = dist_ptr[h + 1];
@@ -1148,6 +1178,7 @@ __device__ __forceinline__ int64_t ashape_pairs_in_block(int kb, int B, int r0, 
 __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head_info, const int32_t* blk_ptr,
                               const int32_t* blk_idx, const int32_t* dist_ptr, const int32_t* dist,
                               const int32_t* col_ptr, const int32_t* col_idx, unsigned long long* pairs) {
+  pdl_prologue();
   const int qb = blockIdx.x;
   const int h = blockIdx.y;
   const int kind = head_info[h * 4];
@@ -1366,9 +1397,9 @@ dsa_status launch_vs(const HeadTab& ht, const Layout& L, const void* Q, int64_t 
   do {                                                                                                     \
     cudaFuncSetAttribute(k_vs<D, R, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
     cudaFuncSetAttribute(k_vs<D, R, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
-    k_vs<D, R, 1><<<grid, 256, smem, st>>>(ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);                        \
-    k_vs_rowstats<<<L.nvs, 128, 0, st>>>(ht, L, ws);                                                       \
-    k_vs<D, R, 2><<<grid, 256, smem, st>>>(ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);                        \
+    launch_pdl(k_vs<D, R, 1>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
+    launch_pdl(k_vs_rowstats, dim3(L.nvs), dim3(128), 0, st, ht, L, ws);                                    \
+    launch_pdl(k_vs<D, R, 2>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
   } while (0)
   switch (RT) {
     case 1: DSA_VS_LAUNCH(1); break;
@@ -1411,51 +1442,55 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
     e = (x);                               \
     if (e != cudaSuccess) return cuda_fail(e); \
   } while (0)
-  DSA_CK(cudaMemsetAsync(out.blk_ptr, 0, sizeof(int32_t) * nrows, st));
-  DSA_CK(cudaMemsetAsync(out.col_ptr, 0, sizeof(int32_t) * nrows, st));
-  DSA_CK(cudaMemsetAsync(out.dist_ptr, 0, sizeof(int32_t) * (p.Hq + 1), st));
-  k_head_info<<<ceil_div(p.Hq, 128), 128, 0, st>>>(ht, p.Hq, out.head_info);
-  k_ashape_count<<<dim3(ceil_div(L.nqb, 128), p.Hq), 128, 0, st>>>(ht, L, out.blk_ptr);
+  // every kernel below starts with pdl_prologue(); the pointer arrays are
+  // cleared by k_head_info / k_ashape_count where no count kernel writes them
+  DSA_CK(launch_pdl(k_head_info, dim3(ceil_div(p.Hq, 128)), dim3(128), 0, st, ht, p.Hq, out.head_info, out.dist_ptr));
+  DSA_CK(launch_pdl(k_ashape_count, dim3(ceil_div(L.nqb, 128), p.Hq), dim3(128), 0, st, ht, L, out.blk_ptr,
+                    out.col_ptr));
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   if (L.nbh > 0) {
     if (p.d == 128) {
-      k_pool<128><<<dim3(L.nqb, p.Hkv), 256, 0, st>>>(ct, L, k, p.k_head_stride, p.k_token_stride, ws);
+      DSA_CK(launch_pdl(k_pool<128>, dim3(L.nqb, p.Hkv), dim3(256), 0, st, ct, L, k, p.k_head_stride,
+                        p.k_token_stride, ws));
       const int ri = sel_blocks_per_cta(p.block);
       const size_t sel_smem = sel_smem_bytes(128, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<128><<<dim3(ceil_div(L.nqb, ri), L.nbh), SEL_NT, sel_smem, st>>>(
-          ht, L, q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri);
+      DSA_CK(launch_pdl(k_block_select<128>, dim3(ceil_div(L.nqb, ri), L.nbh), dim3(SEL_NT), sel_smem, st, ht, L,
+                        q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri));
     } else {
-      k_pool<64><<<dim3(L.nqb, p.Hkv), 256, 0, st>>>(ct, L, k, p.k_head_stride, p.k_token_stride, ws);
+      DSA_CK(launch_pdl(k_pool<64>, dim3(L.nqb, p.Hkv), dim3(256), 0, st, ct, L, k, p.k_head_stride,
+                        p.k_token_stride, ws));
       const int ri = sel_blocks_per_cta(p.block);
       const size_t sel_smem = sel_smem_bytes(64, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
-      k_block_select<64><<<dim3(ceil_div(L.nqb, ri), L.nbh), SEL_NT, sel_smem, st>>>(
-          ht, L, q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri);
+      DSA_CK(launch_pdl(k_block_select<64>, dim3(ceil_div(L.nqb, ri), L.nbh), dim3(SEL_NT), sel_smem, st, ht, L,
+                        q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri));
     }
   }
   if (L.nvs > 0) {
-    DSA_CK(cudaMemsetAsync(ws + L.off_s, 0, (size_t)L.nvs * p.N * 4, st));
     s = (p.d == 128) ? launch_vs<128>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
                                       p.k_token_stride, ws, st)
                      : launch_vs<64>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
                                      p.k_token_stride, ws, st);
     if (s != DSA_OK) return s;
-    k_vs_topk<<<dim3(L.nvs, 2), 1024, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride, out.slash_idx,
-                                                out.slash_stride);
-    k_vs_dist<<<L.nvs, 1024, L.nkw * 32, st>>>(ht, L, ws, out.slash_idx, out.slash_stride, out.dist_ptr);
-    k_vs_cols<false><<<dim3(ceil_div(L.nqb, 8), L.nvs), 256, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride,
-                                                                      out.col_ptr, out.col_idx, out.col_cap, status);
+    DSA_CK(launch_pdl(k_vs_topk, dim3(L.nvs, 2), dim3(1024), 0, st, ht, L, ws, out.vert_idx, out.vert_stride,
+                      out.slash_idx, out.slash_stride));
+    DSA_CK(launch_pdl(k_vs_dist, dim3(L.nvs), dim3(1024), (size_t)L.nkw * 32, st, ht, L, ws, out.slash_idx,
+                      out.slash_stride, out.dist_ptr));
+    DSA_CK(launch_pdl(k_vs_cols<false>, dim3(ceil_div(L.nqb, 8), L.nvs), dim3(256), 0, st, ht, L, ws, out.vert_idx,
+                      out.vert_stride, out.col_ptr, out.col_idx, out.col_cap, status));
   }
-  k_scan<<<3, 1024, 0, st>>>(out.blk_ptr, nrows, out.blk_cap, out.col_ptr, nrows, out.col_cap, out.dist_ptr,
-                             p.Hq + 1, out.dist_cap, status);
-  k_blk_fill<<<dim3(ceil_div(L.nqb, 8), p.Hq), 256, 0, st>>>(ht, L, ws, out.blk_ptr, out.blk_idx, out.blk_cap,
-                                                            status);
+  DSA_CK(launch_pdl(k_scan, dim3(3), dim3(1024), 0, st, out.blk_ptr, nrows, out.blk_cap, out.col_ptr, nrows,
+                    out.col_cap, out.dist_ptr, p.Hq + 1, out.dist_cap, status));
+  DSA_CK(launch_pdl(k_blk_fill, dim3(ceil_div(L.nqb, 8), p.Hq), dim3(256), 0, st, ht, L,
+                    static_cast<const uint8_t*>(ws), static_cast<const int32_t*>(out.blk_ptr), out.blk_idx,
+                    out.blk_cap, status));
   if (L.nvs > 0) {
-    k_dist_fill<<<L.nvs, 256, 0, st>>>(ht, L, ws, out.dist_ptr, out.dist, out.dist_cap, status);
-    k_vs_cols<true><<<dim3(ceil_div(L.nqb, 8), L.nvs), 256, 0, st>>>(ht, L, ws, out.vert_idx, out.vert_stride,
-                                                                     out.col_ptr, out.col_idx, out.col_cap, status);
+    DSA_CK(launch_pdl(k_dist_fill, dim3(L.nvs), dim3(256), 0, st, ht, L, static_cast<const uint8_t*>(ws),
+                      static_cast<const int32_t*>(out.dist_ptr), out.dist, out.dist_cap, status));
+    DSA_CK(launch_pdl(k_vs_cols<true>, dim3(ceil_div(L.nqb, 8), L.nvs), dim3(256), 0, st, ht, L, ws, out.vert_idx,
+                      out.vert_stride, out.col_ptr, out.col_idx, out.col_cap, status));
   }
   DSA_CK(cudaGetLastError());
 #undef DSA_CK
