@@ -342,7 +342,11 @@ def main():
 
     pk, pk_src = peaks()
     tflops = f_sel / (ms_attn * 1e-3) / 1e12
-    peak_tf = pk["bf16_tflops"]
+    # a kernel timed alone gets the burst peak; one timed inside seconds of
+    # back-to-back steps runs under the power cap and gets the sustained one
+    long_run = tot[0] > 2000.0
+    peak_tf = pk["bf16_tflops_sustained"] if long_run else pk["bf16_tflops"]
+    peak_kind = "bf16 sustained (cuBLAS, seconds under the power cap)" if long_run else "bf16 burst (cuBLAS)"
     idx_bytes, nqb = algorithmic_index_bytes(w, pats)
     idx_gbs = idx_bytes / (ms_build * 1e-3) / 1e9
     traffic = None
@@ -367,7 +371,7 @@ def main():
                    "parallelism": f"independent layer per rank x{world}"},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": tflops / peak_tf, "traffic": traffic,
-                     "kernel": "sparse_attn_kernel<128>", "peak_source": f"{pk_src} bf16 burst (cuBLAS)",
+                     "kernel": "sparse_attn_kernel<128>", "peak_source": f"{pk_src} {peak_kind}",
                      "work": f"F_sel = 4*d*|M| = {f_sel:.4e} FLOP per launch ({pairs} allowed pairs)"},
         "attention": {"ms": ms_attn, "tflops": tflops, "frac_peak": tflops / peak_tf,
                       "density_vs_causal": pairs / causal_pairs},
