@@ -222,6 +222,10 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--N", type=int, default=0, help="override the token count (smaller profiling cases)")
+    ap.add_argument("--shard-heads", action="store_true",
+                    help="strong scaling: the ranks split ONE layer by KV groups (default: one layer per rank)")
+    ap.add_argument("--gather", action="store_true",
+                    help="with --shard-heads: all-gather every rank's O into the full layer output each step")
     args = ap.parse_args()
     rank, world, local = dist_env()
     w = synth.workload(args.workload, **({"N": args.N} if args.N else {}))
@@ -260,8 +264,16 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=dev)
-    Q, K, V, pats = build_workload(w, dev, seed_offset=rank)
-    N, Hq, d = w["N"], w["Hq"], w["d"]
+    if args.shard_heads:
+        # every rank builds the same layer and keeps its KV groups (heads are independent)
+        from dynamic_sparse_attention_build_b200 import shard
+        Qf, Kf, Vf, pf = build_workload(w, dev)
+        Q, K, V, pats = shard.shard_inputs(Qf, Kf, Vf, pf, rank, world)
+        del Qf, Kf, Vf
+    else:
+        Q, K, V, pats = build_workload(w, dev, seed_offset=rank)
+    N, Hq, d = w["N"], Q.shape[0], w["d"]
+    gather = args.shard_heads and args.gather and world > 1
     pats_c = dsa.make_patterns(pats)
     bufs = dsa.build_indices(Q, K, pats_c, w["B"])
     O = torch.empty_like(Q)
@@ -283,6 +295,8 @@ def main():
         if ev is not None:
             ev[1].record(stream)
         dsa.sparse_prefill(Q, K, V, bufs, O=O)
+        if gather:
+            shard.gather_heads(O, w["Hq"], w["Hkv"])
         if ev is not None:
             ev[2].record(stream)
 
@@ -362,13 +376,16 @@ def main():
             traffic = tr.get("dram_bytes_per_launch")
 
     line = {
-        "metric": METRIC, "value": whole_job_tokens_per_s(N, world, ms_step), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC, "value": (N / (ms_step * 1e-3) if args.shard_heads else whole_job_tokens_per_s(N, world, ms_step)),
+        "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "strong" if args.shard_heads else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
                    "patterns": PATTERN_TEXT.get(w["mix"], w["mix"]),
                    "l2": "flushed by a 256 MiB write before every timed step (outside its events)",
-                   "parallelism": f"independent layer per rank x{world}"},
+                   "parallelism": (f"one layer, heads sharded by KV group x{world}"
+                                   + (", O all-gathered each step" if gather else "")
+                                   if args.shard_heads else f"independent layer per rank x{world}")},
         "roofline": {"bound": "tensor", "achieved": tflops, "peak": peak_tf, "unit": "TFLOP/s",
                      "frac": tflops / peak_tf, "traffic": traffic,
                      "kernel": "sparse_attn_kernel<128>", "peak_source": f"{pk_src} {peak_kind}",
@@ -377,7 +394,8 @@ def main():
                       "density_vs_causal": pairs / causal_pairs},
         "index_build": {"ms": ms_build, "algorithmic_bytes": idx_bytes, "gbs": idx_gbs,
                         "frac_hbm": idx_gbs / pk["hbm_gbs"], "hbm_peak_source": pk_src},
-        "e2e": {"value": whole_job_tokens_per_s(N, world, e2e_ms), "unit": "tokens/s",
+        "e2e": {"value": (N / (e2e_ms * 1e-3) if args.shard_heads else whole_job_tokens_per_s(N, world, e2e_ms)),
+                "unit": "tokens/s",
                 "h2d_bytes_per_step": (Q.numel() + K.numel() + V.numel()) * 2,
                 "d2h_bytes_per_step": O.numel() * 2, "ms_per_step": e2e_ms},
         "gpu_launches": kernel_launches_per_step(pats) * args.steps,
