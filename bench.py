@@ -221,6 +221,7 @@ def main():
     ap.add_argument("--workload", type=int, default=2)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--e2e-chunks", type=int, default=8, help="KV-group chunks of the overlapped host path")
     ap.add_argument("--N", type=int, default=0, help="override the token count (smaller profiling cases)")
     ap.add_argument("--shard-heads", action="store_true",
                     help="strong scaling: the ranks split ONE layer by KV groups (default: one layer per rank)")
@@ -327,20 +328,16 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status {st} detail {det}")
 
-    # end to end through the public API with pinned host buffers
+    # end to end through the public API with pinned host buffers: HostPrefill
+    # uploads, computes and downloads KV-group chunks on three streams
     Qh = Q.cpu().pin_memory()
     Kh = K.cpu().pin_memory()
     Vh = V.cpu().pin_memory()
     Oh = torch.empty_like(Qh).pin_memory()
-    Qe, Ke, Ve = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    hp = dsa.HostPrefill(Hq, K.shape[0], N, d, pats, w["B"], chunks=args.e2e_chunks, device=dev)
 
     def e2e_step():
-        Qe.copy_(Qh, non_blocking=True)
-        Ke.copy_(Kh, non_blocking=True)
-        Ve.copy_(Vh, non_blocking=True)
-        dsa.build_indices(Qe, Ke, pats_c, w["B"], bufs=bufs)
-        dsa.sparse_prefill(Qe, Ke, Ve, bufs, O=O)
-        Oh.copy_(O, non_blocking=True)
+        hp.run(Qh, Kh, Vh, Oh)
 
     e2e_step()
     torch.cuda.synchronize()

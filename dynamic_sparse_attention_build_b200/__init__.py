@@ -11,5 +11,5 @@ Two calls, implemented as sm_100a CUDA kernels in ``libdsa.so`` (C ABI in
 Importing the package does not load the library; the first call does, and fails
 loudly if it has not been built (``python -m dynamic_sparse_attention_build_b200.build``).
 """
-from .api import (IndexBuffers, alloc_indices, build_indices, count_pairs, device_status,  # noqa: F401
-                  indices_from_lists, make_patterns, make_problem, sparse_prefill)
+from .api import (HostPrefill, IndexBuffers, alloc_indices, build_indices, count_pairs,  # noqa: F401
+                  device_status, indices_from_lists, make_patterns, make_problem, sparse_prefill)

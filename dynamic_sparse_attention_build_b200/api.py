@@ -233,3 +233,69 @@ def indices_from_lists(heads, N, block, device="cuda") -> IndexBuffers:
                         blk_idx=t(bi), dist_ptr=t(dp), dist=t(di), col_ptr=t(cp), col_idx=t(ci),
                         vert_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device),
                         slash_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device))
+
+
+class HostPrefill:
+    """Prefill of one layer whose Q, K, V and O live in pinned host memory, with
+    the copies overlapped: the layer's KV groups are split into ``chunks``
+    contiguous runs (heads are independent); chunk c's inputs go to the GPU on a
+    copy stream while chunk c - 1 computes and chunk c - 2's output comes back on
+    another, so a step costs about the largest of the three totals instead of
+    their sum.  Device buffers and per-chunk index buffers are allocated once
+    and reused by every ``run``; results equal those of the device-resident
+    calls head for head."""
+
+    def __init__(self, Hq, Hkv, N, d, patterns, block, chunks=4, device="cuda"):
+        from .shard import kv_group_range
+        if Hq % Hkv:
+            raise ValueError("Hq must be a multiple of Hkv")
+        self.G = Hq // Hkv
+        self.block = block
+        self.device = torch.device(device)
+        bf = dict(dtype=torch.bfloat16, device=self.device)
+        self.Q = torch.empty(Hq, N, d, **bf)
+        self.K = torch.empty(Hkv, N, d, **bf)
+        self.V = torch.empty(Hkv, N, d, **bf)
+        self.O = torch.empty(Hq, N, d, **bf)
+        n = max(1, min(chunks, Hkv))
+        self.ranges = [kv_group_range(c, n, Hkv) for c in range(n)]
+        self.pats = [make_patterns(patterns[k0 * self.G:k1 * self.G]) for k0, k1 in self.ranges]
+        # index buffers of every chunk, allocated (and zero-filled on the current
+        # stream) here, before any run
+        self.bufs = [alloc_indices(make_problem(self.Q[k0 * self.G:k1 * self.G], self.K[k0:k1], block=block),
+                                   self.pats[c], self.device) for c, (k0, k1) in enumerate(self.ranges)]
+        self.h2d = torch.cuda.Stream(self.device)
+        self.comp = torch.cuda.Stream(self.device)
+        self.d2h = torch.cuda.Stream(self.device)
+
+    def run(self, Qh, Kh, Vh, Oh):
+        """Q/K/V (pinned host, [heads, N, d] bf16) -> Oh (pinned host).  Asynchronous
+        with respect to the host; the caller's current stream waits for the last
+        output copy, so synchronising it (or an event recorded on it) suffices."""
+        cur = torch.cuda.current_stream(self.device)
+        # everything the caller's stream did before (including the previous run,
+        # which it waits for) happens before this run touches the device buffers
+        for s in (self.h2d, self.comp, self.d2h):
+            s.wait_stream(cur)
+        last = None
+        for c, (k0, k1) in enumerate(self.ranges):
+            q0, q1 = k0 * self.G, k1 * self.G
+            with torch.cuda.stream(self.h2d):
+                self.Q[q0:q1].copy_(Qh[q0:q1], non_blocking=True)
+                self.K[k0:k1].copy_(Kh[k0:k1], non_blocking=True)
+                self.V[k0:k1].copy_(Vh[k0:k1], non_blocking=True)
+                ev_in = torch.cuda.Event()
+                ev_in.record(self.h2d)
+            self.comp.wait_event(ev_in)
+            q, k, v, o = self.Q[q0:q1], self.K[k0:k1], self.V[k0:k1], self.O[q0:q1]
+            self.bufs[c] = build_indices(q, k, self.pats[c], self.block, bufs=self.bufs[c], stream=self.comp)
+            sparse_prefill(q, k, v, self.bufs[c], O=o, stream=self.comp)
+            ev_out = torch.cuda.Event()
+            ev_out.record(self.comp)
+            self.d2h.wait_event(ev_out)
+            with torch.cuda.stream(self.d2h):
+                Oh[q0:q1].copy_(o, non_blocking=True)
+                last = torch.cuda.Event()
+                last.record(self.d2h)
+        cur.wait_event(last)
+        return Oh
