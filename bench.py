@@ -119,6 +119,18 @@ def reduce_max_over_ranks(values, device="cpu"):
     return t.tolist()
 
 
+def kernel_source_hash(path):
+    """16 hex digits of the SHA-256 of a CUDA source with its // comments and
+    blank lines removed: profiler counters stay tied to the code, not its prose."""
+    import hashlib
+    lines = []
+    for ln in open(path, encoding="utf-8").read().splitlines():
+        code = ln.split("//", 1)[0].rstrip()
+        if code:
+            lines.append(code)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
+
+
 def whole_job_tokens_per_s(N, world, ms_per_step):
     """Every rank processes its own N-token layer per step (weak scaling)."""
     return N * world / (ms_per_step * 1e-3)
@@ -365,10 +377,9 @@ def main():
     if os.path.exists(tp):
         # DRAM bytes per launch from an ncu capture; only valid for the kernel
         # source it was taken on and for this workload
-        import hashlib
         tr = json.load(open(tp))
         src = os.path.join(ROOT, "dynamic_sparse_attention_build_b200", "csrc", "dsa_attn.cu")
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        sha = kernel_source_hash(src)
         if tr.get("workload") == w["name"] and tr.get("kernel_source_sha256_16") == sha and w["N"] == 32768:
             traffic = tr.get("dram_bytes_per_launch")
 

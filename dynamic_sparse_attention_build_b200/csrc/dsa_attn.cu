@@ -17,13 +17,16 @@
 //     halves that listed it (the other half masks it out);
 //   * column lists are gathered into dense 64-key tiles (gather-and-densify); a
 //     column inside a block the half already keeps is masked out;
-//   * warps 0,2,3 build the bitmaps, issue TMA loads (SWIZZLE_128B boxes of
-//     64 x 64) into two K and two V buffers and gather column rows; warp 1 issues
-//     tcgen05.mma; warps 4-7 run the online softmax (one thread per row) and the
-//     epilogue.  The loaders read the next item's lists and load its Q while the
-//     other warps finish the current item, so an item's set-up is off the
-//     critical path; tile and item counters run across items, so every barrier
-//     keeps its phase from one item to the next;
+//   * warps 2-3 (decoders) fetch items, turn an item's lists into bitmap set
+//     (item & 1) up to one item ahead, publish it, and gather its column rows;
+//     warp 0 (one thread) loads each item's Q and issues the TMA loads
+//     (SWIZZLE_128B boxes of 64 x 64) of its key units into two K and two V
+//     buffers; tiles are issued strictly in order (units, then columns, item by
+//     item), which keeps every empty-buffer parity wait unambiguous; warp 1 (one
+//     thread) issues each tile's tcgen05.mma from one asm block; warps 4-7 run the
+//     online softmax (one thread per row) and the epilogue.  Tile and item
+//     counters run across items, so every barrier keeps its phase from one item
+//     to the next;
 //   * TMEM (256 columns per CTA): O at [0, 128), two S buffers of 64 columns at
 //     128 and 192.  S(t+1) = Q K(t+1)^T is computed while the softmax works on
 //     S(t); the softmax writes P(t) as bf16 pairs over the first 32 columns of its

@@ -15,6 +15,9 @@
 //                 MoBA may first run a causal depthwise conv with SiLU and a
 //                 residual over the keys ("2. キーに対する畳み込み適用").
 // Every list is produced by count -> scan -> fill into caller-owned CSR arrays.
+// Every kernel is launched with programmatic dependent launch (pdl_prologue in
+// dsa_common.cuh), and the build issues no memsets: the count kernels clear the
+// pointer entries no other kernel writes, VS pass 1 clears the slash sums.
 #include <math.h>
 #include <string.h>
 
