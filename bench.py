@@ -235,13 +235,22 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-chunks", type=int, default=8, help="KV-group chunks of the overlapped host path")
     ap.add_argument("--N", type=int, default=0, help="override the token count (smaller profiling cases)")
+    ap.add_argument("--B", type=int, default=0, help="override the block size (the MoBA workload's B sweep)")
+    ap.add_argument("--conv", type=int, default=-1, help="override the MoBA key-conv width (0 = off)")
     ap.add_argument("--shard-heads", action="store_true",
                     help="strong scaling: the ranks split ONE layer by KV groups (default: one layer per rank)")
     ap.add_argument("--gather", action="store_true",
                     help="with --shard-heads: all-gather every rank's O into the full layer output each step")
     args = ap.parse_args()
     rank, world, local = dist_env()
-    w = synth.workload(args.workload, **({"N": args.N} if args.N else {}))
+    over = {}
+    if args.N:
+        over["N"] = args.N
+    if args.B:
+        over["B"] = args.B
+    if args.conv >= 0:
+        over["conv_width"] = args.conv
+    w = synth.workload(args.workload, **over)
 
     if args.impl == "reference":
         # the oracle, as it stands, on the host cores; rank 0 only
@@ -389,6 +398,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.shard_heads else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
+                   "key_conv_width": int(w.get("conv_width", 0) or 0),
                    "patterns": PATTERN_TEXT.get(w["mix"], w["mix"]),
                    "l2": "flushed by a 256 MiB write before every timed step (outside its events)",
                    "parallelism": (f"one layer, heads sharded by KV group x{world}"

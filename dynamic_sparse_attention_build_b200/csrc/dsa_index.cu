@@ -268,12 +268,67 @@ __global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int
   blk_ptr[1 + h * L.nqb + qb] = cnt;
 }
 
+// Causal depthwise key conv (width W, SiLU, residual) summed over a contiguous
+// run of rows [r0, r1) for this thread's 8 channels: weights in registers, the
+// last W rows in a register window, one 16-byte load per row (four in flight).
+template <int W>
+__device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts, int c0, int r0, int r1,
+                                              const float* cw, const float* cb, float* acc) {
+  float wt[W][8], bias[8], win[W][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    bias[i] = cb[c0 + i];
+#pragma unroll
+    for (int t = 0; t < W; ++t) wt[t][i] = cw[(c0 + i) * W + t];
+  }
+  // before row r is shifted in, win[t] = k[r - 1 - t] (t < W - 1); after the
+  // shift win[t] = k[r - t].  Rows before 0 are zero (causal, zero padded).
+#pragma unroll
+  for (int t = 0; t < W - 1; ++t) {
+    const int rr = r0 - 1 - t;
+    uint4 raw = make_uint4(0, 0, 0, 0);
+    if (rr >= 0 && r0 < r1) raw = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)rr * ts + c0));
+    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) win[t][i] = __bfloat162float(e[i]);
+  }
+  for (int r = r0; r < r1; r += 4) {
+    uint4 raw[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      raw[u] = (r + u < r1) ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r + u) * ts + c0))
+                            : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (r + u >= r1) break;
+#pragma unroll
+      for (int t = W - 1; t > 0; --t) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) win[t][i] = win[t - 1][i];
+      }
+      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) win[0][i] = __bfloat162float(e[i]);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float c = bias[i];
+#pragma unroll
+        for (int t = 0; t < W; ++t) c = fmaf(wt[t][i], win[t][i], c);
+        acc[i] += win[0][i] + __fdividef(c, 1.f + __expf(-c));
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // key mean pooling (+ optional causal depthwise key conv with SiLU and residual)
 // ---------------------------------------------------------------------------
 // grid: (nqb, Hkv); KV heads that no block head reads are skipped.  Queries are
-// pooled inside k_block_select.
-template <int D>
+// pooled inside k_block_select.  CW = 0: plain mean, for the KV heads without a
+// key conv; CW = W in 1..8: the conv of width W, for the KV heads with that
+// width (one launch per width present, so each instantiation holds exactly the
+// registers its width needs).
+template <int D, int CW>
 __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct, Layout L,
                                               const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws) {
   pdl_prologue();
@@ -282,14 +337,11 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct
   __shared__ float part[RG][D];
   const int b = blockIdx.x;
   const int kvh = blockIdx.y;
-  if (!ct.need[kvh]) return;
+  if (!ct.need[kvh] || ct.width[kvh] != CW) return;
   const __nv_bfloat16* X = K + kvh * k_hs;
   const int64_t ts = k_ts;
   // the pooled row as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
   __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * 2 * D;
-  const int W = ct.width[kvh];
-  const float* cw = ct.w[kvh];
-  const float* cb = ct.b[kvh];
   const int rg = threadIdx.x / TPR;
   const int c0 = (threadIdx.x % TPR) * 8;
   const int r_beg = b * L.B;
@@ -297,7 +349,7 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  if (W == 0) {
+  if constexpr (CW == 0) {
     // plain mean: eight independent row loads in flight per thread
     int r = r_beg + rg;
     for (; r + 7 * RG < r_end; r += 8 * RG) {
@@ -318,25 +370,11 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct
       for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
     }
   } else {
-    for (int r = r_beg + rg; r < r_end; r += RG) {
-      const uint4 raw = *reinterpret_cast<const uint4*>(X + (int64_t)r * ts + c0);
-      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
-      float x[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) x[i] = __bfloat162float(e[i]);
-      float conv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) conv[i] = cb[c0 + i];
-      for (int t = 0; t < W; ++t) {
-        if (r - t < 0) break;
-        const uint4 rr = (t == 0) ? raw : *reinterpret_cast<const uint4*>(X + (int64_t)(r - t) * ts + c0);
-        const __nv_bfloat16* ee = reinterpret_cast<const __nv_bfloat16*>(&rr);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) conv[i] = fmaf(cw[(c0 + i) * W + t], __bfloat162float(ee[i]), conv[i]);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] += x[i] + conv[i] / (1.f + expf(-conv[i]));
-    }
+    // each row group takes a contiguous run of the block's rows (the conv window
+    // slides along it)
+    const int run = (r_end - r_beg + RG - 1) / RG;
+    const int r0 = min(r_end, r_beg + rg * run), r1 = min(r_end, r0 + run);
+    conv_rows_sum<CW>(X, ts, c0, r0, r1, ct.w[kvh], ct.b[kvh], acc);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) part[rg][c0 + i] = acc[i];
@@ -349,6 +387,27 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct
     out[threadIdx.x] = hi;
     out[D + threadIdx.x] = __float2bfloat16_rn(x - __bfloat162float(hi));
   }
+}
+
+// the plain pooling for the KV heads without a conv and one launch per conv width present
+template <int D>
+cudaError_t launch_pool(const ConvTab& ct, const Layout& L, const __nv_bfloat16* k, int64_t k_hs, int64_t k_ts,
+                        uint8_t* ws, cudaStream_t st) {
+  bool has[9] = {};
+  for (int h = 0; h < L.Hkv; ++h)
+    if (ct.need[h]) has[ct.width[h] < 0 || ct.width[h] > 8 ? 0 : ct.width[h]] = true;
+  const dim3 grid(L.nqb, L.Hkv), block(256);
+  cudaError_t e = cudaSuccess;
+  if (has[0]) e = launch_pdl(k_pool<D, 0>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[1]) e = launch_pdl(k_pool<D, 1>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[2]) e = launch_pdl(k_pool<D, 2>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[3]) e = launch_pdl(k_pool<D, 3>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[4]) e = launch_pdl(k_pool<D, 4>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[5]) e = launch_pdl(k_pool<D, 5>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[6]) e = launch_pdl(k_pool<D, 6>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[7]) e = launch_pdl(k_pool<D, 7>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (e == cudaSuccess && has[8]) e = launch_pdl(k_pool<D, 8>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  return e;
 }
 
 // ---------------------------------------------------------------------------
@@ -1454,16 +1513,14 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
   const auto* k = static_cast<const __nv_bfloat16*>(K);
   if (L.nbh > 0) {
     if (p.d == 128) {
-      DSA_CK(launch_pdl(k_pool<128>, dim3(L.nqb, p.Hkv), dim3(256), 0, st, ct, L, k, p.k_head_stride,
-                        p.k_token_stride, ws));
+      DSA_CK(launch_pool<128>(ct, L, k, p.k_head_stride, p.k_token_stride, ws, st));
       const int ri = sel_blocks_per_cta(p.block);
       const size_t sel_smem = sel_smem_bytes(128, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
       DSA_CK(launch_pdl(k_block_select<128>, dim3(ceil_div(L.nqb, ri), L.nbh), dim3(SEL_NT), sel_smem, st, ht, L,
                         q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri));
     } else {
-      DSA_CK(launch_pdl(k_pool<64>, dim3(L.nqb, p.Hkv), dim3(256), 0, st, ct, L, k, p.k_head_stride,
-                        p.k_token_stride, ws));
+      DSA_CK(launch_pool<64>(ct, L, k, p.k_head_stride, p.k_token_stride, ws, st));
       const int ri = sel_blocks_per_cta(p.block);
       const size_t sel_smem = sel_smem_bytes(64, L.nkw);
       DSA_CK(cudaFuncSetAttribute(k_block_select<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sel_smem));
