@@ -61,7 +61,7 @@ struct ConvTab {
 
 struct Layout {
   int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_nchunks, vs_lmax;
-  int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, total;
+  int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, off_spart, total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
@@ -775,11 +775,6 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   }
   float* part = reinterpret_cast<float*>(ws + L.off_part);
   float* stat = reinterpret_cast<float*>(ws + L.off_stat);
-  if (PASS == 1) {
-    // pass 2 adds its diagonal sums into s with atomics: clear this chunk of it
-    float* sout = reinterpret_cast<float*>(ws + L.off_s) + (int64_t)vslot * L.N;
-    for (int j = j0 + tid; j < j1; j += 256) sout[j] = 0.f;
-  }
   if (PASS == 2) {
     for (int i = tid; i < VS_CHUNK + LP; i += 256) sbuf[i] = 0.f;
     for (int i = tid; i < VS_CHUNK; i += 256) vbuf[i] = 0.f;
@@ -926,14 +921,39 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   } else {
     __syncthreads();
     float* vout = reinterpret_cast<float*>(ws + L.off_v) + (int64_t)vslot * L.N;
-    float* sout = reinterpret_cast<float*>(ws + L.off_s) + (int64_t)vslot * L.N;
     for (int j = j0 + tid; j < j1; j += 256) vout[j] = vbuf[j - j0];
-    for (int t = tid; t < VS_CHUNK + LP; t += 256) {
-      const int o = obase + t;
-      const float val = sbuf[t];
-      if (o >= 0 && o < L.N && val != 0.f) atomicAdd(&sout[o], val);
+    // this chunk's window of slash sums (offset o at index o - obase); the
+    // windows of neighbouring chunks overlap and are added in a fixed order by
+    // k_vs_slash_combine, so s is the same bit for bit on every run
+    float* win = reinterpret_cast<float*>(ws + L.off_spart) +
+                 ((int64_t)vslot * L.vs_nchunks + chunk) * (VS_CHUNK + VS_MAXL);
+    for (int t = tid; t < VS_CHUNK + VS_MAXL; t += 256) win[t] = (t < VS_CHUNK + LP) ? sbuf[t] : 0.f;
+  }
+}
+
+// s[o] of one VS head from the windows of the (at most two) key chunks whose
+// keys meet offset o from the estimate rows, in ascending chunk order.
+__global__ void __launch_bounds__(256) k_vs_slash_combine(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws) {
+  pdl_prologue();
+  const int vslot = blockIdx.y;
+  const int o = blockIdx.x * blockDim.x + threadIdx.x;
+  if (o >= L.N) return;
+  const int h = ht.vhead[vslot];
+  const int Lq = min(ht.last_q[h], L.N);
+  const int i0 = L.N - Lq;
+  const float* wins =
+      reinterpret_cast<const float*>(ws + L.off_spart) + (int64_t)vslot * L.vs_nchunks * (VS_CHUNK + VS_MAXL);
+  // chunk c holds the offsets (i0 - (c + 1) VS_CHUNK, i0 + Lq - 1 - c VS_CHUNK]
+  const int hi = i0 + Lq - 1 - o;  // the largest key an estimate row meets at offset o
+  float acc = 0.f;
+  if (hi >= 0) {
+    const int c_hi = min(L.vs_nchunks - 1, hi / VS_CHUNK);
+    for (int c = max(0, c_hi - 1); c <= c_hi; ++c) {
+      const int t = o - (i0 - (c * VS_CHUNK + VS_CHUNK - 1));
+      if (t >= 0 && t < VS_CHUNK + VS_MAXL) acc += wins[(int64_t)c * (VS_CHUNK + VS_MAXL) + t];
     }
   }
+  reinterpret_cast<float*>(ws + L.off_s)[(int64_t)vslot * L.N + o] = acc;
 }
 
 // merge the per-chunk (max, sum) partials (log2 units) into the row softmax statistics
@@ -1427,6 +1447,8 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->off_stat = off; off = align256(off + (int64_t)L->nvs * VS_MAXL * 2 * 4);
   L->off_dtmp = off; off = align256(off + (int64_t)L->nvs * nqb * 4);
   L->off_dbits = off; off = align256(off + (int64_t)L->nvs * L->nkw * 4);
+  // per-chunk windows of the slash sums (VS_CHUNK + VS_MAXL offsets each)
+  L->off_spart = off; off = align256(off + (int64_t)L->nvs * L->vs_nchunks * (VS_CHUNK + VS_MAXL) * 4);
   L->total = std::max<int64_t>(off, 256);
   if (sz) {
     sz->nqb = nqb;
@@ -1462,6 +1484,7 @@ dsa_status launch_vs(const HeadTab& ht, const Layout& L, const void* Q, int64_t 
     launch_pdl(k_vs<D, R, 1>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
     launch_pdl(k_vs_rowstats, dim3(L.nvs), dim3(128), 0, st, ht, L, ws);                                    \
     launch_pdl(k_vs<D, R, 2>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
+    launch_pdl(k_vs_slash_combine, dim3(ceil_div(L.N, 256), L.nvs), dim3(256), 0, st, ht, L, ws);           \
   } while (0)
   switch (RT) {
     case 1: DSA_VS_LAUNCH(1); break;

@@ -140,3 +140,20 @@ def test_threshold_topics(dsa):
     lists = bufs.host_lists()[0]["blocks"]
     hits = sum(int(all(topic[J] == topic[I] for J in lists[I] if J not in (0, I))) for I in range(len(lists)))
     assert hits >= 0.9 * len(lists)
+
+
+def test_index_build_is_deterministic(dsa):
+    """Two builds of the same layer give the same lists bit for bit: the VS sums
+    use no floating-point atomics (each key chunk writes its own window of slash
+    sums; windows that overlap are added in a fixed order)."""
+    w = synth.workload(2, N=6000, Hq=8, Hkv=2)
+    Q, K, V, _ = synth.make_inputs(w)
+    pats = synth.head_patterns(w)
+    Qd, Kd = Q.cuda(), K.cuda()
+    a = dsa.build_indices(Qd, Kd, pats, w["B"])
+    b = dsa.build_indices(Qd, Kd, pats, w["B"])
+    torch.cuda.synchronize()
+    for name in ("head_info", "blk_ptr", "blk_idx", "dist_ptr", "dist", "col_ptr", "col_idx", "vert_idx",
+                 "slash_idx"):
+        assert torch.equal(getattr(a, name), getattr(b, name)), name
+    assert any(p["kind"] == "vs" for p in pats)
