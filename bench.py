@@ -154,7 +154,7 @@ def kernel_launches_per_step(pats):
     if any(k in ("block_topk", "block_threshold", "moba") for k in kinds):
         n += 2  # pool, block score/select
     if "vs" in kinds:
-        n += 8  # VS pass 1, row stats, pass 2, top-k, distances, column count, distance fill, column fill
+        n += 9  # VS pass 1, row stats, pass 2, slash combine, top-k, distances, column count, distance fill, column fill
     return n + 1  # attention
 
 
