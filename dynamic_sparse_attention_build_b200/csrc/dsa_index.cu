@@ -76,19 +76,28 @@ __device__ __forceinline__ uint32_t fkey(float f) {
 // CTA-wide helpers (blockDim.x threads, multiple of 32, <= 1024)
 // ---------------------------------------------------------------------------
 // Exact top-k of vals[0..n) (ties to the lower index), n > k >= 1.  Finds the
-// k-th largest key T by 4 radix passes of 8 bits, and how many keys equal to T
-// to take.  hist: shared int[256 * nwarps]; red: shared int[64].
+// k-th largest key T by three radix passes over the 32-bit key, most
+// significant digit first (12, 12 and 8 bits), and how many keys equal to T to
+// take.  One 4096-bin histogram for the whole CTA: the first digit is the sign,
+// the exponent and the top mantissa bits, so sums of similar magnitude still
+// spread over many bins and few lanes of a warp add to the same bin at once
+// (an 8-bit first digit is the exponent alone: ~20 lanes of every warp hit one
+// bin on the VS sums).  blockDim.x: a power of two, 32..1024.
+// hist: shared int[RADIX_BINS]; red: shared int[>= 2 + blockDim.x / 32].
 constexpr int RB = 8;  // keys loaded per thread before use in the CTA-wide select
+constexpr int RADIX_BINS = 4096;
 
 template <typename Loader>
 __device__ void radix_kth(const Loader& load, int n, int k, int* hist, int* red, uint32_t* T_out,
                           int* take_eq_out) {
-  const int nw = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bpt = RADIX_BINS / blockDim.x;  // bins per thread in the digit search
   uint32_t prefix = 0, mask = 0;
-  int need = k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
-    for (int i = threadIdx.x; i < 256 * nw; i += blockDim.x) hist[i] = 0;
+  int need = k;  // keys still to take among those matching prefix (>= 1)
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
+    for (int i = threadIdx.x; i < RADIX_BINS; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     // RB independent loads in flight per thread before their keys are counted
     for (int i0 = 0; i0 < n; i0 += RB * blockDim.x) {
@@ -101,55 +110,41 @@ __device__ void radix_kth(const Loader& load, int n, int k, int* hist, int* red,
 #pragma unroll
       for (int q = 0; q < RB; ++q) {
         const int i = i0 + q * blockDim.x + threadIdx.x;
-        if (i < n && (key[q] & mask) == prefix) atomicAdd(&hist[warp * 256 + ((key[q] >> shift) & 255u)], 1);
+        if (i < n && (key[q] & mask) == prefix) atomicAdd(&hist[(key[q] >> shift) & dmask], 1);
       }
     }
     __syncthreads();
-    for (int b = threadIdx.x; b < 256; b += blockDim.x) {
-      int s = 0;
-      for (int w = 0; w < nw; ++w) s += hist[w * 256 + b];
-      hist[b] = s;
+    // thread t takes bins RADIX_BINS-1-t*bpt downwards (bins above the digit
+    // width are empty); a CTA-wide exclusive scan of the per-thread sums is the
+    // count of keys in higher bins; the one thread whose run crosses `need`
+    // holds the digit
+    const int top = RADIX_BINS - 1 - threadIdx.x * bpt;
+    int tot = 0;
+    for (int q = 0; q < bpt; ++q) tot += hist[top - q];
+    int incl = tot;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    if (lane == 31) red[2 + warp] = incl;
     __syncthreads();
-    if (warp == 0) {
-      // the digit whose bin takes the count from the top past `need`: lane l
-      // holds bins 255 - 8l .. 248 - 8l, a warp scan gives the count above them
-      int c[8], tot = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        c[q] = hist[255 - (lane * 8 + q)];
-        tot += c[q];
-      }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int above = incl - tot, digit = -1, ab = 0;
-#pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        if (digit < 0) {
-          if (above + c[q] >= need) {
-            digit = 255 - (lane * 8 + q);
-            ab = above;
-          } else {
-            above += c[q];
-          }
+    int above = incl - tot;
+    for (int w = 0; w < warp; ++w) above += red[2 + w];
+    if (above < need && above + tot >= need) {
+      for (int q = 0; q < bpt; ++q) {
+        const int c = hist[top - q];
+        if (above + c >= need) {
+          red[0] = top - q;
+          red[1] = above;
+          break;
         }
-      }
-      const unsigned found = __ballot_sync(0xffffffffu, digit >= 0);
-      const int src = __ffs(found) - 1;  // the candidates always hold `need` keys
-      digit = __shfl_sync(0xffffffffu, digit, src);
-      ab = __shfl_sync(0xffffffffu, ab, src);
-      if (lane == 0) {
-        red[0] = digit;
-        red[1] = ab;
+        above += c;
       }
     }
     __syncthreads();
     prefix |= (uint32_t)red[0] << shift;
-    mask |= 255u << shift;
+    mask |= dmask << shift;
     need -= red[1];
     __syncthreads();
   }
@@ -983,7 +978,7 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
                                                   int32_t* vert_idx, int vert_stride, int32_t* slash_idx,
                                                   int slash_stride) {
   pdl_prologue();
-  __shared__ int hist[256 * 32];
+  __shared__ int hist[RADIX_BINS];
   __shared__ int red[80];
   const int vslot = blockIdx.x;
   const int which = blockIdx.y;
