@@ -31,9 +31,16 @@ namespace {
 
 constexpr int MAXH = 256;     // heads per layer this build accepts
 constexpr int MAXKV = 256;
-constexpr int VS_CHUNK = 1024;  // keys per CTA of the VS estimate
+// keys per CTA of the VS estimate: one of VS_CHUNKS, chosen per problem by
+// choose_vs_chunk (all multiples of VS_SUB and >= VS_MAXL)
+constexpr int VS_CHUNKS[3] = {1024, 768, 512};
+constexpr int VS_CHUNK_MAX = 1024;
 constexpr int VS_SUB = 128;     // keys per sub-tile
 constexpr int VS_MAXL = 128;    // last_q limit
+static_assert(VS_CHUNKS[0] == VS_CHUNK_MAX && VS_CHUNKS[0] % VS_SUB == 0 && VS_CHUNKS[1] % VS_SUB == 0 &&
+                  VS_CHUNKS[2] % VS_SUB == 0,
+              "chunks are whole sub-tiles");
+static_assert(VS_CHUNKS[2] >= VS_MAXL, "the keys an offset meets from the estimate rows span at most two chunks");
 
 struct HeadTab {
   int kind[MAXH];
@@ -60,7 +67,7 @@ struct ConvTab {
 };
 
 struct Layout {
-  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_nchunks, vs_lmax;
+  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_chunk, vs_nchunks, vs_lmax;
   int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, off_spart, total;
 };
 
@@ -727,9 +734,10 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   constexpr int PP = VS_SUB + 4;         // padded fp32 row of the P tile
   __nv_bfloat16* ks = qs + LP * DP;                                      // [VS_SUB][DP]
   float* ps = reinterpret_cast<float*>(ks + VS_SUB * DP);                // [LP][PP] (pass 2)
-  float* sbuf = ps + LP * PP;                                            // [VS_CHUNK + LP]
-  float* vbuf = sbuf + VS_CHUNK + LP;                                    // [VS_CHUNK]
-  float* rowm = vbuf + VS_CHUNK;                                         // [LP]
+  const int CHK = L.vs_chunk;
+  float* sbuf = ps + LP * PP;                                            // [CHK + LP]
+  float* vbuf = sbuf + CHK + LP;                                         // [CHK]
+  float* rowm = vbuf + CHK;                                              // [LP]
   float* rowl = rowm + LP;                                               // [LP]
   float* wpart = rowl + LP;                                              // [8][LP][2] (pass 1)
 
@@ -740,8 +748,8 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   const int kvh = h / L.G;
   const int Lq = min(ht.last_q[h], L.N);
   const int i0 = L.N - Lq;  // first estimate row
-  const int j0 = chunk * VS_CHUNK;
-  const int j1 = min(L.N, j0 + VS_CHUNK);
+  const int j0 = chunk * CHK;
+  const int j1 = min(L.N, j0 + CHK);
   const float sc = 1.4426950408889634f * rsqrtf((float)D);  // tau * log2(e)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int rt = warp % RT, kg = warp / RT;
@@ -771,8 +779,8 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
   float* part = reinterpret_cast<float*>(ws + L.off_part);
   float* stat = reinterpret_cast<float*>(ws + L.off_stat);
   if (PASS == 2) {
-    for (int i = tid; i < VS_CHUNK + LP; i += 256) sbuf[i] = 0.f;
-    for (int i = tid; i < VS_CHUNK; i += 256) vbuf[i] = 0.f;
+    for (int i = tid; i < CHK + LP; i += 256) sbuf[i] = 0.f;
+    for (int i = tid; i < CHK; i += 256) vbuf[i] = 0.f;
     for (int r = tid; r < LP; r += 256) {
       rowm[r] = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 0] : 0.f;
       const float l = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 1] : 1.f;
@@ -802,7 +810,7 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
     rl[1] = rowl[rA + 8];
   }
   float run_m[2] = {-INFINITY, -INFINITY}, run_l[2] = {0.f, 0.f};
-  const int obase = i0 - (j0 + VS_CHUNK - 1);  // sbuf index of offset o is o - obase
+  const int obase = i0 - (j0 + CHK - 1);  // sbuf index of offset o is o - obase
   const int nsub = (j1 - j0 + VS_SUB - 1) / VS_SUB;
   for (int si = 0; si < nsub; ++si) {
     const int sub = j0 + si * VS_SUB;
@@ -921,8 +929,8 @@ __global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, 
     // windows of neighbouring chunks overlap and are added in a fixed order by
     // k_vs_slash_combine, so s is the same bit for bit on every run
     float* win = reinterpret_cast<float*>(ws + L.off_spart) +
-                 ((int64_t)vslot * L.vs_nchunks + chunk) * (VS_CHUNK + VS_MAXL);
-    for (int t = tid; t < VS_CHUNK + VS_MAXL; t += 256) win[t] = (t < VS_CHUNK + LP) ? sbuf[t] : 0.f;
+                 ((int64_t)vslot * L.vs_nchunks + chunk) * (CHK + VS_MAXL);
+    for (int t = tid; t < CHK + VS_MAXL; t += 256) win[t] = (t < CHK + LP) ? sbuf[t] : 0.f;
   }
 }
 
@@ -937,15 +945,16 @@ __global__ void __launch_bounds__(256) k_vs_slash_combine(const __grid_constant_
   const int Lq = min(ht.last_q[h], L.N);
   const int i0 = L.N - Lq;
   const float* wins =
-      reinterpret_cast<const float*>(ws + L.off_spart) + (int64_t)vslot * L.vs_nchunks * (VS_CHUNK + VS_MAXL);
-  // chunk c holds the offsets (i0 - (c + 1) VS_CHUNK, i0 + Lq - 1 - c VS_CHUNK]
+      reinterpret_cast<const float*>(ws + L.off_spart) + (int64_t)vslot * L.vs_nchunks * (L.vs_chunk + VS_MAXL);
+  // chunk c holds the offsets (i0 - (c + 1) C, i0 + Lq - 1 - c C], C = L.vs_chunk
   const int hi = i0 + Lq - 1 - o;  // the largest key an estimate row meets at offset o
   float acc = 0.f;
   if (hi >= 0) {
-    const int c_hi = min(L.vs_nchunks - 1, hi / VS_CHUNK);
+    const int C = L.vs_chunk;
+    const int c_hi = min(L.vs_nchunks - 1, hi / C);
     for (int c = max(0, c_hi - 1); c <= c_hi; ++c) {
-      const int t = o - (i0 - (c * VS_CHUNK + VS_CHUNK - 1));
-      if (t >= 0 && t < VS_CHUNK + VS_MAXL) acc += wins[(int64_t)c * (VS_CHUNK + VS_MAXL) + t];
+      const int t = o - (i0 - (c * C + C - 1));
+      if (t >= 0 && t < C + VS_MAXL) acc += wins[(int64_t)c * (C + VS_MAXL) + t];
     }
   }
   reinterpret_cast<float*>(ws + L.off_s)[(int64_t)vslot * L.N + o] = acc;
@@ -1347,6 +1356,21 @@ int vs_rows_pad(int lq) {
   return rt;
 }
 
+// Key chunk of the VS estimate.  Its grid is one CTA per (VS head, chunk), two
+// resident per SM.  When 1024-key chunks leave SMs idle (fewer CTAs than
+// slots), the smallest chunk whose grid still fits in one wave is used: more
+// CTAs, each with less to do (4K tokens, one VS head: 0.070 -> 0.057 ms of index
+// build).  From one wave up 1024 stays: per-CTA costs (Q rows, statistics, the
+// window write) outweigh the shorter tail (32K tokens, 20 VS heads, 768-key
+// chunks: 0.340 -> 0.362 ms).
+int choose_vs_chunk(int nvs, int N, int sms) {
+  const int64_t slots = 2 * (int64_t)std::max(sms, 1);
+  if ((int64_t)nvs * ceil_div(N, VS_CHUNK_MAX) >= slots) return VS_CHUNK_MAX;
+  for (int i = 2; i >= 1; --i)
+    if ((int64_t)nvs * ceil_div(N, VS_CHUNKS[i]) <= slots) return VS_CHUNKS[i];
+  return VS_CHUNK_MAX;
+}
+
 dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L, HeadTab* ht, ConvTab* ct,
                        dsa_sizes* sz) {
   if (p.Hq > MAXH || p.Hkv > MAXKV) return DSA_ERR_UNSUPPORTED;
@@ -1361,7 +1385,8 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->nbh = 0;
   L->nvs = 0;
   L->vs_lmax = 0;
-  L->vs_nchunks = ceil_div(p.N, VS_CHUNK);
+  L->vs_chunk = VS_CHUNK_MAX;  // launch_build_indices may choose a smaller one
+  L->vs_nchunks = ceil_div(p.N, VS_CHUNK_MAX);
   if (ht) memset(ht, 0, sizeof(HeadTab));
   if (ct) memset(ct, 0, sizeof(ConvTab));
   int64_t blk = 0, dcap = 0, ccap = 0;
@@ -1438,12 +1463,18 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->off_sel = off;  off = align256(off + (int64_t)L->nbh * nqb * L->nkw * 4);
   L->off_v = off;    off = align256(off + (int64_t)L->nvs * N * 4);
   L->off_s = off;    off = align256(off + (int64_t)L->nvs * N * 4);
-  L->off_part = off; off = align256(off + (int64_t)L->nvs * L->vs_nchunks * VS_MAXL * 2 * 4);
+  // the per-chunk regions are sized for the candidate chunk that needs the most
+  int64_t vs_parts = 0, vs_wins = 0;
+  for (int c : VS_CHUNKS) {
+    vs_parts = std::max<int64_t>(vs_parts, ceil_div(N, c));
+    vs_wins = std::max<int64_t>(vs_wins, (int64_t)ceil_div(N, c) * (c + VS_MAXL));
+  }
+  L->off_part = off; off = align256(off + (int64_t)L->nvs * vs_parts * VS_MAXL * 2 * 4);
   L->off_stat = off; off = align256(off + (int64_t)L->nvs * VS_MAXL * 2 * 4);
   L->off_dtmp = off; off = align256(off + (int64_t)L->nvs * nqb * 4);
   L->off_dbits = off; off = align256(off + (int64_t)L->nvs * L->nkw * 4);
-  // per-chunk windows of the slash sums (VS_CHUNK + VS_MAXL offsets each)
-  L->off_spart = off; off = align256(off + (int64_t)L->nvs * L->vs_nchunks * (VS_CHUNK + VS_MAXL) * 4);
+  // per-chunk windows of the slash sums (chunk + VS_MAXL offsets each)
+  L->off_spart = off; off = align256(off + (int64_t)L->nvs * vs_wins * 4);
   L->total = std::max<int64_t>(off, 256);
   if (sz) {
     sz->nqb = nqb;
@@ -1468,7 +1499,7 @@ dsa_status launch_vs(const HeadTab& ht, const Layout& L, const void* Q, int64_t 
   const int RT = L.vs_lmax / 16;
   const int LP = L.vs_lmax;
   const size_t smem = (size_t)(LP + VS_SUB) * (D + 8) * 2 + (size_t)LP * (VS_SUB + 4) * 4 +
-                      (size_t)(VS_CHUNK + LP + VS_CHUNK + 2 * LP + 16 * LP) * 4;
+                      (size_t)(L.vs_chunk + LP + L.vs_chunk + 2 * LP + 16 * LP) * 4;
   const dim3 grid(L.vs_nchunks * L.nvs);
   const auto* q = static_cast<const __nv_bfloat16*>(Q);
   const auto* k = static_cast<const __nv_bfloat16*>(K);
@@ -1517,6 +1548,14 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
   uint8_t* ws = static_cast<uint8_t*>(ws_v);
   const int nrows = p.Hq * L.nqb + 1;
   cudaError_t e;
+  if (L.nvs > 0) {
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    L.vs_chunk = choose_vs_chunk(L.nvs, p.N, sms);
+    L.vs_nchunks = ceil_div(p.N, L.vs_chunk);
+  }
 #define DSA_CK(x)                          \
   do {                                     \
     e = (x);                               \
