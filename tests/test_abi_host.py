@@ -123,6 +123,25 @@ def test_capacities_are_exact_or_bounds(B):
     assert sz.workspace_bytes > 0 and sz.workspace_bytes % 256 == 0
 
 
+@pytest.mark.parametrize("N", [129, 1000, 4096, 32768, 100000])
+def test_vs_workspace_covers_every_key_chunk(B, N):
+    # The VS estimate's key chunk (1024, 768 or 512 keys) is chosen at build time
+    # from the device's SM count, so the workspace, sized without a device, must
+    # hold the per-chunk row statistics and slash windows of any of them, on top
+    # of the v and s sums.
+    nvs = 3
+    kinds = [dict(kind="vs", last_q=128, n_vert=10, n_slash=20)] * nvs + [dict(kind="ashape", sink=4, window=100)]
+    p = problem(B, Hq=4, Hkv=2, N=N, block=64)
+    st, sz = status_of(B, p, pats(B, kinds))
+    assert st == 0
+    need = 2 * nvs * N * 4  # v and s
+    for c in (1024, 768, 512):
+        nch = -(-N // c)
+        parts = nvs * nch * 128 * 2 * 4  # (max, sum) of up to 128 estimate rows per chunk
+        wins = nvs * nch * (c + 128) * 4  # slash window per chunk
+        assert sz.workspace_bytes >= need + parts + wins, (N, c)
+
+
 def test_null_pointers_rejected_before_launch(B):
     p = problem(B)
     pp = pats(B, DEF)
