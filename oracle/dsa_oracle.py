@@ -38,6 +38,9 @@ Readings where the pages are silent:
 * VS index form: block-distance set D = {floor(o/B), ceil(o/B) : o in S} (clipped
   to [0, nkb)), query block qb keeps key blocks {qb - delta : delta in D, delta <= qb},
   and its columns are the verticals j <= qb*B+B-1 whose block is not already kept;
+  with ``slash_cover="windows"`` the slashes are instead covered by the exact keys
+  they reach from each query block, merged into runs (not aligned to blocks),
+  and the columns are the verticals outside those runs;
 * threshold in probability space: keep J <= I with P_IJ >= alpha * max_J P_IJ,
   plus the sink block 0 and the local block I when asked;
 * MoBA: top-k over J < I by tau * qbar_I . kbar_J, plus the own block I; the key
@@ -149,6 +152,38 @@ def vs_columns(V: np.ndarray, D: np.ndarray, qb: int, B: int) -> np.ndarray:
     return np.asarray(keep, dtype=np.int64)
 
 
+def vs_slash_runs(S: np.ndarray, qb: int, B: int, N: int) -> np.ndarray:
+    """The keys that slash lines S reach from query block qb, as maximal runs.
+
+    Rows r0..r1 of the block meet slash o at keys r0 - o .. r1 - o, a window of the
+    block's height; keys below 0 do not exist.  Windows that overlap or touch are
+    merged.  Returns an int64 array [n, 2] of (first, last) keys, inclusive, in
+    ascending order.  (The unaligned alternative to covering each slash with two
+    aligned key blocks; the key set equals {i - o : r0 <= i <= r1, o in S, i >= o}.)"""
+    r0 = qb * B
+    r1 = min(N, r0 + B) - 1
+    runs = []
+    # larger offsets start further left: descending o gives ascending windows
+    for o in sorted((int(x) for x in S), reverse=True):
+        if o > r1:
+            continue
+        a, b = max(0, r0 - o), r1 - o
+        if runs and a <= runs[-1][1] + 1:
+            runs[-1][1] = max(runs[-1][1], b)
+        else:
+            runs.append([a, b])
+    return np.asarray(runs, dtype=np.int64).reshape(-1, 2)
+
+
+def vs_window_columns(V: np.ndarray, runs: np.ndarray, qb: int, B: int) -> np.ndarray:
+    """Vertical columns query block qb adds on top of its slash runs: j in V that
+    some row of the block can see (j <= qb*B+B-1) and that lies in no run."""
+    V = np.asarray(V, dtype=np.int64)
+    keep = [int(j) for j in V
+            if j <= qb * B + B - 1 and not any(a <= j <= b for a, b in runs)]
+    return np.asarray(keep, dtype=np.int64)
+
+
 # ---------------------------------------------------------------------------
 # Block scoring  [MI] (mean-pool Q and K per block, block-level attention),
 # [FP] 2.1 (mean-pooled key per block), [MoBA] (router over KV blocks).
@@ -232,6 +267,7 @@ class HeadIndex:
     vscore: np.ndarray | None = None
     sscore: np.ndarray | None = None
     block_scores: np.ndarray | None = None   # [nqb, nkb] logits (block kinds)
+    runs: list | None = None   # VS with slash_cover "windows": [n, 2] key runs per query block
 
 
 def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
@@ -254,9 +290,17 @@ def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
         hi.vscore, hi.sscore = v, s
         hi.V = topk_indices(v, int(pattern["n_vert"]))
         hi.S = topk_indices(s, int(pattern["n_slash"]))
-        hi.D = vs_distance_set(hi.S, B, nqb)
-        hi.blocks = [np.sort(qb - hi.D[hi.D <= qb]) for qb in range(nqb)]
-        hi.cols = [vs_columns(hi.V, hi.D, qb, B) for qb in range(nqb)]
+        cover = pattern.get("slash_cover", "blocks")
+        if cover == "blocks":
+            hi.D = vs_distance_set(hi.S, B, nqb)
+            hi.blocks = [np.sort(qb - hi.D[hi.D <= qb]) for qb in range(nqb)]
+            hi.cols = [vs_columns(hi.V, hi.D, qb, B) for qb in range(nqb)]
+        elif cover == "windows":
+            hi.runs = [vs_slash_runs(hi.S, qb, B, N) for qb in range(nqb)]
+            hi.blocks = [empty] * nqb
+            hi.cols = [vs_window_columns(hi.V, hi.runs[qb], qb, B) for qb in range(nqb)]
+        else:
+            raise ValueError(f"unknown slash_cover {cover!r}")
     elif kind in (BLOCK_TOPK, BLOCK_THRESHOLD, MOBA):
         keys = Kh
         if kind == MOBA and conv is not None:
@@ -286,7 +330,7 @@ def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
 # ---------------------------------------------------------------------------
 def allowed_keys(hi: HeadIndex, i: int) -> np.ndarray:
     """The index mask of row i as a sorted set of key positions: keys of the
-    listed blocks and listed columns of row i's query block, restricted to j <= i
+    listed blocks, slash runs and columns of row i's query block, restricted to j <= i
     (and to the A-shape predicate for A-shape heads).  A key listed twice is one
     key."""
     B = hi.B
@@ -294,6 +338,8 @@ def allowed_keys(hi: HeadIndex, i: int) -> np.ndarray:
     blk = np.asarray(hi.blocks[qb], dtype=np.int64)
     from_blocks = (blk[:, None] * B + np.arange(B)[None, :]).ravel() if blk.size else np.zeros(0, np.int64)
     keys = np.union1d(from_blocks, np.asarray(hi.cols[qb], dtype=np.int64))
+    if hi.runs is not None and hi.runs[qb].size:
+        keys = np.union1d(keys, np.concatenate([np.arange(a, b + 1) for a, b in hi.runs[qb]]))
     keys = keys[(keys <= i) & (keys < hi.N)]
     if hi.kind == ASHAPE:
         keys = keys[ashape_allowed(i, keys, hi.sink, hi.window)]

@@ -153,6 +153,64 @@ def test_vs_index_superset_and_no_double_count(rng, N, B, nv, ns):
         assert not any(j // B in covered for j in hi.cols[qb])
 
 
+def test_vs_slash_windows_hand_example():
+    g = json.load(open(os.path.join(GOLDEN, "vs_slash_windows_hand_example.json")))
+    N, B, S, V = g["N"], g["block"], np.array(g["S"]), np.array(g["V"])
+    nqb = (N + B - 1) // B
+    hi = orc.HeadIndex(kind=orc.VS, B=B, N=N, V=V, S=S)
+    hi.runs = [orc.vs_slash_runs(S, qb, B, N) for qb in range(nqb)]
+    hi.blocks = [np.zeros(0, np.int64)] * nqb
+    hi.cols = [orc.vs_window_columns(V, hi.runs[qb], qb, B) for qb in range(nqb)]
+    assert [r.tolist() for r in hi.runs] == g["runs_per_query_block"]
+    assert [list(c) for c in hi.cols] == g["columns_per_query_block"]
+    assert list(orc.allowed_keys(hi, 10)) == g["row_10_keys"]
+
+
+@pytest.mark.parametrize("B", [4, 8, 16])
+def test_vs_slash_runs_are_the_slash_cells_of_each_block(B):
+    rng = np.random.default_rng(100 + B)
+    N = 150
+    for trial in range(20):
+        S = rng.choice(N, size=int(rng.integers(1, 15)), replace=False)
+        for qb in range((N + B - 1) // B):
+            runs = orc.vs_slash_runs(S, qb, B, N)
+            got = set()
+            for a, b in runs:
+                got |= set(range(a, b + 1))
+            want = set()
+            for i in range(qb * B, min(N, qb * B + B)):
+                for o in S:
+                    if i - o >= 0:
+                        want.add(int(i - o))
+            assert got == want
+            # ascending, disjoint and not touching (maximal runs)
+            for (a0, b0), (a1, b1) in zip(runs[:-1], runs[1:]):
+                assert a0 <= b0 < a1 - 1 < b1
+
+
+@pytest.mark.parametrize("N,B,nv,ns", [(64, 8, 5, 4), (77, 16, 9, 3), (50, 4, 2, 20), (90, 8, 0, 7)])
+def test_vs_window_mask_between_exact_and_aligned_blocks(N, B, nv, ns):
+    rng = np.random.default_rng(N + B)
+    Q = rng.standard_normal((N, 6))
+    K = rng.standard_normal((N, 6))
+    pat = dict(kind="vs", last_q=10, n_vert=nv, n_slash=ns)
+    hw = orc.build_head_index(Q, K, dict(pat, slash_cover="windows"), B)
+    hb = orc.build_head_index(Q, K, pat, B)
+    assert list(hw.V) == list(hb.V) and list(hw.S) == list(hb.S)
+    Mw, Mb = orc.index_mask_dense(hw), orc.index_mask_dense(hb)
+    Vs, Ss = set(int(x) for x in hw.V), set(int(x) for x in hw.S)
+    for i in range(N):
+        for j in range(N):
+            exact = j <= i and (j in Vs or (i - j) in Ss)
+            assert not exact or Mw[i, j]      # every exact VS cell is kept
+            assert not Mw[i, j] or Mb[i, j]   # the runs never go past the aligned blocks
+    for qb in range(len(hw.runs)):
+        in_runs = lambda j: any(a <= j <= b for a, b in hw.runs[qb])
+        want = [j for j in sorted(Vs) if j <= qb * B + B - 1 and not in_runs(j)]
+        assert list(hw.cols[qb]) == want
+    assert orc.selected_pairs(hw) <= orc.selected_pairs(hb)
+
+
 def test_vs_estimate_picks_planted_verticals():
     w = synth.workload(1)
     Q, K, V, planted = synth.make_inputs(w)
