@@ -81,7 +81,7 @@ def test_gathered_shards_equal_the_layer(world):
     Q, K, V, pats = _layer()
     ref = _oracle_compute(Q, K, V, pats, 32).numpy()
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(world, port, out), nprocs=world, join=True)
         res = dict(out)
