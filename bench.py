@@ -119,15 +119,24 @@ def reduce_max_over_ranks(values, device="cpu"):
     return t.tolist()
 
 
-def kernel_source_hash(path):
-    """16 hex digits of the SHA-256 of a CUDA source with its // comments and
-    blank lines removed: profiler counters stay tied to the code, not its prose."""
+# the sources the attention kernel is compiled from (its .cu and the headers it includes)
+ATTN_SOURCES = ("dsa_attn.cu", "dsa_common.cuh", "dsa_internal.h")
+
+
+def kernel_source_hash(paths):
+    """16 hex digits of the SHA-256 of CUDA sources (in the given order) with their
+    // comments and blank lines removed: profiler counters stay tied to the code,
+    not its prose."""
     import hashlib
+    if isinstance(paths, str):
+        paths = [paths]
     lines = []
-    for ln in open(path, encoding="utf-8").read().splitlines():
-        code = ln.split("//", 1)[0].rstrip()
-        if code:
-            lines.append(code)
+    for path in paths:
+        lines.append("@" + os.path.basename(path))
+        for ln in open(path, encoding="utf-8").read().splitlines():
+            code = ln.split("//", 1)[0].rstrip()
+            if code:
+                lines.append(code)
     return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:16]
 
 
@@ -387,8 +396,8 @@ def main():
         # DRAM bytes per launch from an ncu capture; only valid for the kernel
         # source it was taken on and for this workload
         tr = json.load(open(tp))
-        src = os.path.join(ROOT, "dynamic_sparse_attention_build_b200", "csrc", "dsa_attn.cu")
-        sha = kernel_source_hash(src)
+        csrc = os.path.join(ROOT, "dynamic_sparse_attention_build_b200", "csrc")
+        sha = kernel_source_hash([os.path.join(csrc, f) for f in ATTN_SOURCES])
         if tr.get("workload") == w["name"] and tr.get("kernel_source_sha256_16") == sha and w["N"] == 32768:
             traffic = tr.get("dram_bytes_per_launch")
 
