@@ -103,6 +103,14 @@ def test_workload5_slice_4heads_64k(dsa):
     run_workload(dsa, w, [0, 3], row_blocks=4, rows_per_block=8)
 
 
+def test_workload5_slice_3heads_64k(dsa):
+    """Three q-heads on one KV head at 65536 tokens: 192 CTAs of 1024-key estimate
+    chunks leave a 148-SM B200 (296 CTA slots) under one wave and 512-key chunks
+    (384) overflow it, so the VS estimate runs on 768-key chunks (258 CTAs)."""
+    w = synth.workload(5, N=65536, Hq=3, Hkv=1)
+    run_workload(dsa, w, [0, 2], row_blocks=4, rows_per_block=8)
+
+
 def test_workload5_vs_1m(dsa):
     """Full million-token layer: VS top-k of 2 heads against the oracle and 4 heads'
     outputs on one sampled row of each of 16 seeded query blocks."""
