@@ -1,7 +1,7 @@
 // Causal block-sparse attention forward for sm_100a.
 //
-// What it computes (MInference abstract: sparse attention "with the pattern and
-// sparse indices"; FlashPrefill section 2.3: the kernel jumps straight to the
+// What it computes (MInference abstract: attention restricted to the index lists
+// built for each head's pattern; FlashPrefill section 2.3: the kernel jumps straight to the
 // listed blocks instead of testing every block): for row i of head h,
 //   O_i = sum_{j in M_i} softmax_j(tau q_i.k_j) v_j,
 // where M_i holds the keys j <= i of the key blocks listed for i's query block

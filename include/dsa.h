@@ -10,9 +10,10 @@
  *   dsa_sparse_prefill: causal FlashAttention-style forward pass over only the
  *                       listed key blocks and key columns.
  *
- * The split into "build the indices from the assigned pattern" and "run sparse
- * attention with the pattern and the indices" is the one the MInference abstract
- * (zhuanzhiai.com page) states.  Pattern definitions:
+ * The two calls follow the MInference abstract (zhuanzhiai.com page): a head's
+ * pattern is fixed ahead of time, its index lists are built from that pattern
+ * when the layer runs, and attention then reads only those lists.  Pattern
+ * definitions:
  *   - A-shape, Vertical-Slash, block-sparse: "MInference 1.0" summary (abeam.tech),
  *     sections "3つの疎パターン" and "推論時は軽い近似で動的マスクを作る";
  *   - max-relative block threshold: "FlashPrefill" summary (gist.science), section
@@ -157,8 +158,8 @@ typedef struct dsa_sizes {
  * Returns DSA_ERR_INVALID_ARG / DSA_ERR_UNSUPPORTED on a bad request. */
 dsa_status dsa_workspace_size(const dsa_problem* p, const dsa_pattern* pats, dsa_sizes* out);
 
-/* Builds the indices of every head (MInference abstract: "dynamically build sparse
- * indices based on the assigned pattern").  Q, K: device bf16 with the problem's
+/* Builds the index lists of every head from its pattern, at run time (the
+ * MInference abstract's second step).  Q, K: device bf16 with the problem's
  * strides.  pats: host array [Hq].  out: index arrays with capacities at least those
  * of dsa_workspace_size.  workspace: device scratch of at least
  * sizes.workspace_bytes (256-byte aligned); its contents on entry do not matter.
@@ -168,8 +169,8 @@ dsa_status dsa_build_indices(const dsa_problem* p, const void* Q, const void* K,
                              const dsa_pattern* pats, const dsa_indices* out,
                              void* workspace, size_t workspace_bytes, dsa_stream stream);
 
-/* Sparse attention forward (MInference abstract: sparse attention "with the pattern
- * and sparse indices"; FlashPrefill section 2.3: only listed blocks are visited).
+/* Sparse attention forward (MInference abstract: attention over each head's index
+ * lists only; FlashPrefill section 2.3: only listed blocks are visited).
  * Row i of head h attends to key j iff j <= i and (j is in a listed block of its
  * query block, or j is a listed column), and for A-shape heads also
  * (j < sink or i - j < window).  A key listed twice counts once.

@@ -15,9 +15,9 @@ Sources (page title, section):
         three sparse patterns: A-shape, Vertical-Slash, Block-Sparse) and
         "推論時は軽い近似で動的マスクを作る" (building the dynamic mask at inference
         time from Q[-last_q:] x K, or from mean-pooled Q/K blocks).
-* [MIa] MInference abstract (zhuanzhiai.com): indices are built dynamically from
-        the assigned pattern, then sparse attention runs "with the pattern and
-        sparse indices".
+* [MIa] MInference abstract (zhuanzhiai.com): each head's index lists are built
+        at run time from its fixed pattern, and attention is then computed over
+        those lists only.
 * [FP]  "FlashPrefill: Instantaneous Pattern Discovery and Thresholding for
         Ultra-Fast Long-Context Prefilling" (gist.science summary) -- section 2.1
         (mean-pooled key per block) and section 2.2, the equation
@@ -325,8 +325,8 @@ def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
 
 
 # ---------------------------------------------------------------------------
-# Attention given indices  [MIa]: sparse attention "with the pattern and sparse
-# indices"; [FP] 2.3 (only listed blocks are visited).
+# Attention given indices  [MIa]: attention over the index lists of each head's
+# pattern; [FP] 2.3 (only listed blocks are visited).
 # ---------------------------------------------------------------------------
 def allowed_keys(hi: HeadIndex, i: int) -> np.ndarray:
     """The index mask of row i as a sorted set of key positions: keys of the
