@@ -188,6 +188,29 @@ def test_vs_slash_runs_are_the_slash_cells_of_each_block(B):
                 assert a0 <= b0 < a1 - 1 < b1
 
 
+@pytest.mark.parametrize("B", [4, 16, 64])
+def test_vs_slash_runs_are_the_dilated_offsets_mirrored(B):
+    # Key j is reached from rows r0..r1 on slash o iff r0 - o <= j <= r1 - o, i.e.
+    # r1 - j lies in [o, o + L - 1] with L = r1 - r0 + 1.  So the runs of a query
+    # block are the merged intervals of those dilated offsets, mirrored at r1 and
+    # clipped at key 0: one per-head list serves every query block of height L.
+    rng = np.random.default_rng(7 * B)
+    N = 700
+    for trial in range(10):
+        S = rng.choice(N, size=int(rng.integers(1, 40)), replace=False)
+        for qb in range((N + B - 1) // B):
+            r0, r1 = qb * B, min(N, qb * B + B) - 1
+            L = r1 - r0 + 1
+            ivs = []
+            for o in sorted(int(x) for x in S):  # merged [o, o + L - 1], ascending
+                if ivs and o <= ivs[-1][1] + 1:
+                    ivs[-1][1] = max(ivs[-1][1], o + L - 1)
+                else:
+                    ivs.append([o, o + L - 1])
+            mirrored = [[max(0, r1 - hi), r1 - lo] for lo, hi in reversed(ivs) if r1 - lo >= 0]
+            assert orc.vs_slash_runs(S, qb, B, N).tolist() == mirrored
+
+
 @pytest.mark.parametrize("N,B,nv,ns", [(64, 8, 5, 4), (77, 16, 9, 3), (50, 4, 2, 20), (90, 8, 0, 7)])
 def test_vs_window_mask_between_exact_and_aligned_blocks(N, B, nv, ns):
     rng = np.random.default_rng(N + B)
