@@ -124,6 +124,25 @@ def test_distance_set_covers_slash_cells(B):
                 assert dist == set(int(x) for x in D)
 
 
+@pytest.mark.parametrize("B", [4, 8, 16])
+def test_distance_set_is_exactly_the_reached_distances(B):
+    # With N a multiple of B the last query block is full, so every distance in D
+    # is reached by some block's slash cells and no other distance is: D holds
+    # nothing that can never apply (no distance >= the number of key blocks).
+    rng = np.random.default_rng(50 + B)
+    N = 160
+    nb = N // B
+    for trial in range(20):
+        S = rng.choice(N, size=int(rng.integers(1, 12)), replace=False)
+        reached = set()
+        for qb in range(nb):
+            for i in range(qb * B, qb * B + B):
+                for o in S:
+                    if i - o >= 0:
+                        reached.add(qb - (i - int(o)) // B)
+        assert set(int(x) for x in orc.vs_distance_set(S, B, nb)) == reached
+
+
 def _vs_head(rng, N, d, B, last_q, n_vert, n_slash):
     Q = rng.standard_normal((N, d))
     K = rng.standard_normal((N, d))
