@@ -48,7 +48,9 @@ Readings where the pages are silent:
 * a row with no allowed key has O = 0 and LSE = -inf.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against brute force, closed forms or a library routine.  Parity unpinned: the VS
+against brute force, closed forms or a library routine, and
+``tests/test_oracle_mutations.py`` plants plausible mistakes in a copy of this
+module to check that each one fails a pin.  Parity unpinned: the VS
 aggregation rule and the forced blocks of each kind rest on the readings above,
 not on anything the pages fix.
 """
