@@ -233,7 +233,7 @@ PATTERN_TEXT = {
 }
 
 
-def main():
+def build_arg_parser():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
@@ -250,7 +250,11 @@ def main():
                     help="strong scaling: the ranks split ONE layer by KV groups (default: one layer per rank)")
     ap.add_argument("--gather", action="store_true",
                     help="with --shard-heads: all-gather every rank's O into the full layer output each step")
-    args = ap.parse_args()
+    return ap
+
+
+def main():
+    args = build_arg_parser().parse_args()
     rank, world, local = dist_env()
     over = {}
     if args.N:
