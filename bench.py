@@ -2,10 +2,13 @@
 
 One step = the whole hot path over one layer of synthetic input: build the
 per-head sparse indices (dsa_build_indices) and run the sparse attention forward
-(dsa_sparse_prefill).  The default workload is the Llama-3-8B-shaped layer:
-32 q / 8 KV heads, d = 128, N = 32768 tokens, bf16, per-head patterns drawn from
-the seed (20% A-shape 128/1024, 60% Vertical-Slash 64/1000/6096, 20% block
-top-100), block 64.
+(dsa_sparse_prefill).  The default workload is the FlashPrefill-style
+block-threshold layer: 32 q / 8 KV heads, d = 128, N = 131072 tokens, bf16, K/V/Q
+built from 512 latent topics per 128-token block, every head keeping the blocks
+whose pooled score is within alpha = 0.5 (probability space) of the row maximum,
+plus the sink and local block, block 128.  The attention kernel's tensor-peak
+target is stated on this layer.  The other layers (VS 4K, Llama-3-8B-shaped mixed
+32K, MoBA 64K, VS 1M) are behind --workload.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl dsa|reference]
 
@@ -239,7 +242,7 @@ def build_arg_parser():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="dsa", choices=["dsa", "reference"])
-    ap.add_argument("--workload", type=int, default=2)
+    ap.add_argument("--workload", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--e2e-chunks", type=int, default=8, help="KV-group chunks of the overlapped host path")
@@ -387,11 +390,11 @@ def main():
 
     pk, pk_src = peaks()
     tflops = f_sel / (ms_attn * 1e-3) / 1e12
-    # a kernel timed alone gets the burst peak; one timed inside seconds of
-    # back-to-back steps runs under the power cap and gets the sustained one
-    long_run = tot[0] > 2000.0
-    peak_tf = pk["bf16_tflops_sustained"] if long_run else pk["bf16_tflops"]
-    peak_kind = "bf16 sustained (cuBLAS, seconds under the power cap)" if long_run else "bf16 burst (cuBLAS)"
+    # one fixed denominator for the fraction: the measured dense bf16 burst peak;
+    # the fraction of the sustained (power-capped) peak is reported beside it
+    peak_tf = pk["bf16_tflops"]
+    peak_kind = "bf16 burst (cuBLAS)"
+    peak_sus = pk.get("bf16_tflops_sustained")
     idx_bytes, nqb = algorithmic_index_bytes(w, pats)
     idx_gbs = idx_bytes / (ms_build * 1e-3) / 1e9
     traffic = None
@@ -422,6 +425,7 @@ def main():
                      "kernel": "sparse_attn_kernel<128>", "peak_source": f"{pk_src} {peak_kind}",
                      "work": f"F_sel = 4*d*|M| = {f_sel:.4e} FLOP per launch ({pairs} allowed pairs)"},
         "attention": {"ms": ms_attn, "tflops": tflops, "frac_peak": tflops / peak_tf,
+                      "frac_sustained_peak": (tflops / peak_sus) if peak_sus else None,
                       "density_vs_causal": pairs / causal_pairs},
         "index_build": {"ms": ms_build, "algorithmic_bytes": idx_bytes, "gbs": idx_gbs,
                         "frac_hbm": idx_gbs / pk["hbm_gbs"], "hbm_peak_source": pk_src},

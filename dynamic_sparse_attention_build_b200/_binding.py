@@ -31,7 +31,7 @@ KIND_CODES = {"ashape": DSA_KIND_ASHAPE, "vs": DSA_KIND_VS, "block_topk": DSA_KI
 
 EXPORTS = ("dsa_workspace_size", "dsa_build_indices", "dsa_sparse_prefill", "dsa_count_pairs",
            "dsa_get_device_status", "dsa_selftest_wait_timeout", "dsa_status_string",
-           "dsa_last_cuda_error", "dsa_build_indices_static")
+           "dsa_last_cuda_error", "dsa_build_indices_static", "dsa_set_wait_limit")
 
 
 class dsa_problem(ctypes.Structure):
@@ -92,6 +92,7 @@ def lib():
         L.dsa_count_pairs.argtypes = [P(dsa_problem), P(dsa_indices), ctypes.c_void_p, ctypes.c_void_p]
         L.dsa_get_device_status.argtypes = [ctypes.c_void_p, P(ctypes.c_int32)]
         L.dsa_selftest_wait_timeout.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
+        L.dsa_set_wait_limit.argtypes = [ctypes.c_uint64]
         L.dsa_status_string.argtypes = [ctypes.c_int]
         L.dsa_status_string.restype = ctypes.c_char_p
         L.dsa_last_cuda_error.argtypes = []
@@ -150,6 +151,10 @@ def dsa_get_device_status(stream_ptr):
 
 def dsa_selftest_wait_timeout(timeout_us, stream_ptr):
     return lib().dsa_selftest_wait_timeout(timeout_us, stream_ptr)
+
+
+def dsa_set_wait_limit(limit_ns):
+    return lib().dsa_set_wait_limit(limit_ns)
 
 
 def dsa_status_string(status):

@@ -299,3 +299,8 @@ class HostPrefill:
                 last.record(self.d2h)
         cur.wait_event(last)
         return Oh
+
+    def status(self):
+        """(status, detail) of the kernels that ``run`` enqueued (they run on this
+        object's compute stream); synchronises that stream and clears the word."""
+        return device_status(self.comp)

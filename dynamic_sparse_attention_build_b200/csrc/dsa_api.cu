@@ -3,18 +3,32 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
 namespace dsa {
 
-// Per-device status word: [0] first error code, [1] detail, [2] block, [3] spare.
-__device__ unsigned g_status[4];
+// Status words, kStatusSlots per device, each [0] first error code, [1] detail,
+// [2] block, [3] spare.  A call uses the word of its stream's slot, so errors of
+// work on one stream are not reported to a caller of another (unless their
+// handles fall on the same slot).
+constexpr int kStatusSlots = 64;
+__device__ unsigned g_status[kStatusSlots * 4];
 
 namespace {
 thread_local int32_t t_last_cuda_error = 0;
 constexpr int kMaxDevices = 64;
-unsigned* g_status_addr[kMaxDevices] = {};
+std::atomic<unsigned*> g_status_addr[kMaxDevices] = {};
+
+int status_slot(cudaStream_t s) {
+  uint64_t x = static_cast<uint64_t>(reinterpret_cast<uintptr_t>(s));
+  x ^= x >> 29;
+  x *= 0x9E3779B97F4A7C15ull;  // Fibonacci hashing of the handle value
+  return static_cast<int>(x >> 58);  // top 6 bits: 0 .. 63
+}
+static_assert(kStatusSlots == 64, "status_slot returns 6 bits");
 
 __global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns) {
   pdl_prologue();
@@ -33,20 +47,28 @@ __global__ void selftest_wait_kernel(unsigned* status, uint64_t limit_ns) {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 }  // namespace
 
+namespace {
+std::atomic<uint64_t> g_wait_limit{kWaitLimitNs};
+}  // namespace
+
+uint64_t wait_limit_ns() { return g_wait_limit.load(); }
+
 dsa_status cuda_fail(cudaError_t e) {
   t_last_cuda_error = (int32_t)e;
   return DSA_ERR_CUDA;
 }
 
-unsigned* status_ptr() {
+unsigned* status_ptr(cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (g_status_addr[dev] == nullptr) {
+  unsigned* base = g_status_addr[dev].load();
+  if (base == nullptr) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
-    g_status_addr[dev] = static_cast<unsigned*>(p);
+    base = static_cast<unsigned*>(p);
+    g_status_addr[dev].store(base);  // every thread that races here finds the same address
   }
-  return g_status_addr[dev];
+  return base + 4 * status_slot(stream);
 }
 
 dsa_status validate_problem(const dsa_problem* p) {
@@ -97,7 +119,7 @@ dsa_status dsa_build_indices(const dsa_problem* p, const void* Q, const void* K,
   s = validate_indices_ptrs(out, true);
   if (s != DSA_OK) return s;
   if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return DSA_ERR_INVALID_ARG;
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   return launch_build_indices(*p, Q, K, pats, *out, workspace, workspace_bytes, (cudaStream_t)stream, st);
 }
@@ -110,7 +132,7 @@ dsa_status dsa_sparse_prefill(const dsa_problem* p, const void* Q, const void* K
     return DSA_ERR_INVALID_ARG;
   s = validate_indices_ptrs(idx, false);
   if (s != DSA_OK) return s;
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   return launch_sparse_attn(*p, Q, K, V, *idx, O, lse, (cudaStream_t)stream, st);
 }
@@ -121,7 +143,7 @@ dsa_status dsa_count_pairs(const dsa_problem* p, const dsa_indices* idx, int64_t
   if (pairs == nullptr) return DSA_ERR_INVALID_ARG;
   s = validate_indices_ptrs(idx, false);
   if (s != DSA_OK) return s;
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   return launch_count_pairs(*p, *idx, pairs, (cudaStream_t)stream, st);
 }
@@ -129,7 +151,7 @@ dsa_status dsa_count_pairs(const dsa_problem* p, const dsa_indices* idx, int64_t
 dsa_status dsa_get_device_status(dsa_stream stream, int32_t* detail) {
   cudaError_t e = cudaStreamSynchronize((cudaStream_t)stream);
   if (e != cudaSuccess) return cuda_fail(e);
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   unsigned host[4] = {0, 0, 0, 0};
   e = cudaMemcpy(host, st, sizeof(host), cudaMemcpyDeviceToHost);
@@ -150,11 +172,17 @@ dsa_status dsa_get_device_status(dsa_stream stream, int32_t* detail) {
 
 dsa_status dsa_selftest_wait_timeout(uint32_t timeout_us, dsa_stream stream) {
   if (timeout_us == 0 || timeout_us > 10000000u) return DSA_ERR_INVALID_ARG;
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   selftest_wait_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(st, (uint64_t)timeout_us * 1000ull);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
+  return DSA_OK;
+}
+
+dsa_status dsa_set_wait_limit(uint64_t limit_ns) {
+  if (limit_ns > 60ull * 1000000000ull) return DSA_ERR_INVALID_ARG;
+  g_wait_limit.store(limit_ns == 0 ? kWaitLimitNs : limit_ns);
   return DSA_OK;
 }
 

@@ -61,24 +61,11 @@ constexpr int NINFO = 4;           // StageInfo slots (a slot is reused after it
 // after the final division; 2^32 leaves P <= 2^32, l and O <= 2^53 |V| for 2^21
 // keys, far inside fp32 range, and avoids almost every O rescale.
 constexpr float RESCALE_THRESHOLD = 32.0f;
-#ifndef DSA_LOADER_SUSPEND
-#define DSA_LOADER_SUSPEND 1
-#endif
-#ifndef DSA_MMA_SUSPEND
-#define DSA_MMA_SUSPEND 1
-#endif
-// Waits of the TMA producer / MMA thread block in try_wait (the warp then takes
-// no issue slots from the softmax warp that shares its scheduler) instead of
-// polling.
-constexpr bool kLoaderSuspend = DSA_LOADER_SUSPEND != 0;
-constexpr bool kMmaSuspend = DSA_MMA_SUSPEND != 0;
-#ifndef DSA_POLY_PERIOD
-// One exp2 pair in DSA_POLY_PERIOD runs on the FMA pipe (0: none).  Off: the
-// exponentials do not saturate the XU pipe in this kernel, and the smaller loop
-// body measured faster.
-#define DSA_POLY_PERIOD 0
-#endif
-constexpr int kPolyPeriod = DSA_POLY_PERIOD > 0 ? DSA_POLY_PERIOD : 1 << 20;
+// Waits of the TMA producer and of the MMA thread block in try_wait (the warp
+// then takes no issue slots from the softmax warp that shares its scheduler)
+// instead of polling.
+constexpr bool kLoaderSuspend = true;
+constexpr bool kMmaSuspend = true;
 
 struct StageInfo {
   int type;   // 0 = key unit, 1 = column tile
@@ -111,6 +98,7 @@ struct AttnArgs {
   const int32_t* dist;
   const int32_t* col_ptr;
   const int32_t* col_idx;
+  int64_t blk_cap, dist_cap, col_cap;  // lengths of blk_idx, dist, col_idx
   const __nv_bfloat16* K;
   const __nv_bfloat16* V;
   int64_t k_hs, k_ts, v_hs, v_ts;
@@ -119,7 +107,8 @@ struct AttnArgs {
   int o_v8;  // O rows are 32-byte aligned: 256-bit stores
   float* lse;
   float scale_log2;
-  unsigned* sched;  // [0] items handed out past the first wave, [1] CTAs finished
+  unsigned long long* sched;  // item counter: launch epoch (high 32 bits), items handed out (low 32)
+  unsigned epoch;             // this launch's epoch (never 0)
   unsigned* status;
   uint64_t wait_limit_ns;
 };
@@ -198,38 +187,6 @@ __device__ __forceinline__ void fma2(float a0, float a1, float b, float c, float
   asm("mov.b64 %0, {%1, %2};" : "=l"(cv) : "f"(c), "f"(c));
   asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(bv), "l"(cv));
   asm("mov.b64 {%0, %1}, %2;" : "=f"(x0), "=f"(x1) : "l"(r));
-}
-
-// 2^x for two values on the FMA and integer pipes instead of the XU pipe:
-// x = j + f with j = round(x) (taken from the low mantissa bits after adding
-// 1.5 * 2^23) and f in [-1/2, 1/2]; 2^f from a degree-3 polynomial fitted for this
-// library to minimise the relative error on [-1/2, 1/2] (max 7.5e-5, far below the
-// bf16 rounding of P); 2^j is added to the exponent field.  x is clamped at -125 so
-// that the exponent field stays normal, and inputs below -125 (masked keys are
-// -inf) give exactly 0, like ex2.approx.ftz.
-__device__ __forceinline__ void poly_ex2x2(float x0, float x1, float& y0, float& y1) {
-  constexpr float kShift = 12582912.0f;  // 1.5 * 2^23
-  constexpr float c0 = 0.99992807f, c1 = 0.693261f, c2 = 0.24261112f, c3 = 0.05517161f;
-  const float c0x = fmaxf(x0, -125.f);
-  const float c1x = fmaxf(x1, -125.f);
-  uint64_t xv, sh, yv, jv, fv, pv, cv;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(xv) : "f"(c0x), "f"(c1x));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(sh) : "f"(kShift));
-  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(yv) : "l"(xv), "l"(sh));   // y = x + shift
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(jv) : "l"(yv), "l"(sh));   // j = round(x)
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(fv) : "l"(xv), "l"(jv));   // f = x - j
-  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c3));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(pv) : "f"(c2));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(cv), "l"(fv), "l"(pv));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c1));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(pv), "l"(fv), "l"(cv));
-  asm("mov.b64 %0, {%1, %1};" : "=l"(cv) : "f"(c0));
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(pv) : "l"(pv), "l"(fv), "l"(cv));
-  uint32_t p0, p1, j0, j1;
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(p0), "=r"(p1) : "l"(pv));
-  asm("mov.b64 {%0, %1}, %2;" : "=r"(j0), "=r"(j1) : "l"(yv));
-  y0 = x0 > -125.f ? __uint_as_float(p0 + (j0 << 23)) : 0.f;
-  y1 = x1 > -125.f ? __uint_as_float(p1 + (j1 << 23)) : 0.f;
 }
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -324,6 +281,47 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
       : "memory");
 }
 
+// Next item index past the first wave.  The counter word carries the epoch of
+// the launch that last used it in its high 32 bits.  A launch that finds another
+// epoch there (a word left by an earlier launch, even one that ended early)
+// restarts the count at its own epoch: one CTA's compare-and-swap succeeds and
+// takes item 0, the others see the new epoch and count on from it.  So no launch
+// has to clear the word when it ends, and the common case is one atomic add.
+__device__ __forceinline__ int sched_next(unsigned long long* ctr, unsigned epoch) {
+  while (true) {
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    if ((unsigned)(old >> 32) == epoch) return (int)(unsigned)(old & 0xffffffffull);
+    unsigned long long cur = old + 1ull;
+    while ((unsigned)(cur >> 32) != epoch) {
+      const unsigned long long prev = atomicCAS(ctr, cur, ((unsigned long long)epoch << 32) | 1ull);
+      if (prev == cur) return 0;
+      cur = prev;
+    }
+  }
+}
+
+// A CSR row [beg, end) is usable only if 0 <= beg <= end <= cap; otherwise the
+// row is reported (DSA_ERR_DEVICE, `detail`) and treated as empty, so a
+// malformed list never makes the kernel read outside the caller's arrays.
+__device__ __forceinline__ void checked_row(int& beg, int& end, int64_t cap, unsigned* status, unsigned detail) {
+  if (!(0 <= beg && beg <= end && (int64_t)end <= cap)) {
+    report(status, DSA_ERR_DEVICE, detail);
+    beg = 0;
+    end = 0;
+  }
+}
+
+// Waits, bounded by the default limit whatever the launch's own limit and
+// ignoring the abort flag, for a TMA load this CTA issued to land.  Used after an
+// abort, so that no copy can still be writing into the CTA's shared memory when
+// the CTA exits.  A wait that runs out has nothing left to report.
+static __device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -335,8 +333,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR_OFF);
   int* misc = reinterpret_cast<int*>(sm + L::MISC_OFF);
-  // misc: [0] tmem base, [2] abort, [3] unit count, [4] col count half0, [5] col count half1,
-  //       [6] col base half0, [7] col base half1, [9] loader go flag, [10] current item
+  // misc: [0] tmem base, [2] abort, [3] unit count, [9] decoder go flag, [10] current item,
+  //       [11] / [12] K / V tiles the MMA thread has seen land, [13] items whose Q it has seen land
   volatile int* abort_flag = misc + 2;
   uint32_t* bits = reinterpret_cast<uint32_t*>(sm + L::BITS_OFF);  // [set][half][nwords]
   DecInfo* dec = reinterpret_cast<DecInfo*>(sm + L::DEC_OFF);
@@ -359,6 +357,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     }
     fence_barrier_init();
     misc[2] = 0;
+    misc[11] = 0;
+    misc[12] = 0;
+    misc[13] = 0;
   }
   if (warp == 1) {
     tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), TMEM_COLS);
@@ -382,6 +383,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     // Q of every item and the TMA loads of its key units, walking the bitmap set
     // that the decoder warps filled (up to one item ahead).
     if (lane == 0) {
+      // TMA loads issued whose landing this thread has not seen implied yet: the
+      // last Q, and the last K / V tile of each buffer (a later load into the same
+      // buffer is only issued once the earlier one has been consumed)
+      int q_kc = -1, pk[2] = {-1, -1}, pv[2] = {-1, -1};
       for (int kc = 0;; ++kc) {
         const int s = kc & 1;
         if (!mbar_wait_ool(&bars[B_DECFULL + s], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
@@ -394,6 +399,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                                  kLoaderSuspend))
           break;
         mbar_arrive_expect_tx(&bars[B_QFULL], DS * QSLAB);
+        q_kc = kc;
         for (int c = 0; c < DS; ++c)
           tma_load_3d(sm + L::Q_OFF + c * QSLAB, &tmQ, &bars[B_QFULL], c * 64, di.qt * BM, di.h);
         // Tiles are issued in order (units, then columns, item by item): a buffer's
@@ -432,16 +438,31 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
           uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
           mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
+          pk[b] = g;
           for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, u * UNIT, di.kvh);
           if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag, kLoaderSuspend)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
+          pv[b] = g;
           for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, di.kvh);
         }
         if (!ok) break;
         mbar_arrive(&bars[B_UNITS]);  // this item's bitmaps are no longer read here
+      }
+      if (*abort_flag) {
+        // Drain this thread's loads still in flight.  The MMA thread records how
+        // far it has seen K, V and Q land; a load it has not seen may still be in
+        // flight, and no later phase of that buffer's barrier can have completed
+        // (filling the buffer again needs the load consumed first), so the parity
+        // wait is unambiguous.
+        const volatile int* vm = misc;
+        if (q_kc >= 0 && vm[13] <= q_kc) mbar_drain(&bars[B_QFULL], q_kc & 1);
+        for (int b = 0; b < 2; ++b) {
+          if (pk[b] >= 0 && vm[11] <= pk[b]) mbar_drain(&bars[B_KFULL + b], (pk[b] >> 1) & 1);
+          if (pv[b] >= 0 && vm[12] <= pv[b]) mbar_drain(&bars[B_VFULL + b], (pv[b] >> 1) & 1);
+        }
       }
     }
     __syncwarp();
@@ -466,7 +487,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int s = kc & 1;
       if (dtid == 0) {
         misc[10] = next_item;
-        next_item = (int)gridDim.x + (int)atomicAdd(a.sched, 1u);  // fetched one item ahead
+        next_item = (int)gridDim.x + sched_next(a.sched, a.epoch);  // fetched one item ahead
         misc[3] = 0;
       }
       named_barrier(1, 64);
@@ -505,19 +526,21 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       named_barrier(1, 64);
       if (dtid == 32) {
         // column lists: independent of the block lists, read in parallel with them
-        int c0 = 0, c1 = 0, cb0 = 0, cb1 = 0;
+        int ce0 = 0, ce1 = 0, cb0 = 0, cb1 = 0;
         if (live[0]) {
           const int r = h * a.nqb + qbh[0];
           cb0 = a.col_ptr[r];
-          c0 = a.col_ptr[r + 1] - cb0;
+          ce0 = a.col_ptr[r + 1];
+          checked_row(cb0, ce0, a.col_cap, a.status, DETAIL_BAD_COLPTR);
         }
         if (live[1] && !shared_qb) {
           const int r = h * a.nqb + qbh[1];
           cb1 = a.col_ptr[r];
-          c1 = a.col_ptr[r + 1] - cb1;
+          ce1 = a.col_ptr[r + 1];
+          checked_row(cb1, ce1, a.col_cap, a.status, DETAIL_BAD_COLPTR);
         }
-        dec[s].cc[0] = max(0, c0);
-        dec[s].cc[1] = max(0, c1);
+        dec[s].cc[0] = ce0 - cb0;
+        dec[s].cc[1] = ce1 - cb1;
         dec[s].cb[0] = cb0;
         dec[s].cb[1] = cb1;
       }
@@ -528,7 +551,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int qb = qbh[hh];
         const int r1 = r1h[hh];
         if (kind == DSA_KIND_VS) {
-          const int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
+          int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
+          checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
           for (int e = beg + dtid; e < end; e += 64) {
             const int delta = a.dist[e];
             if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
@@ -539,7 +563,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           }
         } else {
           const int r = h * a.nqb + qb;
-          const int beg = a.blk_ptr[r], end = a.blk_ptr[r + 1];
+          int beg = a.blk_ptr[r], end = a.blk_ptr[r + 1];
+          checked_row(beg, end, a.blk_cap, a.status, DETAIL_BAD_BLKPTR);
           for (int e = beg + dtid; e < end; e += 64) {
             const int kb = a.blk_idx[e];
             if (kb < 0 || kb >= a.nqb) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_BLOCK); continue; }
@@ -698,6 +723,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const uint64_t v_desc1 = smem_desc(smem_u32(sm + L::V_OFF + DS * KSLAB), KSLAB, 1024, SWZ_128B);
       bool ok = true;
       int tg = 0;
+      volatile int* seen = misc;  // [11] K, [12] V, [13] Q loads seen landed (for the producer's drain)
       for (int kc = 0; ok; ++kc) {
         const int slot = kc & 1;
         if (!mbar_wait_ool(&bars[B_ITEMFULL + slot], (kc >> 1) & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
@@ -705,6 +731,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         mbar_arrive(&bars[B_ITEMFREE + slot]);
         if (T < 0) break;  // no more items
         if (!mbar_wait_ool(&bars[B_QFULL], kc & 1, limit, a.status, DETAIL_WAIT_Q, abort_flag, kMmaSuspend)) break;
+        seen[13] = kc + 1;
         if (T == 0) tc_commit(&bars[B_QEMPTY]);
         for (int t = 0; t <= T; ++t) {
           if (t < T) {
@@ -713,6 +740,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int b = g & 1;
             const uint32_t use = (g >> 1) & 1;
             if (!mbar_wait_ool(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag, kMmaSuspend)) { ok = false; break; }
+            seen[11] = g + 1;
             // the buffer still holds P(g-2) until that P.V has finished; its
             // V-empty commit says so (a per-buffer barrier: at an item boundary
             // P(g-1) V(g-1) has been issued too, so B_ODONE could be two phases on)
@@ -734,6 +762,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const uint32_t use = (g >> 1) & 1;
             if (!mbar_wait_ool(&bars[B_PFULL + b], use, limit, a.status, DETAIL_WAIT_P, abort_flag, kMmaSuspend)) { ok = false; break; }
             if (!mbar_wait_ool(&bars[B_VFULL + b], use, limit, a.status, DETAIL_WAIT_V, abort_flag, kMmaSuspend)) { ok = false; break; }
+            seen[12] = g + 1;
             tc_fence_after();
             mma_pv_tile(tmem_O, tmem_base + S_COL + 64 * b, b ? v_desc1 : v_desc0, IDESC_PV, u > 0 ? 1u : 0u);
             tc_commit(&bars[B_ODONE]);
@@ -743,9 +772,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (ok && T > 0) tc_commit(&bars[B_OREADY]);  // the item's O is final once this completes
         tg += T;
       }
-      // drain every MMA this thread issued before TMEM is released
+      // drain every MMA this thread issued before TMEM is released (also after
+      // an abort: the wait ignores the abort flag)
       tc_commit(&bars[B_DRAIN]);
-      mbar_wait_ool(&bars[B_DRAIN], 0, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend);
+      mbar_drain(&bars[B_DRAIN], 0);
     }
     __syncwarp();
   } else {
@@ -875,12 +905,8 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           for (int i = 0; i < 16; ++i) {
             float x0, x1, p0, p1;
             fma2(s[k * 32 + 2 * i], s[k * 32 + 2 * i + 1], a.scale_log2, negm, x0, x1);
-            if (kPolyPeriod > 0 && i % kPolyPeriod == kPolyPeriod - 1) {
-              poly_ex2x2(x0, x1, p0, p1);  // part of the pairs on the FMA pipe
-            } else {
-              p0 = fast_ex2(x0);
-              p1 = fast_ex2(x1);
-            }
+            p0 = fast_ex2(x0);
+            p1 = fast_ex2(x1);
             add2(ls[(i & 1) * 2], ls[(i & 1) * 2 + 1], p0, p1);
             __nv_bfloat162 v2 = __floats2bfloat162_rn(p0, p1);
             pk[i] = *reinterpret_cast<uint32_t*>(&v2);
@@ -948,38 +974,35 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
   }
-  if (tid == 0) {
-    // the last CTA out zeroes the item counter for the next launch that uses it
-    __threadfence();
-    if (atomicAdd(a.sched + 1, 1u) == gridDim.x - 1) {
-      a.sched[0] = 0u;
-      a.sched[1] = 0u;
-      __threadfence();
-    }
-  }
 }
 
 // --------------------------------------------------------------------------
 // host side
 // --------------------------------------------------------------------------
-// Item counters of the persistent attention kernel: one pair per launch, taken
+// Item counters of the persistent attention kernel, one per launch taken
 // round-robin from a pool so that launches in flight on different streams do not
-// share one (up to kSchedSlots of them); each launch leaves its pair at zero.
+// share one (up to kSchedSlots of them).  Each use of a slot gets a larger epoch
+// than the one before (sched_next), so a slot needs no clearing between launches.
 constexpr int kSchedSlots = 64;
-__device__ unsigned g_sched[2 * kSchedSlots];
+__device__ unsigned long long g_sched[kSchedSlots];
 
-unsigned* sched_slot() {
+bool sched_slot(unsigned long long** slot, unsigned* epoch) {
   constexpr int kMaxDev = 64;
-  static unsigned* base[kMaxDev] = {};
-  static std::atomic<unsigned> next{0};
+  static std::atomic<unsigned long long*> base[kMaxDev] = {};
+  static std::atomic<unsigned long long> launches{0};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
-  if (base[dev] == nullptr) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return false;
+  unsigned long long* b = base[dev].load();
+  if (b == nullptr) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_sched) != cudaSuccess) return nullptr;
-    base[dev] = static_cast<unsigned*>(p);
+    if (cudaGetSymbolAddress(&p, g_sched) != cudaSuccess) return false;
+    b = static_cast<unsigned long long*>(p);
+    base[dev].store(b);  // every thread finds the same address
   }
-  return base[dev] + 2 * (next.fetch_add(1u) % kSchedSlots);
+  const unsigned long long n = launches.fetch_add(1ull);
+  *slot = b + (n % kSchedSlots);
+  *epoch = (unsigned)(n / kSchedSlots) + 1u;  // 0 is the value of a never-used slot
+  return true;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1034,6 +1057,9 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   a.dist = idx.dist;
   a.col_ptr = idx.col_ptr;
   a.col_idx = idx.col_idx;
+  a.blk_cap = idx.blk_cap;
+  a.dist_cap = idx.dist_cap;
+  a.col_cap = idx.col_cap;
   a.K = static_cast<const __nv_bfloat16*>(K);
   a.V = static_cast<const __nv_bfloat16*>(V);
   a.k_hs = p.k_head_stride;
@@ -1047,9 +1073,8 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   a.lse = lse;
   a.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   a.status = status;
-  a.sched = sched_slot();
-  if (a.sched == nullptr) return DSA_ERR_CUDA;
-  a.wait_limit_ns = kWaitLimitNs;
+  if (!sched_slot(&a.sched, &a.epoch)) return DSA_ERR_CUDA;
+  a.wait_limit_ns = wait_limit_ns();
   int smem = Smem<D>::bytes(a.nwords);
   // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;

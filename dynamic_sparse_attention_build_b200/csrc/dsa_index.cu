@@ -1263,7 +1263,8 @@ __device__ __forceinline__ int64_t ashape_pairs_in_block(int kb, int B, int r0, 
 
 __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head_info, const int32_t* blk_ptr,
                               const int32_t* blk_idx, const int32_t* dist_ptr, const int32_t* dist,
-                              const int32_t* col_ptr, const int32_t* col_idx, unsigned long long* pairs) {
+                              const int32_t* col_ptr, const int32_t* col_idx, int64_t blk_cap, int64_t dist_cap,
+                              int64_t col_cap, unsigned long long* pairs, unsigned* status) {
   pdl_prologue();
   const int qb = blockIdx.x;
   const int h = blockIdx.y;
@@ -1275,13 +1276,23 @@ __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head
   const int32_t* lst;
   int nl;
   int dsel = 0;
+  // a row is used only if 0 <= beg <= end <= cap (else reported and counted empty)
+  auto row_ok = [&](int beg, int end, int64_t cap, unsigned detail) {
+    if (0 <= beg && beg <= end && (int64_t)end <= cap) return true;
+    if (threadIdx.x == 0) report(status, DSA_ERR_DEVICE, detail);
+    return false;
+  };
   if (kind == DSA_KIND_VS) {
-    lst = dist + dist_ptr[h];
-    nl = dist_ptr[h + 1] - dist_ptr[h];
+    const int beg = dist_ptr[h], end = dist_ptr[h + 1];
+    const bool ok = row_ok(beg, end, dist_cap, DETAIL_BAD_DISTPTR);
+    lst = ok ? dist + beg : dist;
+    nl = ok ? end - beg : 0;
     dsel = 1;
   } else {
-    lst = blk_idx + blk_ptr[h * nqb + qb];
-    nl = blk_ptr[h * nqb + qb + 1] - blk_ptr[h * nqb + qb];
+    const int beg = blk_ptr[h * nqb + qb], end = blk_ptr[h * nqb + qb + 1];
+    const bool ok = row_ok(beg, end, blk_cap, DETAIL_BAD_BLKPTR);
+    lst = ok ? blk_idx + beg : blk_idx;
+    nl = ok ? end - beg : 0;
   }
   for (int e = threadIdx.x; e < nl; e += blockDim.x) {
     const int kb = dsel ? qb - lst[e] : lst[e];
@@ -1296,7 +1307,8 @@ __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head
       tot += (int64_t)nrows * (nrows + 1) / 2;
     }
   }
-  const int cb = col_ptr[h * nqb + qb], ce = col_ptr[h * nqb + qb + 1];
+  int cb = col_ptr[h * nqb + qb], ce = col_ptr[h * nqb + qb + 1];
+  if (!row_ok(cb, ce, col_cap, DETAIL_BAD_COLPTR)) cb = ce = 0;
   for (int e = cb + threadIdx.x; e < ce; e += blockDim.x) {
     const int j = col_idx[e];
     if (j < 0 || j > r1) continue;
@@ -1616,13 +1628,13 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
 
 dsa_status launch_count_pairs(const dsa_problem& p, const dsa_indices& idx, int64_t* pairs, cudaStream_t st,
                               unsigned* status) {
-  (void)status;
   const int nqb = ceil_div(p.N, p.block);
   cudaError_t e = cudaMemsetAsync(pairs, 0, sizeof(int64_t) * p.Hq, st);
   if (e != cudaSuccess) return cuda_fail(e);
   k_count_pairs<<<dim3(nqb, p.Hq), 128, 0, st>>>(p.Hq, p.N, p.block, nqb, idx.head_info, idx.blk_ptr, idx.blk_idx,
-                                                 idx.dist_ptr, idx.dist, idx.col_ptr, idx.col_idx,
-                                                 reinterpret_cast<unsigned long long*>(pairs));
+                                                 idx.dist_ptr, idx.dist, idx.col_ptr, idx.col_idx, idx.blk_cap,
+                                                 idx.dist_cap, idx.col_cap,
+                                                 reinterpret_cast<unsigned long long*>(pairs), status);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;

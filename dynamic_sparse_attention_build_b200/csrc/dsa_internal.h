@@ -9,14 +9,18 @@
 
 namespace dsa {
 
-// Device address of this device's status word (4 x uint32), or nullptr on failure.
-unsigned* status_ptr();
+// Device address of the status word (4 x uint32) that work on `stream` reports
+// into on the current device, or nullptr on failure.
+unsigned* status_ptr(cudaStream_t stream);
 
 // Records a CUDA error for dsa_last_cuda_error and returns DSA_ERR_CUDA.
 dsa_status cuda_fail(cudaError_t e);
 
 // Default bound on every in-kernel wait (ns of global time).
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
+
+// The bound that launches use now (kWaitLimitNs unless dsa_set_wait_limit changed it).
+uint64_t wait_limit_ns();
 
 dsa_status validate_problem(const dsa_problem* p);
 dsa_status validate_indices_ptrs(const dsa_indices* idx, bool for_build);

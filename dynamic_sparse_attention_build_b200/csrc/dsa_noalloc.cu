@@ -16,6 +16,8 @@
 // builder clears what it accumulates into before each use, so stale contents
 // do not matter, but two calls whose work overlaps on the GPU (different
 // streams, no ordering between them) race on the array.
+#include <atomic>
+
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -29,21 +31,24 @@ static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspa
 
 // Host code may not use g_static_workspace as a pointer: in host code that name
 // is a host-side stand-in, not a device address.  The device address is looked
-// up once per device, with that device current.
-void* g_ws_addr[kMaxDev] = {};
+// up once per device, with that device current (an atomic: host threads that make
+// their first call at the same moment store the same address).  It stays valid
+// for the life of the device's context, so the library must not be used again
+// after a cudaDeviceReset in the same process.
+std::atomic<void*> g_ws_addr[kMaxDev] = {};
 
 dsa_status static_workspace(void** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e);
   if (dev < 0 || dev >= kMaxDev) return DSA_ERR_UNSUPPORTED;
-  if (g_ws_addr[dev] == nullptr) {
-    void* p = nullptr;
+  void* p = g_ws_addr[dev].load();
+  if (p == nullptr) {
     e = cudaGetSymbolAddress(&p, g_static_workspace);
     if (e != cudaSuccess) return cuda_fail(e);
-    g_ws_addr[dev] = p;
+    g_ws_addr[dev].store(p);
   }
-  *out = g_ws_addr[dev];
+  *out = p;
   return DSA_OK;
 }
 
@@ -68,7 +73,7 @@ extern "C" dsa_status dsa_build_indices_static(const dsa_problem* p, const void*
   void* ws = nullptr;
   s = static_workspace(&ws);
   if (s != DSA_OK) return s;
-  unsigned* st = status_ptr();
+  unsigned* st = status_ptr((cudaStream_t)stream);
   if (st == nullptr) return cuda_fail(cudaGetLastError());
   return launch_build_indices(*p, Q, K, pats, *out, ws, kStaticWorkspaceBytes, (cudaStream_t)stream, st);
 }

@@ -31,8 +31,8 @@
  *   - Arguments are validated on the host before any launch; an invalid call
  *     returns an error code and enqueues nothing.  No call throws or aborts.
  *   - Errors a kernel finds (an index list longer than its capacity, an index out
- *     of range, a bounded wait that ran out) are recorded in a per-device status
- *     word and reported by dsa_get_device_status.
+ *     of range, a malformed list, a bounded wait that ran out) are recorded in the
+ *     status word of the call's stream and reported by dsa_get_device_status.
  *   - Batch size is one sequence.  Heads are independent.
  *   - Numerics: bf16 Q/K/V/O, tensor-core products with fp32 accumulation, fp32
  *     softmax and scores; P is rounded to bf16 before the P.V product.
@@ -117,7 +117,11 @@ typedef struct dsa_pattern {
 
 /*
  * Index lists, all device memory owned by the caller, sized from dsa_sizes.
- * Rows of the CSR arrays are r = h * nqb + qb.  All lists are ascending.
+ * Rows of the CSR arrays are r = h * nqb + qb.  All lists are strictly ascending
+ * (no entry repeats within one list).  dsa_sparse_prefill checks every row
+ * against the capacities (0 <= ptr[r] <= ptr[r+1] <= cap) and every entry
+ * against its range; a malformed row or entry is skipped and reported as
+ * DSA_ERR_DEVICE by dsa_get_device_status.
  *   head_info [Hq * 4]          : kind, sink, window, 0 for each head.
  *   blk_ptr   [Hq * nqb + 1]    : key blocks of (h, qb) are blk_idx[blk_ptr[r] .. blk_ptr[r+1]).
  *   blk_idx   [blk_cap]         : (empty for VS heads, whose blocks come from dist)
@@ -188,10 +192,15 @@ dsa_status dsa_sparse_prefill(const dsa_problem* p, const void* Q, const void* K
 dsa_status dsa_count_pairs(const dsa_problem* p, const dsa_indices* idx, int64_t* pairs,
                            dsa_stream stream);
 
-/* Synchronises `stream`, then returns and clears the current device's status word:
- * DSA_OK, DSA_ERR_CAPACITY, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if
- * the synchronisation itself failed).  detail (nullable) receives a kernel-specific
- * code: which list overflowed, or which wait ran out. */
+/* Synchronises `stream`, then returns and clears the status word that work
+ * enqueued on `stream` reports into on the current device: DSA_OK,
+ * DSA_ERR_CAPACITY, DSA_ERR_TIMEOUT or DSA_ERR_DEVICE (or DSA_ERR_CUDA if the
+ * synchronisation itself failed).  detail (nullable) receives a kernel-specific
+ * code: which list overflowed, which wait ran out, or which list was malformed.
+ * Each device has 64 status words; a stream's word is chosen by hashing its
+ * handle, so streams whose handles fall on the same word share it (an error of
+ * one is then reported to a caller of the other).  The first error recorded in a
+ * word is kept until this call clears it. */
 dsa_status dsa_get_device_status(dsa_stream stream, int32_t* detail);
 
 /* Self-test of the bounded-wait path: one CTA waits on a barrier that nothing
@@ -217,6 +226,14 @@ dsa_status dsa_selftest_wait_timeout(uint32_t timeout_us, dsa_stream stream);
 dsa_status dsa_build_indices_static(const dsa_problem* p, const void* Q, const void* K,
                                     const dsa_pattern* pats, const dsa_indices* out,
                                     dsa_stream stream);
+
+/* Sets the bound, in nanoseconds of GPU global time, on every in-kernel wait of
+ * the launches that follow, on every device of this process (0 restores the
+ * default of 4 s; more than 60 s is DSA_ERR_INVALID_ARG).  A wait that runs out
+ * records DSA_ERR_TIMEOUT and its CTA stops its work and exits cleanly; after a
+ * timeout the output of that launch is incomplete.  A diagnostic: a short bound
+ * makes the abort path reachable without any fault. */
+dsa_status dsa_set_wait_limit(uint64_t limit_ns);
 
 /* Static description of a status code. */
 const char* dsa_status_string(dsa_status s);

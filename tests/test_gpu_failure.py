@@ -72,3 +72,97 @@ def test_too_small_capacity_is_rejected_on_the_host(dsa):
         dsa.build_indices(Qd, Kd, pats, 64, bufs=bufs)
     assert e.value.status == B.DSA_ERR_CAPACITY
     assert dsa.device_status() == (0, 0)
+
+
+def _clone_bufs(dsa, bufs):
+    from dynamic_sparse_attention_build_b200.api import IndexBuffers
+    return IndexBuffers(Hq=bufs.Hq, N=bufs.N, block=bufs.block, nqb=bufs.nqb,
+                        head_info=bufs.head_info.clone(), blk_ptr=bufs.blk_ptr.clone(),
+                        blk_idx=bufs.blk_idx.clone(), dist_ptr=bufs.dist_ptr.clone(), dist=bufs.dist.clone(),
+                        col_ptr=bufs.col_ptr.clone(), col_idx=bufs.col_idx.clone(),
+                        vert_idx=bufs.vert_idx.clone(), slash_idx=bufs.slash_idx.clone())
+
+
+@pytest.mark.parametrize("which", ["blk_past_cap", "blk_negative", "col_past_cap", "col_reversed", "dist_past_cap"])
+def test_malformed_rows_are_reported_and_skipped(dsa, which):
+    """A CSR row whose pointers leave [0, cap] (or run backwards) is reported as
+    DSA_ERR_DEVICE with the list's detail code and treated as empty, by the
+    attention kernel and by the pair count; the kernel never reads outside the
+    arrays, and every other row is computed as with well-formed lists."""
+    from dynamic_sparse_attention_build_b200 import _binding as B
+    N, d, Bk = 700, 64, 64
+    nqb = (N + Bk - 1) // Bk
+    Q, K, V = synth.random_qkv(2, 1, N, d, seed=5)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    pats = [dict(kind="block_topk", topk=3), dict(kind="vs", last_q=16, n_vert=40, n_slash=6)]
+    good = dsa.build_indices(Qd, Kd, pats, Bk)
+    O_good, _ = dsa.sparse_prefill(Qd, Kd, Vd, good)
+    pairs_good = dsa.count_pairs(Qd, Kd, good)
+    assert dsa.device_status() == (0, 0)
+    bad = _clone_bufs(dsa, good)
+    cap_b, cap_c, cap_d = bad.blk_idx.numel(), bad.col_idx.numel(), bad.dist.numel()
+    h, qb = (0, 4) if which.startswith("blk") else (1, 6)
+    r = h * nqb + qb
+    if which == "blk_past_cap":
+        bad.blk_ptr[r + 1] = cap_b + 1000       # rows qb and qb + 1 of head 0
+        detail, rows = 33, [(0, qb), (0, qb + 1)]
+    elif which == "blk_negative":
+        bad.blk_ptr[r] = -5                       # rows qb - 1 and qb of head 0
+        detail, rows = 33, [(0, qb - 1), (0, qb)]
+    elif which == "col_past_cap":
+        bad.col_ptr[r + 1] = cap_c + 7
+        detail, rows = 34, [(1, qb), (1, qb + 1)]
+    elif which == "col_reversed":
+        bad.col_ptr[r + 1] = int(bad.col_ptr[r]) - 1   # end before begin
+        detail, rows = 34, [(1, qb), (1, qb + 1)]
+    else:
+        bad.dist_ptr[2] = cap_d + 5               # head 1's distance list
+        detail, rows = 35, [(1, q) for q in range(nqb)]
+    bad.__post_init__()
+    O_bad, _ = dsa.sparse_prefill(Qd, Kd, Vd, bad)
+    status, det = dsa.device_status()
+    assert status == B.DSA_ERR_DEVICE and det == detail, (status, det)
+    pairs_bad = dsa.count_pairs(Qd, Kd, bad)
+    status, det = dsa.device_status()
+    assert status == B.DSA_ERR_DEVICE and det == detail, (status, det)
+    assert dsa.device_status() == (0, 0)
+    skipped = np.zeros((2, N), bool)
+    for hh, q in rows:
+        skipped[hh, q * Bk:min(N, q * Bk + Bk)] = True
+    keep = torch.from_numpy(~skipped)
+    assert torch.equal(O_bad.cpu()[keep], O_good.cpu()[keep])
+    assert torch.isfinite(O_bad.float()).all()
+    assert int(pairs_bad[1 - rows[0][0]]) == int(pairs_good[1 - rows[0][0]])
+    if which != "col_reversed":  # there the next row reads one column of this one
+        assert int(pairs_bad[rows[0][0]]) < int(pairs_good[rows[0][0]])
+
+
+def test_abort_with_loads_in_flight_leaves_the_next_launch_exact(dsa):
+    """With a wait bound of a few microseconds some wait of the attention kernel
+    runs out while its CTA still has TMA loads and MMAs in flight; the CTA then
+    drains them, frees its tensor memory and exits, the launch reports
+    DSA_ERR_TIMEOUT, and the next launch with the default bound is bit-identical
+    to a clean run."""
+    from dynamic_sparse_attention_build_b200 import _binding as B
+    w = synth.workload(2, N=8192, Hq=8, Hkv=2)
+    Q, K, V, _ = synth.make_inputs(w, device="cuda")
+    pats = synth.head_patterns(w)
+    idx = dsa.build_indices(Q, K, pats, w["B"])
+    O_ref, lse_ref = dsa.sparse_prefill(Q, K, V, idx, want_lse=True)
+    assert dsa.device_status() == (0, 0)
+    timeouts = 0
+    try:
+        for limit_ns in (300, 1000, 3000, 10000, 30000):
+            assert B.dsa_set_wait_limit(limit_ns) == B.DSA_OK
+            for _ in range(2):
+                dsa.sparse_prefill(Q, K, V, idx)
+                status, det = dsa.device_status()
+                assert status in (B.DSA_OK, B.DSA_ERR_TIMEOUT), (limit_ns, status, det)
+                timeouts += status == B.DSA_ERR_TIMEOUT
+    finally:
+        assert B.dsa_set_wait_limit(0) == B.DSA_OK
+    assert timeouts > 0, "no wait ran out: the abort path was not reached"
+    O, lse = dsa.sparse_prefill(Q, K, V, idx, want_lse=True)
+    assert dsa.device_status() == (0, 0)
+    assert torch.equal(O, O_ref) and torch.equal(lse, lse_ref)
+    assert B.dsa_set_wait_limit(61 * 10**9) == B.DSA_ERR_INVALID_ARG

@@ -35,6 +35,6 @@ def test_host_prefill_equals_device_path(dsa, chunks):
         Oh = torch.empty_like(Q).pin_memory()
         hp.run(Qh, Kh, Vh, Oh)
         torch.cuda.current_stream().synchronize()
-        st, det = dsa.device_status()
+        st, det = hp.status()
         assert st == 0, (st, det)
         assert torch.equal(Oh, O_ref.cpu())

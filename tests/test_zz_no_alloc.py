@@ -5,9 +5,11 @@ scratch is a fixed buffer inside the library, so the caller passes only inputs
 and output index arrays.
 
 Checked through the C ABI against the regular dsa_build_indices on the same
-inputs, on two calls in a row (the shared buffer keeps the previous call's
-contents, which must not leak into the next result), plus the attention output
-built from those indices.  Kept in a file of its own so that it runs last."""
+inputs, on two calls in a row, after a call on an unrelated problem (another
+seed, length and set of patterns) has left its own data in the shared buffer:
+the buffer keeps the previous call's contents, which must not leak into the
+next result.  The attention output built from those indices is checked too.
+Kept in a file of its own so that it runs last."""
 import ctypes
 
 import numpy as np
@@ -54,9 +56,13 @@ def same_indices(a, b, Q, K, N, B):
         v, s = orc.vs_estimate(to64(Q[h]), to64(K[h // G]), PATS[h]["last_q"])
         assert topk_set_ok(x["vert"], y["vert"], v, PATS[h]["n_vert"])[0]
         assert topk_set_ok(x["slash"], y["slash"], s, PATS[h]["n_slash"])[0]
+        nqb = (N + B - 1) // B
         for z in (x, y):
-            D = orc.vs_distance_set(np.asarray(z["slash"], np.int64), B, (N + B - 1) // B)
+            D = orc.vs_distance_set(np.asarray(z["slash"], np.int64), B, nqb)
             assert np.array_equal(z["dist"], D)
+            vert = np.asarray(z["vert"], np.int64)
+            for qb in range(nqb):
+                assert np.array_equal(z["cols"][qb], orc.vs_columns(vert, D, qb, B)), (h, qb)
 
 
 def test_static_workspace_matches_regular_builder(dsa):
@@ -71,6 +77,21 @@ def test_static_workspace_matches_regular_builder(dsa):
     O_ref, _ = dsa.sparse_prefill(Qd, Kd, Vd, ref)
     prob = make_problem(Qd, Kd, block=B)
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    # an unrelated problem first, so the shared buffer holds other data (other
+    # maxima, bitmaps, sums and counts) when the checked calls start
+    N2 = 5000
+    Q2, K2, _ = synth.random_qkv(8, 4, N2, d, seed=97)
+    Q2d, K2d = Q2.cuda() * 3, K2.cuda()
+    pats2 = make_patterns([dict(kind="moba", topk=9), dict(kind="vs", last_q=128, n_vert=700, n_slash=900),
+                           dict(kind="block_threshold", alpha=0.2, keep_sink=1, keep_local=1),
+                           dict(kind="block_topk", topk=40)] * 2)
+    prob2 = make_problem(Q2d, K2d, block=B)
+    out2 = alloc_indices(prob2, pats2, "cuda")
+    st = Bi.dsa_build_indices_static(prob2, ctypes.c_void_p(Q2d.data_ptr()), ctypes.c_void_p(K2d.data_ptr()),
+                                     pats2, out2.c, stream)
+    assert st == Bi.DSA_OK, Bi.dsa_status_string(st)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == (0, 0)
     for call in range(2):
         out = alloc_indices(prob, pats_c, "cuda")  # outputs belong to the caller
         out.workspace = None
