@@ -425,3 +425,35 @@ def selected_pairs(hi: HeadIndex) -> int:
     for i in range(hi.N):
         total += allowed_keys(hi, i).size
     return total
+
+
+def selected_pairs_by_block(hi: HeadIndex) -> int:
+    """|M| of one head counted one query block at a time (fast enough for
+    full-length layers).  The keys a query block lists (its blocks' keys, its
+    slash runs and its columns, as a set) are the same for every row of the
+    block; row i keeps those with j <= i, found by a binary search in the sorted
+    set, and for A-shape heads only those with j < sink or i - j < window
+    ([MI] "3つの疎パターン": sink tokens plus a local window), counted as
+    |{j < sink}| + |{j > i - window}| - |{both}| among the keys j <= i."""
+    B, N = hi.B, hi.N
+    total = 0
+    for qb in range(n_blocks(N, B)):
+        blk = np.asarray(hi.blocks[qb], dtype=np.int64)
+        parts = [(blk[:, None] * B + np.arange(B)[None, :]).ravel(), np.asarray(hi.cols[qb], dtype=np.int64)]
+        if hi.runs is not None and hi.runs[qb].size:
+            parts += [np.arange(a, b + 1) for a, b in hi.runs[qb]]
+        keys = np.unique(np.concatenate(parts))
+        keys = keys[keys < N]
+        rows = np.arange(qb * B, min(N, qb * B + B), dtype=np.int64)
+        upto_i = np.searchsorted(keys, rows, side="right")          # keys j <= i
+        if hi.kind != ASHAPE:
+            total += int(upto_i.sum())
+            continue
+        sink_n = np.searchsorted(keys, np.minimum(rows + 1, hi.sink), side="left")   # j <= i, j < sink
+        win_lo = rows - hi.window + 1                                               # window: j >= i - window + 1
+        win_n = upto_i - np.searchsorted(keys, win_lo, side="left")
+        both_hi = np.minimum(rows + 1, hi.sink)                                      # j < min(i + 1, sink)
+        both_n = (np.searchsorted(keys, both_hi, side="left")                         # ... and j >= i - window + 1
+                  - np.searchsorted(keys, np.minimum(win_lo, both_hi), side="left"))
+        total += int((sink_n + win_n - both_n).sum())
+    return total

@@ -73,6 +73,12 @@ MUTANTS = [
      "        if J.size == 0:\n            J = np.array([i])", ATT),
     ("pair count off by one", "total += allowed_keys(hi, i).size",
      "total += allowed_keys(hi, i).size + (1 if i == 0 else 0)", "pairs"),
+    ("block pair count excludes the diagonal key", 'upto_i = np.searchsorted(keys, rows, side="right")',
+     'upto_i = np.searchsorted(keys, rows, side="left")', "pairs_by_block"),
+    ("block pair count adds the sink twice", "total += int((sink_n + win_n - both_n).sum())",
+     "total += int((sink_n + win_n).sum())", "pairs_by_block"),
+    ("block pair count window one short", "win_lo = rows - hi.window + 1", "win_lo = rows - hi.window + 2",
+     "pairs_by_block"),
     ("slash runs: touching windows not merged", "if runs and a <= runs[-1][1] + 1:",
      "if runs and a <= runs[-1][1]:", RUNS),
     ("slash runs: window end from r0 + B", "a, b = max(0, r0 - o), r1 - o", "a, b = max(0, r0 - o), r0 + B - 1 - o",

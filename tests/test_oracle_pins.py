@@ -406,3 +406,28 @@ def test_empty_rows_and_duplicates():
 def test_selected_pairs_counts_mask(rng):
     hi = _vs_head(rng, 48, 4, 8, 5, 3, 4)
     assert orc.selected_pairs(hi) == int(orc.index_mask_dense(hi).sum())
+
+
+@pytest.mark.parametrize("N,B", [(200, 16), (131, 8), (64, 64), (97, 32)])
+def test_selected_pairs_by_block_equals_the_mask_count(rng, N, B):
+    """The block-wise count (one sorted key set per query block, binary search
+    per row, the A-shape predicate by inclusion-exclusion) equals the number of
+    True entries of the dense index mask, for every pattern kind, slash runs
+    and columns that repeat keys of listed blocks included."""
+    d = 8
+    Q = rng.standard_normal((N, d))
+    K = rng.standard_normal((N, d))
+    pats = [dict(kind="ashape", sink=5, window=11), dict(kind="ashape", sink=0, window=1),
+            dict(kind="ashape", sink=N, window=3), dict(kind="ashape", sink=2 * B + 3, window=B + 1),
+            dict(kind="vs", last_q=16, n_vert=9, n_slash=7),
+            dict(kind="vs", last_q=16, n_vert=9, n_slash=7, slash_cover="windows"),
+            dict(kind="block_topk", topk=3), dict(kind="block_threshold", alpha=0.4),
+            dict(kind="moba", topk=2)]
+    for p in pats:
+        hi = orc.build_head_index(Q, K, p, B)
+        if p["kind"] == "block_topk":  # columns inside listed blocks must count once
+            hi.cols = [np.sort(rng.choice(min(N, qb * B + B), size=min(5, qb * B + B), replace=False))
+                       for qb in range(len(hi.blocks))]
+        want = int(orc.index_mask_dense(hi).sum())
+        assert orc.selected_pairs_by_block(hi) == want, p
+        assert orc.selected_pairs(hi) == want, p
