@@ -171,12 +171,18 @@ def kernel_launches_per_step(pats):
 
 
 # --------------------------------------------------------------------------- oracle timing
-def oracle_sample(w, Q, K, V, pats, target_s=15.0):
-    """Times the CPU oracle on a bounded sample of the layer and extrapolates to
-    the whole layer.  Sample: the full index build of one head of each pattern
-    kind present, and the attention of evenly spaced rows of those heads (time per
-    row scales with the row's allowed keys, so rows are spread over the sequence).
-    Returns (estimated layer seconds, description, threads)."""
+ORACLE_SAMPLE_ROWS = 512
+
+
+def oracle_sample(w, Q, K, V, pats, rows_per_kind=ORACLE_SAMPLE_ROWS):
+    """Times the CPU oracle on one fixed, bounded sample of the layer and
+    extrapolates to the whole layer.  The sample: the full index build of one
+    head of each pattern kind present, and the attention of `rows_per_kind`
+    evenly spaced rows of those heads (a row's cost grows with its allowed keys,
+    so the rows are spread over the sequence).  Layer estimate = index time x
+    heads of that kind + attention time per row x N x heads of that kind.  The
+    CPU-baseline leg and the reference arm both use this same sample.
+    Returns (estimated layer seconds, description, threads, seconds spent)."""
     from oracle import dsa_oracle as orc
     N, B, G = w["N"], w["B"], w["Hq"] // w["Hkv"]
     q = Q.to("cpu", torch.float64).numpy()
@@ -185,11 +191,8 @@ def oracle_sample(w, Q, K, V, pats, target_s=15.0):
     by_kind = {}
     for h, p in enumerate(pats):
         by_kind.setdefault(p["kind"], []).append(h)
-    est = 0.0
-    parts = []
-    budget_rows = 0
-    t_idx = {}
-    heads = {}
+    rows = np.unique(np.linspace(0, N - 1, min(N, rows_per_kind)).astype(np.int64))
+    est = spent = 0.0
     for kind, hs in by_kind.items():
         h = hs[0]
         conv = None
@@ -198,32 +201,27 @@ def oracle_sample(w, Q, K, V, pats, target_s=15.0):
             cw, cb = p.pop("conv")
             conv = (cw.double().cpu().numpy(), cb.double().cpu().numpy())
         t0 = time.perf_counter()
-        heads[kind] = orc.build_head_index(q[h], k[h // G], p, B, conv)
-        t_idx[kind] = time.perf_counter() - t0
-        est += t_idx[kind] * len(hs)
-    # attention: rows spread over the sequence, grown until the budget is used
-    t_att = {}
-    n_rows = 8
-    spent = sum(t_idx.values())
-    while True:
-        rows = np.unique(np.linspace(0, N - 1, n_rows).astype(np.int64))
-        t_att = {}
-        for kind, hs in by_kind.items():
-            h = hs[0]
-            t0 = time.perf_counter()
-            orc.attention_rows(q[h], k[h // G], v[h // G], heads[kind], rows)
-            t_att[kind] = time.perf_counter() - t0
-        spent += sum(t_att.values())
-        if spent > target_s or n_rows >= N:
-            break
-        n_rows *= 2
-    for kind, hs in by_kind.items():
-        est += t_att[kind] / rows.size * N * len(hs)
-    budget_rows = rows.size
+        hi = orc.build_head_index(q[h], k[h // G], p, B, conv)
+        t1 = time.perf_counter()
+        orc.attention_rows(q[h], k[h // G], v[h // G], hi, rows)
+        t2 = time.perf_counter()
+        est += (t1 - t0) * len(hs) + (t2 - t1) / rows.size * N * len(hs)
+        spent += t2 - t0
     desc = (f"full index build of one head per pattern kind ({', '.join(sorted(by_kind))}) and attention of "
-            f"{budget_rows} evenly spaced rows of each; extrapolated to {w['Hq']} heads x {N} rows")
+            f"{rows.size} evenly spaced rows of each; extrapolated to {w['Hq']} heads x {N} rows")
     threads = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
     return est, desc, threads, spent
+
+
+def oracle_baseline(w, Q, K, V, pats, min_seconds=10.0):
+    """The sample of oracle_sample repeated until at least `min_seconds` of CPU
+    work are spent; the mean layer estimate."""
+    ests, spent = [], 0.0
+    while spent < min_seconds or not ests:
+        est, desc, threads, s = oracle_sample(w, Q, K, V, pats)
+        ests.append(est)
+        spent += s
+    return statistics.mean(ests), desc + f" ({len(ests)} repetitions, {spent:.1f} s of CPU work)", threads
 
 
 # --------------------------------------------------------------------------- main
@@ -274,23 +272,26 @@ def main():
             return
         torch.manual_seed(0)
         Q, K, V, pats = build_workload(w, "cuda" if torch.cuda.is_available() else "cpu")
-        per_step = min(15.0, max(2.0, 150.0 / max(1, args.steps + args.warmup)))
         for _ in range(args.warmup):
-            oracle_sample(w, Q, K, V, pats, target_s=1.0)
-        times = []
+            oracle_sample(w, Q, K, V, pats)
+        times, spent = [], 0.0
         desc = threads = None
         for _ in range(args.steps):
-            est, desc, threads, spent = oracle_sample(w, Q, K, V, pats, target_s=per_step)
+            est, desc, threads, s = oracle_sample(w, Q, K, V, pats)
             times.append(est)
+            spent += s
         t = statistics.mean(times)
         val = w["N"] / t
         line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "tokens/s", "n_gpus": args.gpus,
-                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3,
+                "ms_per_step_kind": (f"extrapolated: each step times the oracle on one fixed sample "
+                                     f"({spent / max(1, args.steps):.2f} s of CPU work) and scales it to the layer"),
+                "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
                 "config": {"workload": w["name"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
                            "block": w["B"]},
                 "cpu_baseline": {"value": val, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                 "sample": desc},
+                                 "sample": desc + f" (one sample per step, {args.steps} steps)"},
                 "e2e": {"value": val, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
         return
@@ -437,9 +438,9 @@ def main():
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, desc, threads, spent = oracle_sample(w, Q, K, V, pats)
+        est, desc, threads = oracle_baseline(w, Q, K, V, pats)
         line["cpu_baseline"] = {"value": N / est, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                                "sample": desc + f" ({spent:.1f} s of CPU work)"}
+                                "sample": desc}
     if rank == 0:
         print(json.dumps(line))
     if world > 1:

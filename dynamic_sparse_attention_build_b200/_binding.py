@@ -25,9 +25,11 @@ DSA_KIND_VS = 1
 DSA_KIND_BLOCK_TOPK = 2
 DSA_KIND_BLOCK_THRESHOLD = 3
 DSA_KIND_MOBA = 4
+DSA_KIND_UNIFIED = 5
 
 KIND_CODES = {"ashape": DSA_KIND_ASHAPE, "vs": DSA_KIND_VS, "block_topk": DSA_KIND_BLOCK_TOPK,
-              "block_threshold": DSA_KIND_BLOCK_THRESHOLD, "moba": DSA_KIND_MOBA}
+              "block_threshold": DSA_KIND_BLOCK_THRESHOLD, "moba": DSA_KIND_MOBA,
+              "unified": DSA_KIND_UNIFIED}
 
 EXPORTS = ("dsa_workspace_size", "dsa_build_indices", "dsa_sparse_prefill", "dsa_count_pairs",
            "dsa_get_device_status", "dsa_selftest_wait_timeout", "dsa_status_string",

@@ -287,25 +287,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* v) {
 // restarts the count at its own epoch: one CTA's compare-and-swap succeeds and
 // takes item 0, the others see the new epoch and count on from it.  So no launch
 // has to clear the word when it ends, and the common case is one atomic add.
-__device__ __forceinline__ int sched_next(unsigned long long* ctr, unsigned epoch) {
+static __device__ __noinline__ int sched_restart(unsigned long long* ctr, unsigned epoch, unsigned long long old) {
   while (true) {
-    const unsigned long long old = atomicAdd(ctr, 1ull);
-    if ((unsigned)(old >> 32) == epoch) return (int)(unsigned)(old & 0xffffffffull);
     unsigned long long cur = old + 1ull;
     while ((unsigned)(cur >> 32) != epoch) {
       const unsigned long long prev = atomicCAS(ctr, cur, ((unsigned long long)epoch << 32) | 1ull);
       if (prev == cur) return 0;
       cur = prev;
     }
+    old = atomicAdd(ctr, 1ull);
+    if ((unsigned)(old >> 32) == epoch) return (int)(unsigned)(old & 0xffffffffull);
   }
+}
+__device__ __forceinline__ int sched_next(unsigned long long* ctr, unsigned epoch) {
+  const unsigned long long old = atomicAdd(ctr, 1ull);
+  if ((unsigned)(old >> 32) == epoch) return (int)(unsigned)(old & 0xffffffffull);
+  return sched_restart(ctr, epoch, old);  // out of line: once per launch and CTA at most
 }
 
 // A CSR row [beg, end) is usable only if 0 <= beg <= end <= cap; otherwise the
 // row is reported (DSA_ERR_DEVICE, `detail`) and treated as empty, so a
 // malformed list never makes the kernel read outside the caller's arrays.
+static __device__ __noinline__ void report_bad_row(unsigned* status, unsigned detail) {
+  report(status, DSA_ERR_DEVICE, detail);
+}
 __device__ __forceinline__ void checked_row(int& beg, int& end, int64_t cap, unsigned* status, unsigned detail) {
   if (!(0 <= beg && beg <= end && (int64_t)end <= cap)) {
-    report(status, DSA_ERR_DEVICE, detail);
+    report_bad_row(status, detail);
     beg = 0;
     end = 0;
   }
@@ -319,6 +327,22 @@ static __device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
+
+// After an abort, the producer drains its loads still in flight.  The MMA
+// thread records how far it has seen K, V and Q land (misc[11], [12], [13]); a
+// load it has not seen may still be in flight, and no later phase of that
+// buffer's barrier can have completed (filling the buffer again needs the load
+// consumed first), so the parity wait is unambiguous.
+static __device__ __noinline__ void drain_loads(uint64_t* bars, const int* misc, int q_kc, int pk0, int pk1,
+                                                int pv0, int pv1) {
+  const volatile int* vm = misc;
+  if (q_kc >= 0 && vm[13] <= q_kc) mbar_drain(&bars[B_QFULL], q_kc & 1);
+  const int pk[2] = {pk0, pk1}, pv[2] = {pv0, pv1};
+  for (int b = 0; b < 2; ++b) {
+    if (pk[b] >= 0 && vm[11] <= pk[b]) mbar_drain(&bars[B_KFULL + b], (pk[b] >> 1) & 1);
+    if (pv[b] >= 0 && vm[12] <= pv[b]) mbar_drain(&bars[B_VFULL + b], (pv[b] >> 1) & 1);
   }
 }
 
@@ -451,19 +475,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         if (!ok) break;
         mbar_arrive(&bars[B_UNITS]);  // this item's bitmaps are no longer read here
       }
-      if (*abort_flag) {
-        // Drain this thread's loads still in flight.  The MMA thread records how
-        // far it has seen K, V and Q land; a load it has not seen may still be in
-        // flight, and no later phase of that buffer's barrier can have completed
-        // (filling the buffer again needs the load consumed first), so the parity
-        // wait is unambiguous.
-        const volatile int* vm = misc;
-        if (q_kc >= 0 && vm[13] <= q_kc) mbar_drain(&bars[B_QFULL], q_kc & 1);
-        for (int b = 0; b < 2; ++b) {
-          if (pk[b] >= 0 && vm[11] <= pk[b]) mbar_drain(&bars[B_KFULL + b], (pk[b] >> 1) & 1);
-          if (pv[b] >= 0 && vm[12] <= pv[b]) mbar_drain(&bars[B_VFULL + b], (pv[b] >> 1) & 1);
-        }
-      }
+      if (*abort_flag) drain_loads(bars, misc, q_kc, pk[0], pk[1], pv[0], pv[1]);
     }
     __syncwarp();
   } else if (warp == 2 || warp == 3) {
@@ -509,6 +521,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int h = item % a.Hq;
       const int qt = a.n_qtiles - 1 - item / a.Hq;
       const int row0 = qt * BM;
+      // The item's Q tile is read from HBM once, by the producer, when the item
+      // before it has finished its last Q K^T; fetching it into L2 now (about
+      // one item ahead) takes the HBM latency off that hand-over.
+      if (dtid == 0)
+        for (int c = 0; c < DS; ++c) tma_prefetch_l2_3d(&tmQ, c * 64, row0, h);
       const int kind = a.head_info[h * 4 + 0];
       uint32_t* b0 = bits + s * 2 * a.nwords;
       uint32_t* b1 = b0 + a.nwords;
@@ -1095,6 +1112,11 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
 }
 
 }  // namespace
+
+bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int N, int H, int64_t ts, int64_t hs,
+                          int box_rows) {
+  return make_map(map, base, d, N, H, ts, hs, box_rows);
+}
 
 dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K, const void* V,
                               const dsa_indices& idx, void* O, float* lse, cudaStream_t stream, unsigned* status) {

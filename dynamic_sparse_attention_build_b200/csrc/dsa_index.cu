@@ -54,6 +54,8 @@ struct HeadTab {
   int keep_sink[MAXH];
   int keep_local[MAXH];
   int bslot[MAXH];  // slot among block-kind heads, -1 otherwise
+  int uslot[MAXH];  // slot among unified-discovery heads, -1 otherwise
+  int uhead[MAXH];  // q-head of unified slot s
   int vslot[MAXH];  // slot among VS heads, -1 otherwise
   int bhead[MAXH];  // q-head of block slot s
   int vhead[MAXH];  // q-head of VS slot s
@@ -67,8 +69,8 @@ struct ConvTab {
 };
 
 struct Layout {
-  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_chunk, vs_nchunks, vs_lmax;
-  int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, off_spart, total;
+  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_chunk, vs_nchunks, vs_lmax, nuh, sel_ri, sel_nx;
+  int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, off_spart, off_upart, total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
@@ -273,15 +275,26 @@ __global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int
 // Causal depthwise key conv (width W, SiLU, residual) summed over a contiguous
 // run of rows [r0, r1) for this thread's 8 channels: weights in registers, the
 // last W rows in a register window, one 16-byte load per row (four in flight).
+__device__ __forceinline__ float tanh_approx(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Sum over rows r0 <= r < r1 of k_r + SiLU(conv_r) for 8 channels, where
+// conv_r = b + sum_t w_t k_{r - t}.  SiLU(c) = c sigmoid(c) = h + h tanh(h) with
+// h = c / 2 (sigmoid(c) = (1 + tanh(c / 2)) / 2): one tanh.approx (relative error
+// about 2^-11, far below what routing on pooled keys can see) instead of an
+// exponential and a division; the halving is folded into the weights and bias.
 template <int W>
 __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts, int c0, int r0, int r1,
                                               const float* cw, const float* cb, float* acc) {
   float wt[W][8], bias[8], win[W][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    bias[i] = cb[c0 + i];
+    bias[i] = 0.5f * cb[c0 + i];
 #pragma unroll
-    for (int t = 0; t < W; ++t) wt[t][i] = cw[(c0 + i) * W + t];
+    for (int t = 0; t < W; ++t) wt[t][i] = 0.5f * cw[(c0 + i) * W + t];
   }
   // before row r is shifted in, win[t] = k[r - 1 - t] (t < W - 1); after the
   // shift win[t] = k[r - t].  Rows before 0 are zero (causal, zero padded).
@@ -313,10 +326,10 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
       for (int i = 0; i < 8; ++i) win[0][i] = __bfloat162float(e[i]);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        float c = bias[i];
+        float h = bias[i];
 #pragma unroll
-        for (int t = 0; t < W; ++t) c = fmaf(wt[t][i], win[t][i], c);
-        acc[i] += win[0][i] + __fdividef(c, 1.f + __expf(-c));
+        for (int t = 0; t < W; ++t) h = fmaf(wt[t][i], win[t][i], h);
+        acc[i] += win[0][i] + fmaf(h, tanh_approx(h), h);
       }
     }
   }
@@ -642,7 +655,32 @@ __global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__
     uint32_t* sel = reinterpret_cast<uint32_t*>(ws + L.off_sel) + ((int64_t)slot * L.nqb + I) * L.nkw;
     const int ncand = (kind == DSA_KIND_MOBA) ? I : I + 1;
     int count = 0;
-    if (kind == DSA_KIND_BLOCK_THRESHOLD) {
+    if (kind == DSA_KIND_UNIFIED) {
+      // row-normalised weights P_IJ = exp(s_IJ - max) / sum, written over the
+      // row's scores for the CTA's column and diagonal sums below; the row's own
+      // blocks are those with s_IJ >= max + ln(alpha) (the threshold rule)
+      float mx = -INFINITY;
+      for (int J = lane; J < ncand; J += 32) mx = fmaxf(mx, row[J]);
+      mx = warp_max(mx);
+      float sum = 0.f;
+      for (int J = lane; J < ncand; J += 32) sum += __expf(row[J] - mx);
+      sum = warp_sum(sum);
+      const float thr = mx + ht.lnalpha[h];
+      const float inv = 1.f / sum;
+      float* prow = sc + rr * SEL_RS(npad);
+      for (int w0 = 0; w0 <= (I >> 5); ++w0) {
+        const int J = w0 * 32 + lane;
+        bool keep = J < ncand && row[J] >= thr;
+        if (J == 0 && ht.keep_sink[h]) keep = true;
+        if (J == I && ht.keep_local[h]) keep = true;
+        const float pj = J < ncand ? __expf(row[J] - mx) * inv : 0.f;
+        __syncwarp();
+        prow[J] = pj;
+        const unsigned bits = __ballot_sync(0xffffffffu, keep);
+        if (lane == 0) sel[w0] = bits;
+        count += __popc(bits);
+      }
+    } else if (kind == DSA_KIND_BLOCK_THRESHOLD) {
       float mx = -INFINITY;
       for (int J = lane; J < ncand; J += 32) mx = fmaxf(mx, row[J]);
       mx = warp_max(mx);
@@ -686,251 +724,515 @@ __global__ void __launch_bounds__(SEL_NT) k_block_select(const __grid_constant__
     }
     if (lane == 0) blk_ptr[1 + h * L.nqb + I] = count;
   }
+  if (kind == DSA_KIND_UNIFIED) {
+    // this CTA's share of the vertical sums V_J = sum_I P_IJ and diagonal sums
+    // G_d = sum_I P_{I, I-d}, over its rows in ascending order (k_unified_merge
+    // adds the CTAs' shares in ascending order: the same sums on every run)
+    __syncthreads();
+    float* up = reinterpret_cast<float*>(ws + L.off_upart) +
+                ((int64_t)ht.uslot[h] * L.sel_nx + blockIdx.x) * 2 * L.nqb;
+    for (int x = tid; x < L.nqb; x += SEL_NT) {
+      float v = 0.f, gd = 0.f;
+      for (int rr = 0; rr < nI; ++rr) {
+        const int I = I0 + rr;
+        if (x <= I) {
+          v += sc[rr * SEL_RS(npad) + x];
+          gd += sc[rr * SEL_RS(npad) + (I - x)];
+        }
+      }
+      up[x] = v;
+      up[L.nqb + x] = gd;
+    }
+  }
 }
 
-// ---------------------------------------------------------------------------
-// VS estimate: logits of the last Lq rows against one chunk of keys, bf16
-// mma.sync m16n8k16 with fp32 accumulate, in log2 units (x = tau log2(e) q.k,
-// so every exponential is one ex2).
-//   PASS 1: per-row max and sum of 2^(x - max) over the chunk -> partials
-//   PASS 2: p = 2^(x - m_i) / l_i into a shared fp32 tile; v[j] (column sums,
-//           owned by this CTA) and s[o] (diagonal sums: one thread per offset
-//           over the rows that offset meets, global atomics at the chunk edges)
-// K sub-tiles arrive by cp.async (zero-filled past the end) into one buffer,
-// refilled as soon as the sub-tile's MMAs have read it, so the next load
-// overlaps the exponentials and the sums.
-// Rows padded to LP = 16 * RT; warps: RT row tiles x (8 / RT) key groups.
-// ---------------------------------------------------------------------------
-// 16 bytes global -> shared, asynchronously; src_bytes = 0 writes zeros
-__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem_dst)), "l"(gsrc),
-               "r"(src_bytes)
-               : "memory");
+__device__ __forceinline__ uint32_t low_mask_upto(int n) {  // bits 0..n (n in 0..31)
+  return n >= 31 ? 0xffffffffu : ((2u << n) - 1u);
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+
+// Unified discovery, per head: adds the CTAs' shares of the vertical and
+// diagonal sums (ascending CTA order), keeps the verticals V_J >= alpha max V
+// and diagonals G_d >= alpha max G, and adds to every query block's selection
+// the verticals J <= I and the blocks I - d of the diagonals d <= I; the row
+// counts are rewritten.  The kept verticals and diagonals are also written,
+// ascending and -1 padded, to the vertical / slash lists of the head.
+__global__ void __launch_bounds__(1024) k_unified_merge(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
+                                                        int32_t* blk_ptr, int32_t* vert_idx, int vert_stride,
+                                                        int32_t* slash_idx, int slash_stride) {
+  pdl_prologue();
+  extern __shared__ float um[];  // V[nqb], G[nqb], then the kept bitmaps as words
+  const int uslot = blockIdx.x;
+  const int h = ht.uhead[uslot];
+  const int nqb = L.nqb;
+  float* V = um;
+  float* G = um + nqb;
+  uint32_t* vb = reinterpret_cast<uint32_t*>(um + 2 * nqb);  // [nkw] vertical bits
+  uint32_t* db = vb + L.nkw;                                  // [nkw] diagonal bits
+  __shared__ float red[2][32];
+  __shared__ int cnt[2][32];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const float* up = reinterpret_cast<const float*>(ws + L.off_upart) + (int64_t)uslot * L.sel_nx * 2 * nqb;
+  float mv = 0.f, mg = 0.f;
+  for (int x = tid; x < nqb; x += blockDim.x) {
+    float v = 0.f, gd = 0.f;
+    for (int c = 0; c < L.sel_nx; ++c) {
+      v += up[(int64_t)c * 2 * nqb + x];
+      gd += up[(int64_t)c * 2 * nqb + nqb + x];
+    }
+    V[x] = v;
+    G[x] = gd;
+    mv = fmaxf(mv, v);
+    mg = fmaxf(mg, gd);
+  }
+  mv = warp_max(mv);
+  mg = warp_max(mg);
+  if (lane == 0) {
+    red[0][warp] = mv;
+    red[1][warp] = mg;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    float a = lane < nw ? red[0][lane] : 0.f, b = lane < nw ? red[1][lane] : 0.f;
+    a = warp_max(a);
+    b = warp_max(b);
+    if (lane == 0) {
+      red[0][0] = a;
+      red[1][0] = b;
+    }
+  }
+  __syncthreads();
+  // alpha in probability space: V_J >= alpha max V  <=>  V_J >= exp(ln alpha) max V
+  const float alpha = __expf(ht.lnalpha[h]);
+  const float tv = alpha * red[0][0], tg = alpha * red[1][0];
+  for (int w0 = warp; w0 < L.nkw; w0 += blockDim.x >> 5) {
+    const int x = w0 * 32 + lane;
+    const unsigned bv = __ballot_sync(0xffffffffu, x < nqb && V[x] >= tv);
+    const unsigned bd = __ballot_sync(0xffffffffu, x < nqb && G[x] >= tg);
+    if (lane == 0) {
+      vb[w0] = bv;
+      db[w0] = bd;
+    }
+  }
+  __syncthreads();
+  // the kept lists, ascending (warp 0: verticals, warp 1: diagonals)
+  if (warp < 2) {
+    const uint32_t* bits = warp == 0 ? vb : db;
+    int32_t* out = warp == 0 ? vert_idx + (int64_t)h * vert_stride : slash_idx + (int64_t)h * slash_stride;
+    const int stride = warp == 0 ? vert_stride : slash_stride;
+    int pos = 0;
+    for (int w0 = 0; w0 < L.nkw; ++w0) {
+      const uint32_t word = bits[w0];
+      const int x = w0 * 32 + lane;
+      const bool on = (word >> lane) & 1u;
+      const int at = pos + __popc(word & ((1u << lane) - 1u));
+      if (on && at < stride) out[at] = x;
+      pos += __popc(word);
+    }
+    for (int i = pos + lane; i < stride; i += 32) out[i] = -1;
+  }
+  // rows: OR in the verticals J <= I and the diagonal blocks I - d (d <= I)
+  uint32_t* sel0 = reinterpret_cast<uint32_t*>(ws + L.off_sel) + (int64_t)ht.bslot[h] * nqb * L.nkw;
+  for (int I = warp; I < nqb; I += blockDim.x >> 5) {
+    uint32_t* sel = sel0 + (int64_t)I * L.nkw;
+    int count = 0;
+    for (int w0 = 0; w0 <= (I >> 5); ++w0) {
+      const int J = w0 * 32 + lane;
+      const int dd = I - J;  // J = I - d
+      bool keep = J <= I && (((vb[w0] >> lane) & 1u) || (dd >= 0 && ((db[dd >> 5] >> (dd & 31)) & 1u)));
+      const unsigned add = __ballot_sync(0xffffffffu, keep);
+      uint32_t word = sel[w0];
+      word |= add;
+      if (w0 == (I >> 5)) word &= low_mask_upto(I & 31);  // candidates J <= I only
+      if (lane == 0) sel[w0] = word;
+      count += __popc(word);
+    }
+    if (lane == 0) blk_ptr[1 + h * nqb + I] = count;
+  }
 }
+
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-template <int D, int RT, int PASS>
-__global__ void __launch_bounds__(256) k_vs(const __grid_constant__ HeadTab ht, Layout L, const __nv_bfloat16* Q,
-                                            int64_t q_hs, int64_t q_ts, const __nv_bfloat16* K, int64_t k_hs,
-                                            int64_t k_ts, uint8_t* ws) {
-  pdl_prologue();
-  constexpr int LP = 16 * RT;
-  constexpr int WPR = 8 / RT;            // warps per row tile
-  constexpr int KPW = VS_SUB / WPR;      // keys per warp per sub-tile
-  constexpr int NT = KPW / 8;            // n-tiles per warp
-  constexpr int DP = D + 8;              // padded smem row (bf16)
-  constexpr int CH = D / 8;              // 16-byte pieces per row
-  extern __shared__ uint8_t smraw[];
-  __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(smraw);          // [LP][DP]
-  constexpr int PP = VS_SUB + 4;         // padded fp32 row of the P tile
-  __nv_bfloat16* ks = qs + LP * DP;                                      // [VS_SUB][DP]
-  float* ps = reinterpret_cast<float*>(ks + VS_SUB * DP);                // [LP][PP] (pass 2)
-  const int CHK = L.vs_chunk;
-  float* sbuf = ps + LP * PP;                                            // [CHK + LP]
-  float* vbuf = sbuf + CHK + LP;                                         // [CHK]
-  float* rowm = vbuf + CHK;                                              // [LP]
-  float* rowl = rowm + LP;                                               // [LP]
-  float* wpart = rowl + LP;                                              // [8][LP][2] (pass 1)
+// Waits, bounded by the default limit and ignoring the abort flag, for a
+// phase to complete (loads or MMAs this CTA issued, before it exits).
+static __device__ __noinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+  }
+}
 
-  // chunk-major order: q-heads of one KV group read the same K chunk back to back
-  const int vslot = blockIdx.x % L.nvs;
-  const int chunk = blockIdx.x / L.nvs;
-  const int h = ht.vhead[vslot];
-  const int kvh = h / L.G;
-  const int Lq = min(ht.last_q[h], L.N);
-  const int i0 = L.N - Lq;  // first estimate row
+// ---------------------------------------------------------------------------
+// VS estimate on the tensor cores.  One CTA per (row tile, key chunk): a row
+// tile stacks the estimate rows of up to two VS q-heads of one KV group (64
+// rows each, or one head of up to 128 rows) into one 128-row operand, so a K
+// sub-tile loaded once by TMA feeds both heads.  Per 128-key sub-tile one
+// elected thread issues the product into tensor memory (two 128-column buffers,
+// so the next product overlaps the work on this one):
+//   PASS 1: S = Qrows K^T (lane = row): running max and sum of 2^(x - max) per
+//           row over the chunk -> per-chunk partials (merged by k_vs_rowstats);
+//   PASS 2: S^T = K Qrows^T (lane = key): p = 2^(x - m_i - log2 l_i) for every
+//           row i; v[j] is a sum over the thread's own values.  s[o] is
+//           summed along the diagonals of each warp's 32-key x 64-row block by
+//           a register that moves up one lane per row (a diagonal enters at
+//           lane 0 and is complete when it leaves lane 31), written once into
+//           the warp's window and merged in a fixed order into the chunk's window
+//           of offsets (no atomics: the sums are the same bit for bit on every run).
+// x = tau log2(e) q.k, so every exponential is one ex2.  Warp 0 issues the TMA
+// loads, warp 1 the MMAs; eight compute warps: two per TMEM lane quadrant, each
+// taking one half (64) of the 128 columns.
+// ---------------------------------------------------------------------------
+// One lane waits (suspended in try_wait), the warp learns the outcome.
+__device__ __forceinline__ bool vt_warp_wait(uint64_t* bar, uint32_t parity, uint64_t limit, unsigned* status,
+                                             unsigned detail, volatile int* abort_flag) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait_ool(bar, parity, limit, status, detail, abort_flag, true) ? 1 : 0;
+  ok = __shfl_sync(0xffffffffu, ok, 0);
+  return ok != 0;
+}
+// Named barrier over n threads that also returns whether `pred` held on all of
+// them, so that the warps of a group leave a loop together.
+__device__ __forceinline__ bool named_barrier_and(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+constexpr int VT_COMPUTE = 256;             // eight compute warps
+constexpr int VT_THREADS = 64 + VT_COMPUTE;
+constexpr int VT_ROWS = 128;                // rows of a row tile (the MMA's M or N)
+constexpr int VT_HALF = 64;                 // columns per compute warp
+constexpr int VT_SLAB = 128 * 128;          // bytes of one 128-row x 64-column bf16 slab
+constexpr int VT_WW = VT_ROWS + 32;         // per-warp window
+
+struct VsTiles {
+  int n;
+  int h0[MAXH];  // first q-head of the tile
+  int h1[MAXH];  // second q-head (-1: the tile holds one head)
+  int lp[MAXH];  // rows per head slot: 64 (two heads) or 128 (one head)
+};
+
+template <int D>
+struct VtSmem {
+  static constexpr int DS = D / 64;
+  static constexpr int Q_OFF = 0;
+  static constexpr int K_OFF = DS * VT_SLAB;                  // two stages
+  static constexpr int BAR_OFF = K_OFF + 2 * DS * VT_SLAB;    // 10 barriers
+  static constexpr int MISC_OFF = BAR_OFF + 10 * 8;           // [0] tmem base, [1] abort
+  static constexpr int ROWM_OFF = MISC_OFF + 16;              // float [VT_ROWS]: m_i + log2 l_i (pass 2)
+  static constexpr int VSUM_OFF = ROWM_OFF + VT_ROWS * 4;     // float [VT_ROWS] (pass 2)
+  // pass 2: float [8 warps][VT_WW] windows; pass 1: float [2][2][VT_ROWS] row partials
+  static constexpr int WIN_OFF = VSUM_OFF + VT_ROWS * 4;
+  static constexpr int CWIN_OFF = WIN_OFF + 8 * VT_WW * 4;    // float [2 slots][chunk + VT_ROWS]
+  static int bytes(int chunk) { return CWIN_OFF + 2 * (chunk + VT_ROWS) * 4 + 1024; }
+};
+static_assert(8 * VT_WW >= 4 * VT_ROWS, "pass-1 partials fit in the window area");
+enum { VB_QFULL = 0, VB_KFULL = 1, VB_KEMPTY = 3, VB_SFULL = 5, VB_SEMPTY = 7, VB_DRAIN = 9 };
+
+template <int D, int PASS>
+__global__ void __launch_bounds__(VT_THREADS, 2)
+k_vs_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+        const __grid_constant__ HeadTab ht, const __grid_constant__ VsTiles vt, Layout L, uint8_t* ws,
+        unsigned* status, uint64_t limit) {
+  pdl_prologue();
+  using S = VtSmem<D>;
+  constexpr int DS = S::DS;
+  extern __shared__ uint8_t vt_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(vt_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + S::BAR_OFF);
+  int* misc = reinterpret_cast<int*>(sm + S::MISC_OFF);
+  volatile int* abort_flag = misc + 1;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tile = blockIdx.x % vt.n;
+  const int chunk = blockIdx.x / vt.n;
+  const int CHK = L.vs_chunk;
   const int j0 = chunk * CHK;
   const int j1 = min(L.N, j0 + CHK);
-  const float sc = 1.4426950408889634f * rsqrtf((float)D);  // tau * log2(e)
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int rt = warp % RT, kg = warp / RT;
-  const int g = lane >> 2, t4 = lane & 3;
-  const __nv_bfloat16* kbase = K + kvh * k_hs;
+  const int nsub = (j1 - j0 + VT_ROWS - 1) / VT_ROWS;
+  const int LP = vt.lp[tile];
+  const int hs[2] = {vt.h0[tile], vt.h1[tile]};
+  const int kvh = hs[0] / L.G;
 
-  auto load_sub = [&](int sub) {
-    __nv_bfloat16* dst = ks;
-#pragma unroll
-    for (int it = 0; it < VS_SUB * CH / 256; ++it) {
-      const int idx = it * 256 + tid;
-      const int r = idx / CH, c = (idx % CH) * 8;
-      const bool in = sub + r < j1;
-      cp_async16(dst + r * DP + c, kbase + (int64_t)(in ? sub + r : j0) * k_ts + c, in ? 16u : 0u);
-    }
-    cp_async_commit();
-  };
-  load_sub(j0);
-
-  // Q rows (padding rows are zero)
-  for (int idx = tid; idx < LP * CH; idx += 256) {
-    const int r = idx / CH, c = (idx % CH) * 8;
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (r < Lq) v = *reinterpret_cast<const uint4*>(Q + h * q_hs + (int64_t)(i0 + r) * q_ts + c);
-    *reinterpret_cast<uint4*>(qs + r * DP + c) = v;
+  if (tid == 0) {
+    for (int i = 0; i < 10; ++i) mbar_init(&bars[i], (i == VB_SEMPTY || i == VB_SEMPTY + 1) ? 8 : 1);
+    fence_barrier_init();
+    misc[1] = 0;
   }
-  float* part = reinterpret_cast<float*>(ws + L.off_part);
-  float* stat = reinterpret_cast<float*>(ws + L.off_stat);
-  if (PASS == 2) {
-    for (int i = tid; i < CHK + LP; i += 256) sbuf[i] = 0.f;
-    for (int i = tid; i < CHK; i += 256) vbuf[i] = 0.f;
-    for (int r = tid; r < LP; r += 256) {
-      rowm[r] = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 0] : 0.f;
-      const float l = (r < Lq) ? stat[((int64_t)vslot * VS_MAXL + r) * 2 + 1] : 1.f;
-      rowl[r] = 1.f / l;
-    }
+  if (warp == 1) {
+    tmem_alloc(reinterpret_cast<uint32_t*>(&misc[0]), 256);
+    tc_fence_before();
+  }
+  if (tid == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
   }
   __syncthreads();
-  // A fragments of this warp's row tile, kept in registers
-  uint32_t af[D / 16][4];
-  {
-    const int q = t4 * 2;
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-      const __nv_bfloat16* base = qs + (rt * 16) * DP + kk * 16;
-      af[kk][0] = *reinterpret_cast<const uint32_t*>(base + g * DP + q);
-      af[kk][1] = *reinterpret_cast<const uint32_t*>(base + (g + 8) * DP + q);
-      af[kk][2] = *reinterpret_cast<const uint32_t*>(base + g * DP + q + 8);
-      af[kk][3] = *reinterpret_cast<const uint32_t*>(base + (g + 8) * DP + q + 8);
-    }
-  }
-  const int rA = rt * 16 + g;  // this thread's two rows: rA, rA + 8
-  float rm[2] = {0.f, 0.f}, rl[2] = {0.f, 0.f};
-  if (PASS == 2) {
-    rm[0] = rowm[rA];
-    rm[1] = rowm[rA + 8];
-    rl[0] = rowl[rA];
-    rl[1] = rowl[rA + 8];
-  }
-  float run_m[2] = {-INFINITY, -INFINITY}, run_l[2] = {0.f, 0.f};
-  const int obase = i0 - (j0 + CHK - 1);  // sbuf index of offset o is o - obase
-  const int nsub = (j1 - j0 + VS_SUB - 1) / VS_SUB;
-  for (int si = 0; si < nsub; ++si) {
-    const int sub = j0 + si * VS_SUB;
-    cp_async_wait<0>();
-    __syncthreads();
-    const __nv_bfloat16* kt = ks;
-    float acc[NT][4];
-#pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
-#pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int key = kg * KPW + n * 8 + g;
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const __nv_bfloat16* kb = kt + key * DP + kk * 16 + t4 * 2;
-        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(kb);
-        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(kb + 8);
-        mma_bf16_16816(acc[n], af[kk], b0, b1);
+  tc_fence_after();
+  const uint32_t tmem = static_cast<uint32_t>(misc[0]);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      // estimate rows: slot s holds rows [N - Lq, N - Lq + LP) of head hs[s]
+      // (rows past N arrive as zeros and are masked)
+      const int nslot = hs[1] >= 0 ? 2 : 1;
+      mbar_arrive_expect_tx(&bars[VB_QFULL], DS * VT_SLAB);
+      for (int s = 0; s < 2; ++s) {
+        const int h = s < nslot ? hs[s] : hs[0];
+        const int i0 = L.N - min(ht.last_q[h], L.N);
+        for (int r = 0; r < (LP == 64 ? 1 : 2) && s * LP + r * 64 < VT_ROWS; ++r)
+          for (int c = 0; c < DS; ++c)
+            tma_load_3d(sm + S::Q_OFF + c * VT_SLAB + (s * LP + r * 64) * 128, &tmQ, &bars[VB_QFULL], c * 64,
+                        i0 + r * 64, h);
+      }
+      int last[2] = {-1, -1};
+      bool ok = true;
+      for (int t = 0; t < nsub; ++t) {
+        const int b = t & 1;
+        if (t >= 2 && !mbar_wait_ool(&bars[VB_KEMPTY + b], ((t >> 1) - 1) & 1, limit, status, DETAIL_WAIT_EMPTY,
+                                     abort_flag, true)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&bars[VB_KFULL + b], DS * VT_SLAB);
+        last[b] = t;
+        for (int c = 0; c < DS; ++c)
+          tma_load_3d(sm + S::K_OFF + (b * DS + c) * VT_SLAB, &tmK, &bars[VB_KFULL + b], c * 64,
+                      j0 + t * VT_ROWS, kvh);
+      }
+      if (!ok) {
+        // a wait ran out: the loads this thread issued land before the CTA exits
+        // (only this thread arms these barriers, so the parities are unambiguous)
+        mbar_drain(&bars[VB_QFULL], 0);
+        for (int b = 0; b < 2; ++b)
+          if (last[b] >= 0) mbar_drain(&bars[VB_KFULL + b], (last[b] >> 1) & 1);
       }
     }
-    __syncthreads();  // every warp has read the sub-tile: refill the buffer
-    if (si + 1 < nsub) load_sub(sub + VS_SUB);
-    // logits in log2 units, masked (row < Lq, key <= row, key < N)
-    const int cb = sub + kg * KPW + t4 * 2;  // column of element (n = 0, e = 0)
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC = idesc_bf16(VT_ROWS, VT_ROWS, 0, 0);
+      const uint64_t qd = smem_desc(smem_u32(sm + S::Q_OFF), 16, 1024, SWZ_128B);
+      bool ok = mbar_wait_ool(&bars[VB_QFULL], 0, limit, status, DETAIL_WAIT_Q, abort_flag, true);
+      for (int t = 0; ok && t < nsub; ++t) {
+        const int b = t & 1;
+        const uint32_t use = (t >> 1) & 1;
+        if (!mbar_wait_ool(&bars[VB_KFULL + b], use, limit, status, DETAIL_WAIT_K, abort_flag, true)) break;
+        if (t >= 2 && !mbar_wait_ool(&bars[VB_SEMPTY + b], use ^ 1, limit, status, DETAIL_WAIT_SFREE, abort_flag, true))
+          break;
+        tc_fence_after();
+        const uint64_t kd = smem_desc(smem_u32(sm + S::K_OFF + b * DS * VT_SLAB), 16, 1024, SWZ_128B);
+        // pass 1: rows x keys (A = Q rows); pass 2: keys x rows (A = K)
+        const uint64_t a0 = PASS == 1 ? qd : kd, b0 = PASS == 1 ? kd : qd;
 #pragma unroll
-    for (int n = 0; n < NT; ++n) {
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)((kk >> 2) * (VT_SLAB >> 4) + (kk & 3) * 2);
+          tc_mma_f16(tmem + 128 * b, a0 + off, b0 + off, IDESC, kk > 0 ? 1u : 0u);
+        }
+        tc_commit(&bars[VB_SFULL + b]);
+        tc_commit(&bars[VB_KEMPTY + b]);
+      }
+      tc_commit(&bars[VB_DRAIN]);
+      mbar_drain(&bars[VB_DRAIN], 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ compute
+    const int cw = warp - 2;                  // 0..7
+    const int q4 = warp & 3;                  // TMEM lane quadrant
+    const int ch = cw >> 2;                   // column half: columns [64 ch, 64 ch + 64)
+    const int lr = q4 * 32 + lane;            // this thread's TMEM lane
+    const uint32_t col0 = (uint32_t)(VT_HALF * ch);
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const float sc = 1.4426950408889634f * rsqrtf((float)D);
+    const int ctid = tid - 64;                // 0..255
+    int lq[2], i0[2], vsl[2];
+    for (int s = 0; s < 2; ++s) {
+      const int h = hs[s];
+      lq[s] = h >= 0 ? min(ht.last_q[h], L.N) : 0;
+      i0[s] = L.N - lq[s];
+      vsl[s] = h >= 0 ? ht.vslot[h] : 0;
+    }
+    float* rowm = reinterpret_cast<float*>(sm + S::ROWM_OFF);
+    float* vsum = reinterpret_cast<float*>(sm + S::VSUM_OFF);
+    float* wins = reinterpret_cast<float*>(sm + S::WIN_OFF);
+    float* win = wins + cw * VT_WW;           // this warp's window (pass 2)
+    float* cwin = reinterpret_cast<float*>(sm + S::CWIN_OFF);
+    // pass 2: this warp's columns are rows [64 ch, 64 ch + 64) of the tile,
+    // i.e. head slot wslot, its rows rr = rbase + c (c < 64)
+    const int wslot = LP == 64 ? ch : 0;
+    const int rbase = LP == 64 ? 0 : VT_HALF * ch;
+    if (PASS == 2) {
+      const float* stat = reinterpret_cast<const float*>(ws + L.off_stat);
+      for (int r = ctid; r < VT_ROWS; r += VT_COMPUTE) {
+        const int s = r / LP, rr = r % LP;
+        const bool valid = s < 2 && hs[s] >= 0 && rr < lq[s];
+        // p = 2^(x - m) / l = 2^(x - (m + log2 l)); rows outside the head: p = 0
+        rowm[r] = valid ? stat[((int64_t)vsl[s] * VS_MAXL + rr) * 2 + 0] +
+                              __log2f(stat[((int64_t)vsl[s] * VS_MAXL + rr) * 2 + 1])
+                        : INFINITY;
+      }
+      for (int i = ctid; i < 8 * VT_WW; i += VT_COMPUTE) wins[i] = 0.f;
+      for (int i = ctid; i < 2 * (CHK + VT_ROWS); i += VT_COMPUTE) cwin[i] = 0.f;
+      named_barrier(1, VT_COMPUTE);
+    }
+    // pass 1 state: this thread's row, over its half of the columns
+    const int ps = lr / LP, prr = lr % LP;
+    const bool prow = PASS == 1 && ps < 2 && hs[ps] >= 0 && prr < lq[ps];
+    const int pi = prow ? i0[ps] + prr : -1;
+    float run_m = -INFINITY, run_l = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nsub; ++t) {
+      const int b = t & 1;
+      const uint32_t use = (t >> 1) & 1;
+      const int jt = j0 + t * VT_ROWS;  // first key of the sub-tile
+      ok = vt_warp_wait(&bars[VB_SFULL + b], use, limit, status, DETAIL_WAIT_S, abort_flag);
+      if (PASS == 2) ok = named_barrier_and(1, VT_COMPUTE, ok);  // the compute warps leave together
+      if (!ok) break;
+      tc_fence_after();
+      float x[VT_HALF];
+      tmem_ld32(tmem + lane_off + 128 * b + col0, x);
+      tmem_ld32(tmem + lane_off + 128 * b + col0 + 32, x + 32);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[VB_SEMPTY + b]);  // the buffer is free for sub-tile t + 2
+      if (PASS == 1) {
+        // row pi against keys jt + 64 ch + c: valid while j <= pi and j < j1
+        const int nv = prow ? min(VT_HALF, min(pi + 1, j1) - (jt + VT_HALF * ch)) : 0;
+        float mx = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int r = rA + ((e >> 1) << 3);
-        const int j = cb + n * 8 + (e & 1);
-        const bool ok = (r < Lq) && (j < j1) && (j <= i0 + r);
-        acc[n][e] = ok ? acc[n][e] * sc : -INFINITY;
+        for (int c = 0; c < VT_HALF; ++c) {
+          x[c] = c < nv ? x[c] * sc : -INFINITY;
+          mx = fmaxf(mx, x[c]);
+        }
+        if (mx != -INFINITY) {
+          if (mx > run_m) {
+            run_l = (run_m == -INFINITY) ? 0.f : run_l * ex2_approx(run_m - mx);
+            run_m = mx;
+          }
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int c = 0; c < VT_HALF; c += 2) {
+            s0 += ex2_approx(x[c] - run_m);
+            s1 += ex2_approx(x[c + 1] - run_m);
+          }
+          run_l += s0 + s1;
+        }
+      } else {
+        // key j = jt + lr against rows rr = rbase + c, c = 0..63, of head slot
+        // wslot (estimate row i = i0 + rr); the pair counts when j <= i and
+        // j < N.  Window index t = c - lane + 31 holds offset o = i - j: the
+        // diagonal of (c, lane); dacc carries diagonal t in lane c - t + 31.
+        const int j = jt + lr;
+        const bool kv = j < j1;
+        const int jlim = min(j1, jt + VT_ROWS) - 1;  // the sub-tile's last key
+        const bool nomask = jlim <= i0[wslot] && jt + VT_ROWS <= j1;
+        const int ilim = i0[wslot] + rbase;  // row of column c is ilim + c
+        float v = 0.f, dacc = 0.f;
+        const float4* rm4 = reinterpret_cast<const float4*>(rowm + VT_HALF * ch);
+#pragma unroll
+        for (int c4 = 0; c4 < VT_HALF / 4; ++c4) {
+          const float4 m4 = rm4[c4];
+          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = c4 * 4 + e;
+            const bool ok_ij = nomask || (kv && j <= ilim + c);
+            const float p = ok_ij ? ex2_approx(fmaf(x[c], sc, -mm[e])) : 0.f;
+            v += p;
+            dacc += p;
+            if (lane == 31) win[c] = dacc;          // diagonal t = c is complete
+            if (c + 1 < VT_HALF) {
+              dacc = __shfl_up_sync(0xffffffffu, dacc, 1);
+              if (lane == 0) dacc = 0.f;            // diagonal t = c + 32 starts
+            }
+          }
+        }
+        if (lane < 31) win[VT_HALF + 30 - lane] = dacc;  // diagonals t = 64 .. 94
+        if (LP != 64) {
+          // one head over both column halves: the two warps of a quadrant add
+          // their key sums in a fixed order (half 0 + half 1)
+          if (ch == 1) vsum[lr] = v;
+          named_barrier(1, VT_COMPUTE);
+          if (ch == 0) v += vsum[lr];
+        }
+        if (kv && (LP == 64 ? hs[wslot] >= 0 : ch == 0)) {
+          float* vout = reinterpret_cast<float*>(ws + L.off_v);
+          vout[(int64_t)vsl[wslot] * L.N + j] = v;
+        }
+        named_barrier(1, VT_COMPUTE);
+        // merge the warps' windows into the chunk window in a fixed order.
+        // Warp (ch, q4) covers keys jt + 32 q4 + lane and rows rbase(ch) + c;
+        // its window index t holds chunk-window index
+        // t + rbase(ch) + CHK - 32 - (jt - j0) - 32 q4 of slot wslot(ch).
+        const int base = CHK - 32 - (jt - j0);
+        const int nslot = LP == 64 ? 2 : 1;
+        for (int e = ctid; e < nslot * (VT_ROWS + 128); e += VT_COMPUTE) {
+          const int s = e / (VT_ROWS + 128);
+          const int idx = base - 96 + (e % (VT_ROWS + 128));  // chunk-window index
+          if ((LP == 64 && hs[s] < 0) || idx < 0 || idx >= CHK + VT_ROWS) continue;
+          float acc = cwin[s * (CHK + VT_ROWS) + idx];
+#pragma unroll
+          for (int w = 0; w < 8; ++w) {
+            const int wch = w >> 2, wq = (w + 2) & 3;  // warp 2 + w: column half, quadrant
+            const int ws_ = LP == 64 ? wch : 0;
+            if (ws_ != s) continue;
+            const int rb = LP == 64 ? 0 : VT_HALF * wch;
+            const int tw = idx - (base + rb - 32 * wq);
+            if (tw >= 0 && tw < VT_WW) acc += wins[w * VT_WW + tw];
+          }
+          cwin[s * (CHK + VT_ROWS) + idx] = acc;
+        }
+        named_barrier(1, VT_COMPUTE);  // every entry t <= 94 is rewritten next sub-tile
       }
     }
     if (PASS == 1) {
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        float mx = -INFINITY;
-#pragma unroll
-        for (int n = 0; n < NT; ++n) mx = fmaxf(mx, fmaxf(acc[n][2 * hr], acc[n][2 * hr + 1]));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float mnew = fmaxf(run_m[hr], mx);
-        const bool live = mnew != -INFINITY;
-        float s = 0.f;
-        if (live) {
-#pragma unroll
-          for (int n = 0; n < NT; ++n) s += ex2_approx(acc[n][2 * hr] - mnew) + ex2_approx(acc[n][2 * hr + 1] - mnew);
-        }
-        s += __shfl_xor_sync(0xffffffffu, s, 1);
-        s += __shfl_xor_sync(0xffffffffu, s, 2);
-        if (live) {
-          run_l[hr] = run_l[hr] * ex2_approx(run_m[hr] - mnew) + s;
-          run_m[hr] = mnew;
-        }
+      // the two column halves of each row: (m, l) pairs combined in a fixed order
+      float* pm = wins;                 // [2][VT_ROWS] max
+      float* pl = wins + 2 * VT_ROWS;   // [2][VT_ROWS] sum
+      pm[ch * VT_ROWS + lr] = run_m;
+      pl[ch * VT_ROWS + lr] = run_l;
+      named_barrier(1, VT_COMPUTE);
+      if (ch == 0 && prow) {
+        const float m0 = pm[lr], m1 = pm[VT_ROWS + lr];
+        const float m = fmaxf(m0, m1);
+        float l = 0.f;
+        if (m0 != -INFINITY) l += pl[lr] * ex2_approx(m0 - m);
+        if (m1 != -INFINITY) l += pl[VT_ROWS + lr] * ex2_approx(m1 - m);
+        float* part = reinterpret_cast<float*>(ws + L.off_part);
+        float* pp = part + (((int64_t)vsl[ps] * L.vs_nchunks + chunk) * VS_MAXL + prr) * 2;
+        pp[0] = m;
+        pp[1] = l;
       }
-    } else {
-      // p into the fp32 tile (masked entries are -inf -> 0)
-#pragma unroll
-      for (int n = 0; n < NT; ++n) {
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int r = rA + ((e >> 1) << 3);
-          const int c = kg * KPW + n * 8 + t4 * 2 + (e & 1);
-          ps[r * PP + c] = ex2_approx(acc[n][e] - rm[e >> 1]) * rl[e >> 1];
-        }
-      }
-      __syncthreads();
-      if (tid < VS_SUB) {
-        float cs = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < LP; ++r) cs += ps[r * PP + tid];
-        vbuf[sub - j0 + tid] += cs;
-      }
-      // offset o meets row r at column c = i0 + r - o - sub, i.e. the rows
-      // [o + sub - i0, o + sub - i0 + VS_SUB) of the tile; neighbouring threads
-      // read neighbouring columns of each row
-      for (int o = i0 - (sub + VS_SUB - 1) + tid; o <= i0 + LP - 1 - sub; o += 256) {
-        const int base = o + sub - i0;
-        const int rlo = max(0, base), rhi = min(LP, base + VS_SUB);
-        float acc_s = 0.f;
-        for (int r = rlo; r < rhi; ++r) acc_s += ps[r * PP + (r - base)];
-        sbuf[o - obase] += acc_s;
+    } else if (ok) {
+      named_barrier(1, VT_COMPUTE);
+      // this chunk's windows of slash sums (offset o at index o - (i0 - (j0 + CHK - 1)))
+      for (int s = 0; s < (hs[1] >= 0 ? 2 : 1); ++s) {
+        float* wout = reinterpret_cast<float*>(ws + L.off_spart) +
+                      ((int64_t)vsl[s] * L.vs_nchunks + chunk) * (CHK + VS_MAXL);
+        for (int t = ctid; t < CHK + VS_MAXL; t += VT_COMPUTE)
+          wout[t] = (t < CHK + lq[s]) ? cwin[s * (CHK + VT_ROWS) + t] : 0.f;
       }
     }
-    __syncthreads();  // the P tile and the sums are done before the next sub-tile
   }
-  if (PASS == 1) {
-    // combine the key-group warps of each row tile
-    if (t4 == 0) {
-#pragma unroll
-      for (int hr = 0; hr < 2; ++hr) {
-        wpart[(kg * LP + rA + 8 * hr) * 2 + 0] = run_m[hr];
-        wpart[(kg * LP + rA + 8 * hr) * 2 + 1] = run_l[hr];
-      }
-    }
-    __syncthreads();
-    for (int r = tid; r < Lq; r += 256) {
-      float m = -INFINITY;
-      for (int gw = 0; gw < WPR; ++gw) m = fmaxf(m, wpart[(gw * LP + r) * 2]);
-      float l = 0.f;
-      if (m != -INFINITY)
-        for (int gw = 0; gw < WPR; ++gw) {
-          const float gm = wpart[(gw * LP + r) * 2];
-          if (gm != -INFINITY) l += wpart[(gw * LP + r) * 2 + 1] * ex2_approx(gm - m);
-        }
-      float* pp = part + (((int64_t)vslot * L.vs_nchunks + chunk) * VS_MAXL + r) * 2;
-      pp[0] = m;
-      pp[1] = l;
-    }
-  } else {
-    __syncthreads();
-    float* vout = reinterpret_cast<float*>(ws + L.off_v) + (int64_t)vslot * L.N;
-    for (int j = j0 + tid; j < j1; j += 256) vout[j] = vbuf[j - j0];
-    // this chunk's window of slash sums (offset o at index o - obase); the
-    // windows of neighbouring chunks overlap and are added in a fixed order by
-    // k_vs_slash_combine, so s is the same bit for bit on every run
-    float* win = reinterpret_cast<float*>(ws + L.off_spart) +
-                 ((int64_t)vslot * L.vs_nchunks + chunk) * (CHK + VS_MAXL);
-    for (int t = tid; t < CHK + VS_MAXL; t += 256) win[t] = (t < CHK + LP) ? sbuf[t] : 0.f;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
   }
 }
 
@@ -1346,6 +1648,7 @@ dsa_status check_pattern(const dsa_problem& p, const dsa_pattern& q) {
       if (q.topk < 1) return DSA_ERR_INVALID_ARG;
       return DSA_OK;
     case DSA_KIND_BLOCK_THRESHOLD:
+    case DSA_KIND_UNIFIED:
       if (!(q.alpha > 0.f && q.alpha <= 1.f)) return DSA_ERR_INVALID_ARG;
       return DSA_OK;
     case DSA_KIND_MOBA:
@@ -1359,7 +1662,7 @@ dsa_status check_pattern(const dsa_problem& p, const dsa_pattern& q) {
 }
 
 bool is_block_kind(int k) {
-  return k == DSA_KIND_BLOCK_TOPK || k == DSA_KIND_BLOCK_THRESHOLD || k == DSA_KIND_MOBA;
+  return k == DSA_KIND_BLOCK_TOPK || k == DSA_KIND_BLOCK_THRESHOLD || k == DSA_KIND_MOBA || k == DSA_KIND_UNIFIED;
 }
 
 int vs_rows_pad(int lq) {
@@ -1396,6 +1699,9 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->nkw = ceil_div(L->nqb, 32);
   L->nbh = 0;
   L->nvs = 0;
+  L->nuh = 0;
+  L->sel_ri = sel_blocks_per_cta(p.block);
+  L->sel_nx = ceil_div(L->nqb, L->sel_ri);
   L->vs_lmax = 0;
   L->vs_chunk = VS_CHUNK_MAX;  // launch_build_indices may choose a smaller one
   L->vs_nchunks = ceil_div(p.N, VS_CHUNK_MAX);
@@ -1416,18 +1722,28 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
       ht->n_vert[h] = q.n_vert;
       ht->n_slash[h] = q.n_slash;
       ht->topk[h] = q.topk;
-      ht->lnalpha[h] = q.kind == DSA_KIND_BLOCK_THRESHOLD ? logf(q.alpha) : 0.f;
+      ht->lnalpha[h] = (q.kind == DSA_KIND_BLOCK_THRESHOLD || q.kind == DSA_KIND_UNIFIED) ? logf(q.alpha) : 0.f;
       ht->keep_sink[h] = q.keep_sink;
       ht->keep_local[h] = q.keep_local;
       ht->bslot[h] = -1;
       ht->vslot[h] = -1;
+      ht->uslot[h] = -1;
     }
     if (is_block_kind(q.kind)) {
       if (ht) {
         ht->bslot[h] = L->nbh;
         ht->bhead[L->nbh] = h;
+        if (q.kind == DSA_KIND_UNIFIED) {
+          ht->uslot[h] = L->nuh;
+          ht->uhead[L->nuh] = h;
+        }
       }
       L->nbh++;
+      if (q.kind == DSA_KIND_UNIFIED) {
+        L->nuh++;
+        vstride = std::max(vstride, nqb);  // kept vertical blocks and diagonals
+        sstride = std::max(sstride, nqb);
+      }
       const int kvh = h / L->G;
       if (ct) {
         if (ct->need[kvh]) {
@@ -1487,6 +1803,8 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->off_dbits = off; off = align256(off + (int64_t)L->nvs * L->nkw * 4);
   // per-chunk windows of the slash sums (chunk + VS_MAXL offsets each)
   L->off_spart = off; off = align256(off + (int64_t)L->nvs * vs_wins * 4);
+  // unified discovery: each select CTA's shares of the vertical and diagonal sums
+  L->off_upart = off; off = align256(off + (int64_t)L->nuh * L->sel_nx * 2 * nqb * 4);
   L->total = std::max<int64_t>(off, 256);
   if (sz) {
     sz->nqb = nqb;
@@ -1505,33 +1823,48 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   return DSA_OK;
 }
 
-template <int D>
-dsa_status launch_vs(const HeadTab& ht, const Layout& L, const void* Q, int64_t q_hs, int64_t q_ts, const void* K,
-                     int64_t k_hs, int64_t k_ts, uint8_t* ws, cudaStream_t st) {
-  const int RT = L.vs_lmax / 16;
-  const int LP = L.vs_lmax;
-  const size_t smem = (size_t)(LP + VS_SUB) * (D + 8) * 2 + (size_t)LP * (VS_SUB + 4) * 4 +
-                      (size_t)(L.vs_chunk + LP + L.vs_chunk + 2 * LP + 16 * LP) * 4;
-  const dim3 grid(L.vs_nchunks * L.nvs);
-  const auto* q = static_cast<const __nv_bfloat16*>(Q);
-  const auto* k = static_cast<const __nv_bfloat16*>(K);
-#define DSA_VS_LAUNCH(R)                                                                                   \
-  do {                                                                                                     \
-    cudaFuncSetAttribute(k_vs<D, R, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
-    cudaFuncSetAttribute(k_vs<D, R, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);           \
-    launch_pdl(k_vs<D, R, 1>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
-    launch_pdl(k_vs_rowstats, dim3(L.nvs), dim3(128), 0, st, ht, L, ws);                                    \
-    launch_pdl(k_vs<D, R, 2>, grid, dim3(256), smem, st, ht, L, q, q_hs, q_ts, k, k_hs, k_ts, ws);          \
-    launch_pdl(k_vs_slash_combine, dim3(ceil_div(L.N, 256), L.nvs), dim3(256), 0, st, ht, L, ws);           \
-  } while (0)
-  switch (RT) {
-    case 1: DSA_VS_LAUNCH(1); break;
-    case 2: DSA_VS_LAUNCH(2); break;
-    case 4: DSA_VS_LAUNCH(4); break;
-    case 8: DSA_VS_LAUNCH(8); break;
-    default: return DSA_ERR_UNSUPPORTED;
+// Row tiles of the VS estimate: the VS q-heads of each KV group, two per tile
+// when both estimate at most 64 rows, one otherwise.
+void make_vs_tiles(const HeadTab& ht, const Layout& L, VsTiles* vt) {
+  vt->n = 0;
+  for (int g = 0; g < L.Hkv; ++g) {
+    int pend = -1;  // a head of <= 64 rows waiting for a partner
+    for (int h = g * L.G; h < (g + 1) * L.G; ++h) {
+      if (ht.kind[h] != DSA_KIND_VS) continue;
+      const int lq = std::min(ht.last_q[h], L.N);
+      if (lq > 64) {
+        vt->h0[vt->n] = h, vt->h1[vt->n] = -1, vt->lp[vt->n] = VT_ROWS, vt->n++;
+      } else if (pend < 0) {
+        pend = h;
+      } else {
+        vt->h0[vt->n] = pend, vt->h1[vt->n] = h, vt->lp[vt->n] = 64, vt->n++;
+        pend = -1;
+      }
+    }
+    if (pend >= 0) vt->h0[vt->n] = pend, vt->h1[vt->n] = -1, vt->lp[vt->n] = 64, vt->n++;
   }
-#undef DSA_VS_LAUNCH
+}
+
+template <int D>
+dsa_status launch_vs(const HeadTab& ht, const VsTiles& vt, const Layout& L, const dsa_problem& p, const void* Q,
+                     const void* K, uint8_t* ws, cudaStream_t st, unsigned* status) {
+  CUtensorMap mq, mk;
+  if (!make_tma_map_bf16_3d(&mq, Q, D, p.N, p.Hq, p.q_token_stride, p.q_head_stride, 64) ||
+      !make_tma_map_bf16_3d(&mk, K, D, p.N, p.Hkv, p.k_token_stride, p.k_head_stride, VT_ROWS))
+    return DSA_ERR_CUDA;
+  const int smem = VtSmem<D>::bytes(L.vs_chunk);
+  cudaError_t e = cudaFuncSetAttribute(k_vs_tc<D, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(k_vs_tc<D, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return cuda_fail(e);
+  const dim3 grid(L.vs_nchunks * vt.n);
+  const uint64_t limit = wait_limit_ns();
+  e = launch_pdl(k_vs_tc<D, 1>, grid, dim3(VT_THREADS), (size_t)smem, st, mq, mk, ht, vt, L, ws, status, limit);
+  if (e == cudaSuccess) e = launch_pdl(k_vs_rowstats, dim3(L.nvs), dim3(128), 0, st, ht, L, ws);
+  if (e == cudaSuccess)
+    e = launch_pdl(k_vs_tc<D, 2>, grid, dim3(VT_THREADS), (size_t)smem, st, mq, mk, ht, vt, L, ws, status, limit);
+  if (e == cudaSuccess)
+    e = launch_pdl(k_vs_slash_combine, dim3(ceil_div(L.N, 256), L.nvs), dim3(256), 0, st, ht, L, ws);
+  if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;
 }
 
@@ -1548,14 +1881,15 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
                                 unsigned* status) {
   static thread_local HeadTab ht;
   static thread_local ConvTab ct;
+  static thread_local VsTiles vt;
   Layout L;
   dsa_sizes sz;
   dsa_status s = make_layout(p, pats, &L, &ht, &ct, &sz);
   if (s != DSA_OK) return s;
   if ((int64_t)ws_bytes < sz.workspace_bytes) return DSA_ERR_CAPACITY;
   if (out.blk_cap < sz.blk_cap || out.dist_cap < sz.dist_cap || out.col_cap < sz.col_cap) return DSA_ERR_CAPACITY;
-  if (L.nvs > 0 && (!out.vert_idx || !out.slash_idx || out.vert_stride < sz.vert_stride ||
-                    out.slash_stride < sz.slash_stride))
+  if ((L.nvs > 0 || L.nuh > 0) && (!out.vert_idx || !out.slash_idx || out.vert_stride < sz.vert_stride ||
+                                   out.slash_stride < sz.slash_stride))
     return DSA_ERR_CAPACITY;
   uint8_t* ws = static_cast<uint8_t*>(ws_v);
   const int nrows = p.Hq * L.nqb + 1;
@@ -1565,7 +1899,8 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
     e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return cuda_fail(e);
-    L.vs_chunk = choose_vs_chunk(L.nvs, p.N, sms);
+    make_vs_tiles(ht, L, &vt);
+    L.vs_chunk = choose_vs_chunk(vt.n, p.N, sms);
     L.vs_nchunks = ceil_div(p.N, L.vs_chunk);
   }
 #define DSA_CK(x)                          \
@@ -1596,12 +1931,15 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
       DSA_CK(launch_pdl(k_block_select<64>, dim3(ceil_div(L.nqb, ri), L.nbh), dim3(SEL_NT), sel_smem, st, ht, L,
                         q, p.q_head_stride, p.q_token_stride, ws, out.blk_ptr, ri));
     }
+    if (L.nuh > 0) {
+      const size_t um = (size_t)(2 * L.nqb + 2 * L.nkw) * 4;
+      DSA_CK(launch_pdl(k_unified_merge, dim3(L.nuh), dim3(1024), um, st, ht, L, ws, out.blk_ptr, out.vert_idx,
+                        out.vert_stride, out.slash_idx, out.slash_stride));
+    }
   }
   if (L.nvs > 0) {
-    s = (p.d == 128) ? launch_vs<128>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
-                                      p.k_token_stride, ws, st)
-                     : launch_vs<64>(ht, L, Q, p.q_head_stride, p.q_token_stride, K, p.k_head_stride,
-                                     p.k_token_stride, ws, st);
+    s = (p.d == 128) ? launch_vs<128>(ht, vt, L, p, Q, K, ws, st, status)
+                     : launch_vs<64>(ht, vt, L, p, Q, K, ws, st, status);
     if (s != DSA_OK) return s;
     DSA_CK(launch_pdl(k_vs_topk, dim3(L.nvs, 2), dim3(1024), 0, st, ht, L, ws, out.vert_idx, out.vert_stride,
                       out.slash_idx, out.slash_stride));

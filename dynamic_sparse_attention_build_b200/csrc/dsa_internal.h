@@ -32,6 +32,12 @@ dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K
 dsa_status launch_count_pairs(const dsa_problem& p, const dsa_indices& idx, int64_t* pairs,
                               cudaStream_t stream, unsigned* status);
 
+// 3-D TMA map over a bf16 tensor [H][N][d] with element strides (token, head):
+// boxes of 64 columns x box_rows rows x 1 head, 128-byte swizzle, zero fill
+// outside the tensor.  False if the driver entry point or the encoding fails.
+bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int N, int H, int64_t ts, int64_t hs,
+                          int box_rows);
+
 dsa_status plan_sizes(const dsa_problem& p, const dsa_pattern* pats, dsa_sizes* out);
 
 dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void* K,

@@ -64,7 +64,9 @@ typedef enum dsa_kind {
     DSA_KIND_VS = 1,              /* Vertical-Slash, estimated from the last last_q queries */
     DSA_KIND_BLOCK_TOPK = 2,      /* MInference block-sparse: top-k pooled block scores, J <= I */
     DSA_KIND_BLOCK_THRESHOLD = 3, /* FlashPrefill: P_IJ >= alpha * max_J P_IJ, plus sink/local */
-    DSA_KIND_MOBA = 4             /* MoBA: top-k over J < I plus the own block I */
+    DSA_KIND_MOBA = 4,            /* MoBA: top-k over J < I plus the own block I */
+    DSA_KIND_UNIFIED = 5          /* FlashPrefill discovery: vertical, diagonal and block
+                                     shapes at once from the pooled block scores */
 } dsa_kind;
 
 /*
@@ -93,7 +95,15 @@ typedef struct dsa_problem {
  *   BLOCK_TOPK:      topk >= 1 (blocks per query block among J <= I).
  *   BLOCK_THRESHOLD: 0 < alpha <= 1, in probability space; keep_sink / keep_local
  *                    force blocks 0 and I.
- *   Block kinds (BLOCK_TOPK, BLOCK_THRESHOLD, MOBA) need nqb = ceil(N / block) <= 2048
+ *   UNIFIED:         0 < alpha <= 1; keep_sink / keep_local as for BLOCK_THRESHOLD.  From
+ *                    the pooled block scores s_IJ (J <= I) and their row softmax P_IJ:
+ *                    vertical sums V_J = sum_I P_IJ, diagonal sums G_d = sum_I P_{I,I-d};
+ *                    query block I keeps {J : P_IJ >= alpha max_J P_IJ}, the verticals
+ *                    J <= I with V_J >= alpha max V, and the blocks I - d of the
+ *                    diagonals d <= I with G_d >= alpha max G ("FlashPrefill" summary,
+ *                    sections 2.1 and 2.2, the max-based threshold applied per shape).
+ *                    The kept verticals and diagonals are written to vert_idx / slash_idx.
+ *   Block kinds (BLOCK_TOPK, BLOCK_THRESHOLD, MOBA, UNIFIED) need nqb = ceil(N / block) <= 2048
  *   (DSA_ERR_UNSUPPORTED otherwise).
  *   MOBA:            topk >= 0 past blocks (J < I) plus the own block I.  Optional
  *                    causal depthwise key conv for routing: conv_width in [0, 8]
@@ -129,8 +139,10 @@ typedef struct dsa_pattern {
  *   dist      [dist_cap]          query block qb keeps key blocks qb - delta for delta <= qb.
  *   col_ptr   [Hq * nqb + 1]    : VS key columns of (h, qb) are col_idx[col_ptr[r] .. col_ptr[r+1]),
  *   col_idx   [col_cap]           none of them inside a block the row already keeps.
- *   vert_idx  [Hq * vert_stride]: chosen vertical columns of VS heads (ascending, -1 padded).
- *   slash_idx [Hq * slash_stride]: chosen slash offsets o = i - j of VS heads (ascending, -1 padded).
+ *   vert_idx  [Hq * vert_stride]: chosen vertical columns of VS heads, vertical key blocks of
+ *                                 UNIFIED heads (ascending, -1 padded).
+ *   slash_idx [Hq * slash_stride]: chosen slash offsets o = i - j of VS heads, diagonal block
+ *                                 distances d of UNIFIED heads (ascending, -1 padded).
  * dsa_sparse_prefill reads only head_info, blk_*, dist*, col_*.
  */
 typedef struct dsa_indices {

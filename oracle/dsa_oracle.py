@@ -68,7 +68,8 @@ VS = "vs"
 BLOCK_TOPK = "block_topk"
 BLOCK_THRESHOLD = "block_threshold"
 MOBA = "moba"
-KINDS = (ASHAPE, VS, BLOCK_TOPK, BLOCK_THRESHOLD, MOBA)
+UNIFIED = "unified"
+KINDS = (ASHAPE, VS, BLOCK_TOPK, BLOCK_THRESHOLD, MOBA, UNIFIED)
 
 
 def n_blocks(N: int, B: int) -> int:
@@ -248,6 +249,47 @@ def select_threshold(scores_row: np.ndarray, I: int, alpha: float,
     return np.union1d(kept, extra).astype(np.int64)
 
 
+def unified_pattern_scores(scores: np.ndarray):
+    """[FP] 2.1: the vertical, diagonal and block shapes are found together from
+    one pooled block search.  From the block logits s_IJ (J <= I):
+      P_IJ = softmax_{J <= I}(s_IJ)                  (row-normalised block weights),
+      V_J  = sum_{I >= J} P_IJ                       (vertical: one key block for every query block),
+      G_d  = sum_{I >= d} P_{I, I - d}               (diagonal: one block distance d),
+    the block-level counterparts of the VS estimate's column and slash sums.
+    Returns (P with zeros above the diagonal, V, G)."""
+    nqb = scores.shape[0]
+    P = np.zeros((nqb, nqb))
+    for I in range(nqb):
+        row = scores[I, : I + 1]
+        w = np.exp(row - row.max())
+        P[I, : I + 1] = w / w.sum()
+    V = P.sum(axis=0)
+    G = np.array([np.trace(P, offset=-dd) for dd in range(nqb)])
+    return P, V, G
+
+
+def select_unified(scores: np.ndarray, alpha: float, keep_sink: bool, keep_local: bool):
+    """The max-based threshold of [FP] 2.2 applied per pattern: verticals
+    {J : V_J >= alpha max V}, diagonals {d : G_d >= alpha max G}, and for each
+    query block I its blocks {J <= I : P_IJ >= alpha max_J P_IJ}.  Query block I
+    keeps the union of its blocks, the verticals J <= I, the blocks I - d of the
+    diagonals d <= I, and block 0 / block I when asked.
+    Returns (list of ascending block arrays, verticals, diagonals)."""
+    P, V, G = unified_pattern_scores(scores)
+    vert = np.nonzero(V >= alpha * V.max())[0]
+    diag = np.nonzero(G >= alpha * G.max())[0]
+    out = []
+    for I in range(scores.shape[0]):
+        row = P[I, : I + 1]
+        parts = [np.nonzero(row >= alpha * row.max())[0], vert[vert <= I], I - diag[diag <= I]]
+        if keep_sink:
+            parts.append(np.array([0]))
+        if keep_local:
+            parts.append(np.array([I]))
+        out.append(np.unique(np.concatenate(parts)).astype(np.int64))
+    return out, vert.astype(np.int64), diag.astype(np.int64)
+
+
 # ---------------------------------------------------------------------------
 # Per-head index construction.
 # ---------------------------------------------------------------------------
@@ -269,6 +311,8 @@ class HeadIndex:
     vscore: np.ndarray | None = None
     sscore: np.ndarray | None = None
     block_scores: np.ndarray | None = None   # [nqb, nkb] logits (block kinds)
+    vert_blocks: np.ndarray | None = None    # unified: kept vertical key blocks
+    diag_blocks: np.ndarray | None = None    # unified: kept diagonal block distances
     runs: list | None = None   # VS with slash_cover "windows": [n, 2] key runs per query block
 
 
@@ -303,6 +347,12 @@ def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
             hi.cols = [vs_window_columns(hi.V, hi.runs[qb], qb, B) for qb in range(nqb)]
         else:
             raise ValueError(f"unknown slash_cover {cover!r}")
+    elif kind == UNIFIED:
+        sc = block_logits(mean_pool(Qh, B), mean_pool(Kh, B), d)
+        hi.block_scores = sc
+        hi.blocks, hi.vert_blocks, hi.diag_blocks = select_unified(
+            sc, float(pattern["alpha"]), bool(pattern.get("keep_sink", 1)), bool(pattern.get("keep_local", 1)))
+        hi.cols = [empty] * nqb
     elif kind in (BLOCK_TOPK, BLOCK_THRESHOLD, MOBA):
         keys = Kh
         if kind == MOBA and conv is not None:

@@ -29,7 +29,7 @@ def oracle_heads_to_lists(heads):
 def gpu_lists_to_oracle_heads(bufs, N, B):
     """Library index buffers -> oracle HeadIndex objects (VS blocks rebuilt from D
     with the oracle's own rule, so the oracle evaluates exactly the GPU's mask)."""
-    kinds = {0: orc.ASHAPE, 1: orc.VS, 2: orc.BLOCK_TOPK, 3: orc.BLOCK_THRESHOLD, 4: orc.MOBA}
+    kinds = {0: orc.ASHAPE, 1: orc.VS, 2: orc.BLOCK_TOPK, 3: orc.BLOCK_THRESHOLD, 4: orc.MOBA, 5: orc.UNIFIED}
     heads = []
     nqb = (N + B - 1) // B
     for hl in bufs.host_lists():

@@ -46,6 +46,24 @@ def check_indices(bufs, ref_heads, pats, N, B, convs_ref=None):
             for qb in range(nqb):
                 want = orc.vs_columns(np.asarray(g["vert"], np.int64), D, qb, B)
                 assert list(g["cols"][qb]) == list(want), (h, qb)
+        elif kind == "unified":
+            # the kept verticals and diagonals against the oracle's (tie-aware at
+            # alpha times the maximum), then each row: its own threshold blocks
+            # (tie-aware) plus exactly the GPU's verticals and diagonals
+            P, Vs, Gs = orc.unified_pattern_scores(r.block_scores)
+            a = p["alpha"]
+            for got, want, sums in ((g["vert"], r.vert_blocks, Vs), (g["slash"], r.diag_blocks, Gs)):
+                bad = [x for x in set(got.tolist()) ^ set(want.tolist()) if abs(sums[x] / sums.max() - a) > 1e-3 * a]
+                assert not bad, f"head {h}: pattern sets differ beyond the tie band at {bad[:10]}"
+            gv, gd = np.asarray(g["vert"]), np.asarray(g["slash"])
+            for I in range(nqb):
+                extra = set(gv[gv <= I].tolist()) | set((I - gd[gd <= I]).tolist())
+                forced = extra | ({0} if p.get("keep_sink", 1) else set()) | ({I} if p.get("keep_local", 1) else set())
+                row = P[I, : I + 1]
+                ref_rows = set(np.nonzero(row >= a * row.max())[0].tolist()) | forced
+                ok, msg = threshold_set_ok(g["blocks"][I], sorted(ref_rows), r.block_scores[I], I, a, forced)
+                assert ok, f"head {h} block {I}: {msg}"
+                assert set(g["blocks"][I].tolist()) >= forced
         else:
             sc = r.block_scores
             for I in range(nqb):
@@ -120,6 +138,25 @@ def test_mixed_gqa_ragged(dsa):
     run(dsa, Q, K, V, pats, B)
 
 
+def test_vs_row_tiles_d64(dsa):
+    """The VS estimate stacks the estimate rows of two VS heads of a KV group
+    (64 rows each) into one tensor-core operand, or takes one head of up to 128
+    rows alone: five VS heads of one KV group with 64, 30, 100, 1 and 64 rows
+    give two pairs and one single head, next to other kinds, at d = 64 and a
+    ragged length."""
+    N, d, B = 2100, 64, 64
+    Q, K, V = synth.random_qkv(8, 1, N, d, seed=41)
+    pats = [dict(kind="vs", last_q=64, n_vert=70, n_slash=40),
+            dict(kind="vs", last_q=30, n_vert=10, n_slash=300),
+            dict(kind="block_topk", topk=4),
+            dict(kind="vs", last_q=100, n_vert=128, n_slash=64),
+            dict(kind="vs", last_q=1, n_vert=5, n_slash=5),
+            dict(kind="ashape", sink=64, window=200),
+            dict(kind="vs", last_q=64, n_vert=1, n_slash=1000),
+            dict(kind="block_threshold", alpha=0.6)]
+    run(dsa, Q, K, V, pats, B, rows=np.r_[0:80, 1000:1100, N - 150:N])
+
+
 @pytest.mark.parametrize("B", [128, 512])
 @pytest.mark.parametrize("conv", [False, True])
 def test_moba(dsa, B, conv):
@@ -140,6 +177,23 @@ def test_threshold_topics(dsa):
     lists = bufs.host_lists()[0]["blocks"]
     hits = sum(int(all(topic[J] == topic[I] for J in lists[I] if J not in (0, I))) for I in range(len(lists)))
     assert hits >= 0.9 * len(lists)
+
+
+@pytest.mark.parametrize("wid", [2, 3])
+def test_unified_discovery(dsa, wid):
+    """FlashPrefill-style discovery of vertical, diagonal and block shapes from one
+    pooled block search (DSA_KIND_UNIFIED) on two layers: planted vertical tokens
+    and periodic slashes (the mixed layer's data), and per-block topics; with
+    another kind in the same KV group and a ragged length."""
+    N = 4000 if wid == 2 else 4096
+    w = synth.workload(wid, N=N, Hq=4, Hkv=2)
+    Q, K, V, _ = synth.make_inputs(w)
+    B = w["B"]
+    pats = [dict(kind="unified", alpha=0.5), dict(kind="unified", alpha=0.1, keep_sink=0, keep_local=0),
+            dict(kind="block_threshold", alpha=0.5), dict(kind="unified", alpha=0.9)]
+    bufs = run(dsa, Q, K, V, pats, B, rows=np.r_[0:80, 1800:1900, N - 120:N])
+    lists = bufs.host_lists()
+    assert all(len(lists[h]["vert"]) > 0 and len(lists[h]["slash"]) > 0 for h in (0, 1, 3))
 
 
 def test_index_build_is_deterministic(dsa):

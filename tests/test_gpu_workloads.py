@@ -1,8 +1,10 @@
 """GPU parity at the full sizes of the five workloads, in the launch configuration
-bench.py times: index sets of sampled heads against the oracle (tie-aware), and
-attention outputs of sampled rows against the oracle evaluating the GPU's own
-indices.  The million-token workload is also run as the 4-head x 65536-token
-slice (KV head 0) as a standalone problem."""
+bench.py times: index sets against the oracle (tie-aware; every head of the
+32K and 128K layers), the selected-pair count behind the roofline's FLOP figure
+(dsa_count_pairs against the oracle's block-wise count of the same lists, every
+head), and attention outputs of sampled rows against the oracle evaluating the
+GPU's own indices.  The million-token workload is also run as the 4-head x
+65536-token slice (KV head 0) as a standalone problem."""
 import numpy as np
 import pytest
 import torch
@@ -23,9 +25,19 @@ def dsa():
     return m
 
 
-def run_workload(dsa, w, index_heads, row_blocks, rows_per_block=64, seed=0):
+def check_pair_counts(dsa, Q, K, bufs, heads, which):
+    """dsa_count_pairs (the F_sel = 4 d |M| numerator) equals the oracle's
+    block-wise count of the same index lists, exactly, for the given heads."""
+    pairs = dsa.count_pairs(Q, K, bufs).cpu().numpy()
+    assert dsa.device_status() == (0, 0)
+    for h in which:
+        assert int(pairs[h]) == orc.selected_pairs_by_block(heads[h]), f"head {h}"
+
+
+def run_workload(dsa, w, index_heads, row_blocks, rows_per_block=64, seed=0, pair_heads=None):
     """Builds indices and attention on the GPU for workload w; checks the index
-    sets of `index_heads` and the outputs of sampled rows of every head."""
+    sets of `index_heads`, the pair counts of `pair_heads` (default: every head)
+    and the outputs of sampled rows of every head."""
     Q, K, V, planted = synth.make_inputs(w, device="cuda")
     pats = synth.head_patterns(w)
     convs = synth.conv_weights(w, device="cuda")
@@ -62,6 +74,7 @@ def run_workload(dsa, w, index_heads, row_blocks, rows_per_block=64, seed=0):
     qbs = sorted(set([nqb - 1] + list(rng.choice(nqb, size=min(nqb, row_blocks - 1), replace=False))))
     rows = np.concatenate([np.arange(qb * B, min(N, qb * B + B))[:rows_per_block] for qb in qbs])
     heads = gpu_lists_to_oracle_heads(bufs, N, B)
+    check_pair_counts(dsa, Q, K, bufs, heads, range(w["Hq"]) if pair_heads is None else pair_heads)
     Qc, Kc, Vc = to64(Q), to64(K), to64(V)
     O_ref, lse_ref = orc.sparse_attention(Qc, Kc, Vc, heads, rows)
     assert_close_outputs(to64(O)[:, rows], O_ref, w["name"])
@@ -73,17 +86,17 @@ def test_workload2_llama3_mixed_32k(dsa):
     w = synth.workload(2)
     pats = synth.head_patterns(w)
     kinds = [p["kind"] for p in pats]
-    idx_heads = [kinds.index("vs"), kinds.index("ashape"), kinds.index("block_topk")]
-    bufs, planted = run_workload(dsa, w, idx_heads, row_blocks=3, rows_per_block=16)
-    # planted verticals are found by the VS heads
-    hv = idx_heads[0]
+    bufs, planted = run_workload(dsa, w, list(range(w["Hq"])), row_blocks=3, rows_per_block=16)
+    # the planted verticals are found by the first VS head (the others are held
+    # to the oracle's own selection above, planted or not)
     G = w["Hq"] // w["Hkv"]
+    hv = kinds.index("vs")
     assert set(planted["vert"][hv // G].tolist()) <= set(bufs.host_lists()[hv]["vert"].tolist())
 
 
 def test_workload3_flashprefill_threshold_128k(dsa):
     w = synth.workload(3)
-    bufs, planted = run_workload(dsa, w, [0, 17], row_blocks=4, rows_per_block=16)
+    bufs, planted = run_workload(dsa, w, list(range(w["Hq"])), row_blocks=4, rows_per_block=16)
     # kept blocks beyond sink and local share the query block's topic
     topic = planted["topic"][0].numpy()
     lists = bufs.host_lists()[0]["blocks"]
@@ -131,9 +144,15 @@ def test_workload5_vs_1m(dsa):
         ok, msg = topk_set_ok(lists[h]["slash"], orc.topk_indices(s, pats[h]["n_slash"]), s, pats[h]["n_slash"])
         assert ok, msg
         assert set(planted["vert"][h // G].tolist()) <= set(lists[h]["vert"].tolist())
+    nqb = N // B
+    for h in (0, 5):  # distances and columns follow the GPU's own selection exactly
+        D = orc.vs_distance_set(np.asarray(lists[h]["slash"], np.int64), B, nqb)
+        assert np.array_equal(lists[h]["dist"], D), f"head {h} distances"
+        vert = np.asarray(lists[h]["vert"], np.int64)
+        for qb in range(nqb):
+            assert np.array_equal(lists[h]["cols"][qb], orc.vs_columns(vert, D, qb, B)), (h, qb)
     heads = gpu_lists_to_oracle_heads(bufs, N, B)
     rng = np.random.default_rng(5)
-    nqb = N // B
     rows = np.sort(np.concatenate([[N - 1], rng.choice(nqb, 15, replace=False) * B + rng.integers(0, B, 15)]))
     for h in (0, 1, 2, 3):
         Oh, lh = orc.attention_rows(to64(Q[h]), to64(K[h // G]), to64(V[h // G]), heads[h], rows)

@@ -79,6 +79,10 @@ MUTANTS = [
      "total += int((sink_n + win_n).sum())", "pairs_by_block"),
     ("block pair count window one short", "win_lo = rows - hi.window + 1", "win_lo = rows - hi.window + 2",
      "pairs_by_block"),
+    ("unified vertical sums over the keys", "V = P.sum(axis=0)", "V = P.sum(axis=1)", "unified"),
+    ("unified diagonal above the main one", "G = np.array([np.trace(P, offset=-dd) for dd in range(nqb)])",
+     "G = np.array([np.trace(P, offset=dd) for dd in range(nqb)])", "unified"),
+    ("unified diagonal block one off", "I - diag[diag <= I]", "I - diag[diag <= I] - 1", "unified"),
     ("slash runs: touching windows not merged", "if runs and a <= runs[-1][1] + 1:",
      "if runs and a <= runs[-1][1]:", RUNS),
     ("slash runs: window end from r0 + B", "a, b = max(0, r0 - o), r1 - o", "a, b = max(0, r0 - o), r0 + B - 1 - o",

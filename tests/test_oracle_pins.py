@@ -431,3 +431,65 @@ def test_selected_pairs_by_block_equals_the_mask_count(rng, N, B):
         want = int(orc.index_mask_dense(hi).sum())
         assert orc.selected_pairs_by_block(hi) == want, p
         assert orc.selected_pairs(hi) == want, p
+
+
+# --------------------------------------------------------------------------- unified discovery
+def _lower(rows):
+    n = len(rows)
+    sc = np.full((n, n), -7.0)  # above the diagonal: never read
+    for I, r in enumerate(rows):
+        sc[I, : I + 1] = r
+    return sc
+
+
+def test_unified_hand_example():
+    g = json.load(open(os.path.join(GOLDEN, "unified_discovery_hand_example.json")))
+    sc = _lower(g["logits_lower"])
+    P, V, G = orc.unified_pattern_scores(sc)
+    for I, row in enumerate(g["P"]):
+        np.testing.assert_allclose(P[I, : I + 1], row, rtol=1e-12)
+    np.testing.assert_allclose(V, g["V"], rtol=1e-12)
+    np.testing.assert_allclose(G, g["G"], rtol=1e-12)
+    blocks, vert, diag = orc.select_unified(sc, g["alpha"], False, False)
+    assert list(vert) == g["verticals"] and list(diag) == g["diagonals"]
+    assert [list(b) for b in blocks] == g["blocks"]
+
+
+def test_unified_sums_bruteforce_and_limits(rng):
+    """V and G against explicit loops over (I, J); alpha -> 0 keeps every J <= I,
+    alpha = 1 keeps the argmax sets; the per-row rule is the threshold kind's."""
+    n = 13
+    sc = rng.standard_normal((n, n)) * 2
+    P, V, G = orc.unified_pattern_scores(sc)
+    for I in range(n):
+        w = [math.exp(sc[I, J]) for J in range(I + 1)]
+        for J in range(I + 1):
+            assert abs(P[I, J] - w[J] / sum(w)) < 1e-12
+    for J in range(n):
+        assert abs(V[J] - sum(P[I, J] for I in range(J, n))) < 1e-12
+    for dd in range(n):
+        assert abs(G[dd] - sum(P[I, I - dd] for I in range(dd, n))) < 1e-12
+    blocks, vert, diag = orc.select_unified(sc, 1e-300, False, False)
+    assert all(list(b) == list(range(I + 1)) for I, b in enumerate(blocks))
+    blocks, vert, diag = orc.select_unified(sc, 1.0, False, False)
+    assert list(vert) == [int(np.argmax(V))] and list(diag) == [int(np.argmax(G))]
+    for I in range(n):
+        thr = orc.select_threshold(sc[I], I, 0.3, False, False)
+        b, _, _ = orc.select_unified(sc, 0.3, False, False)
+        assert set(thr) <= set(b[I])
+
+
+def test_unified_finds_planted_vertical_and_diagonal(rng):
+    """A key block that every query block favours is a vertical; a block
+    distance every query block favours is a diagonal; both reach every row."""
+    n = 40
+    sc = rng.standard_normal((n, n)) * 0.1
+    for I in range(n):
+        if I >= 7:
+            sc[I, 7] += 6.0          # planted vertical at key block 7
+        if I >= 3:
+            sc[I, I - 3] += 6.0      # planted diagonal at distance 3
+    blocks, vert, diag = orc.select_unified(sc, 0.5, True, True)
+    assert 7 in vert and 3 in diag
+    for I in range(10, n):
+        assert {0, 7, I - 3, I} <= set(blocks[I])
