@@ -521,11 +521,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       const int h = item % a.Hq;
       const int qt = a.n_qtiles - 1 - item / a.Hq;
       const int row0 = qt * BM;
-      // The item's Q tile is read from HBM once, by the producer, when the item
-      // before it has finished its last Q K^T; fetching it into L2 now (about
-      // one item ahead) takes the HBM latency off that hand-over.
-      if (dtid == 0)
-        for (int c = 0; c < DS; ++c) tma_prefetch_l2_3d(&tmQ, c * 64, row0, h);
       const int kind = a.head_info[h * 4 + 0];
       uint32_t* b0 = bits + s * 2 * a.nwords;
       uint32_t* b1 = b0 + a.nwords;
