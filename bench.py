@@ -401,13 +401,17 @@ def main():
     traffic = None
     tp = os.path.join(ROOT, "profiles", "attention_traffic.json")
     if os.path.exists(tp):
-        # DRAM bytes per launch from an ncu capture; only valid for the kernel
-        # source it was taken on and for this workload
-        tr = json.load(open(tp))
+        # DRAM bytes per launch from an ncu capture of a smaller case of the same
+        # workload, scaled by the token count (the kernel's DRAM traffic is Q read,
+        # O written and K/V first touches, each proportional to N); only valid
+        # for the kernel source it was taken on
         csrc = os.path.join(ROOT, "dynamic_sparse_attention_build_b200", "csrc")
         sha = kernel_source_hash([os.path.join(csrc, f) for f in ATTN_SOURCES])
-        if tr.get("workload") == w["name"] and tr.get("kernel_source_sha256_16") == sha and w["N"] == 32768:
-            traffic = tr.get("dram_bytes_per_launch")
+        for rec in json.load(open(tp)).get("records", []):
+            if (rec.get("workload") == w["name"] and rec.get("kernel_source_sha256_16") == sha
+                    and rec.get("block") == w["B"]):
+                traffic = int(round(rec["dram_bytes_per_launch_at_capture"] * w["N"] / rec["captured_N"]))
+                break
 
     line = {
         "metric": METRIC, "value": (N / (ms_step * 1e-3) if args.shard_heads else whole_job_tokens_per_s(N, world, ms_step)),

@@ -26,10 +26,11 @@ DSA_KIND_BLOCK_TOPK = 2
 DSA_KIND_BLOCK_THRESHOLD = 3
 DSA_KIND_MOBA = 4
 DSA_KIND_UNIFIED = 5
+DSA_KIND_VS_WINDOWS = 6
 
 KIND_CODES = {"ashape": DSA_KIND_ASHAPE, "vs": DSA_KIND_VS, "block_topk": DSA_KIND_BLOCK_TOPK,
               "block_threshold": DSA_KIND_BLOCK_THRESHOLD, "moba": DSA_KIND_MOBA,
-              "unified": DSA_KIND_UNIFIED}
+              "unified": DSA_KIND_UNIFIED, "vs_windows": DSA_KIND_VS_WINDOWS}
 
 EXPORTS = ("dsa_workspace_size", "dsa_build_indices", "dsa_sparse_prefill", "dsa_count_pairs",
            "dsa_get_device_status", "dsa_selftest_wait_timeout", "dsa_status_string",
@@ -60,7 +61,8 @@ class dsa_indices(ctypes.Structure):
                 ("col_ptr", ctypes.c_void_p), ("col_idx", ctypes.c_void_p),
                 ("vert_idx", ctypes.c_void_p), ("slash_idx", ctypes.c_void_p),
                 ("blk_cap", ctypes.c_int64), ("dist_cap", ctypes.c_int64), ("col_cap", ctypes.c_int64),
-                ("vert_stride", ctypes.c_int32), ("slash_stride", ctypes.c_int32)]
+                ("vert_stride", ctypes.c_int32), ("slash_stride", ctypes.c_int32),
+                ("kinds_present", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class dsa_sizes(ctypes.Structure):

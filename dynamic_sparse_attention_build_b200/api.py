@@ -88,6 +88,7 @@ class IndexBuffers:
     vert_idx: torch.Tensor
     slash_idx: torch.Tensor
     workspace: torch.Tensor | None = None
+    kinds_present: int = 0  # bit k: some head has kind k (dsa_kind codes)
     c: B.dsa_indices = field(default=None)
 
     def __post_init__(self):
@@ -106,6 +107,7 @@ class IndexBuffers:
         c.col_cap = self.col_idx.numel()
         c.vert_stride = self.vert_idx.numel() // max(1, self.Hq)
         c.slash_stride = self.slash_idx.numel() // max(1, self.Hq)
+        c.kinds_present = self.kinds_present
         self.c = c
 
     def host_lists(self):
@@ -146,8 +148,16 @@ def alloc_indices(problem, pats_c, device="cuda") -> IndexBuffers:
         vert_idx=torch.full((problem.Hq * sz.vert_stride,), -1, **i32),
         slash_idx=torch.full((problem.Hq * sz.slash_stride,), -1, **i32),
         workspace=torch.empty(int(sz.workspace_bytes), dtype=torch.uint8, device=device),
+        kinds_present=_kinds_mask(int(pats_c[h].kind) for h in range(problem.Hq)),
     )
     return bufs
+
+
+def _kinds_mask(codes):
+    m = 0
+    for k in codes:
+        m |= 1 << int(k)
+    return m
 
 
 def build_indices(Q, K, patterns, block, bufs: IndexBuffers | None = None, stream=None) -> IndexBuffers:
@@ -204,12 +214,12 @@ def indices_from_lists(heads, N, block, device="cuda") -> IndexBuffers:
         info[h, 0] = B.KIND_CODES[hd["kind"]]
         info[h, 1] = hd.get("sink", 0)
         info[h, 2] = hd.get("window", 0)
-        if hd["kind"] == "vs":
+        if hd["kind"] in ("vs", "vs_windows"):
             d = np.asarray(hd["dist"], np.int32)
             dist_all.append(d)
             dist_cnt[h] = d.size
         for q in range(nqb):
-            if hd["kind"] != "vs":
+            if hd["kind"] not in ("vs", "vs_windows"):
                 b = np.asarray(hd["blocks"][q], np.int32)
                 blk_all.append(b)
                 blk_cnt[h * nqb + q] = b.size
@@ -232,7 +242,8 @@ def indices_from_lists(heads, N, block, device="cuda") -> IndexBuffers:
     return IndexBuffers(Hq=Hq, N=N, block=block, nqb=nqb, head_info=t(info.ravel()), blk_ptr=t(bp),
                         blk_idx=t(bi), dist_ptr=t(dp), dist=t(di), col_ptr=t(cp), col_idx=t(ci),
                         vert_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device),
-                        slash_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device))
+                        slash_idx=torch.full((Hq,), -1, dtype=torch.int32, device=device),
+                        kinds_present=_kinds_mask(info[:, 0]))
 
 
 class HostPrefill:

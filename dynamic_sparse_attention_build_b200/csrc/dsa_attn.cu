@@ -68,10 +68,10 @@ constexpr bool kLoaderSuspend = true;
 constexpr bool kMmaSuspend = true;
 
 struct StageInfo {
-  int type;   // 0 = key unit, 1 = column tile
-  int u;      // unit id (type 0)
+  int type;   // 0 = key unit, 1 = column tile, 2 = slash-run tile
+  int u;      // unit id (type 0), first key (type 2)
   int flags;  // bit h: half h of the rows uses this tile
-  int ncols;  // valid columns (type 1)
+  int ncols;  // valid columns (type 1), valid keys from the first (type 2)
 };
 
 struct ItemInfo {
@@ -87,6 +87,10 @@ struct DecInfo {
   int tg;      // tiles of this CTA's earlier items
   int flags1;  // halves that use half 0's column tiles (3 when both halves share a query block)
   int cc[2], cb[2];  // column count / first column of each half
+  // slash runs (VS_WINDOWS heads): per half, the interval list of its query
+  // block's height (an index into dist), its length, the block's last row, and
+  // the run tiles it gives (half 1 has none when both halves share the block)
+  int rbeg[2], rn[2], rr1[2], rt[2];
 };
 
 struct AttnArgs {
@@ -346,7 +350,31 @@ static __device__ __noinline__ void drain_loads(uint64_t* bars, const int* misc,
   }
 }
 
-template <int D>
+// The run tiles of one slash-run list (VS_WINDOWS): interval [a, b] of offsets
+// is the key run [max(0, r1 - b), r1 - a], cut into 64-key tiles from its first
+// key.  Threads tid0, tid0 + nt, ... share the intervals; returns their share.
+__device__ __forceinline__ int run_tiles(const int32_t* iv, int n, int r1, int tid0, int nt) {
+  int c = 0;
+  for (int k = tid0; k < n; k += nt) {
+    const int hi = r1 - iv[2 * k], lo = max(0, r1 - iv[2 * k + 1]);
+    if (hi >= lo) c += (hi - lo) / UNIT + 1;
+  }
+  return c;
+}
+
+// Key j lies in one of the runs of a list (offset intervals [a_k, b_k],
+// ascending, of a block whose last row is r1) iff r1 - j falls in an interval.
+__device__ __forceinline__ bool key_in_runs(const int32_t* iv, int n, int r1, int j) {
+  const int d = r1 - j;
+  int lo = 0, hi = n;  // first interval with a > d
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (iv[2 * mid] <= d) lo = mid + 1; else hi = mid;
+  }
+  return lo > 0 && d <= iv[2 * (lo - 1) + 1];
+}
+
+template <int D, bool RUNS>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
@@ -472,6 +500,49 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           pv[b] = g;
           for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, di.kvh);
         }
+        if constexpr (RUNS) {
+          // slash-run tiles (VS_WINDOWS): 64 keys from any first key, TMA boxes
+          // at that key row; half 0's runs (both halves' when they share the
+          // query block), then half 1's
+          int t = di.T_u;
+          for (int hh = 0; ok && hh < 2; ++hh) {
+            if (di.rt[hh] == 0) continue;
+            const int32_t* iv = a.dist + di.rbeg[hh];
+            const int fl = hh == 0 ? di.flags1 : 2;
+            for (int k = 0; ok && k < di.rn[hh]; ++k) {
+              const int hi = di.rr1[hh] - iv[2 * k], lo = max(0, di.rr1[hh] - iv[2 * k + 1]);
+              for (int st = lo; ok && st <= hi; st += UNIT, ++t) {
+                const int g = di.tg + t;
+                const int b = g & 1;
+                const uint32_t use = (g >> 1) & 1;
+                if (!mbar_wait_ool(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+                                   kLoaderSuspend)) {
+                  ok = false;
+                  break;
+                }
+                StageInfo& si = info[g % NINFO];
+                si.type = 2;
+                si.u = st;
+                si.flags = fl;
+                si.ncols = min(UNIT, hi - st + 1);
+                mbar_arrive(&bars[B_INFO + g % NINFO]);
+                uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
+                uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
+                mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
+                pk[b] = g;
+                for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, st, di.kvh);
+                if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
+                                   kLoaderSuspend)) {
+                  ok = false;
+                  break;
+                }
+                mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
+                pv[b] = g;
+                for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, st, di.kvh);
+              }
+            }
+          }
+        }
         if (!ok) break;
         mbar_arrive(&bars[B_UNITS]);  // this item's bitmaps are no longer read here
       }
@@ -501,6 +572,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         misc[10] = next_item;
         next_item = (int)gridDim.x + sched_next(a.sched, a.epoch);  // fetched one item ahead
         misc[3] = 0;
+        if constexpr (RUNS) {
+          misc[4] = 0;
+          misc[5] = 0;
+        }
       }
       named_barrier(1, 64);
       const int item = misc[10];
@@ -562,7 +637,38 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         uint32_t* bb = hh ? b1 : b0;
         const int qb = qbh[hh];
         const int r1 = r1h[hh];
-        if (kind == DSA_KIND_VS) {
+        if (kind == DSA_KIND_VS_WINDOWS) {
+          if constexpr (RUNS) {
+            // the slash runs of the half's query block (both halves share them
+            // when they share the block): count their 64-key tiles
+            if (hh == 1 && shared_qb) continue;
+            int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
+            checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
+            int n = 0, nl = 0;
+            if (end - beg >= 2) {
+              n = a.dist[beg];
+              nl = a.dist[beg + 1];
+            }
+            if (end - beg < 2 || n < 0 || nl < 0 || 2 + 2 * ((int64_t)n + nl) != end - beg) {
+              report_bad_row(a.status, DETAIL_BAD_DISTPTR);
+              n = nl = 0;
+            }
+            const bool lastb = qb == a.nqb - 1;
+            const int r1b = min(a.N - 1, qb * a.B + a.B - 1);
+            const int off = beg + 2 + (lastb ? 2 * n : 0);
+            const int m = lastb ? nl : n;
+            int c = run_tiles(a.dist + off, m, r1b, dtid, 64);
+            c = warp_sum_int(c);
+            if (lane == 0 && c) atomicAdd(&misc[4 + hh], c);
+            if (dtid == 0) {
+              dec[s].rbeg[hh] = off;
+              dec[s].rn[hh] = m;
+              dec[s].rr1[hh] = r1b;
+            }
+          } else {
+            report_bad_row(a.status, DETAIL_BAD_KIND);  // this build's kernel has no run tiles
+          }
+        } else if (kind == DSA_KIND_VS) {
           int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
           checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
           for (int e = beg + dtid; e < end; e += 64) {
@@ -602,6 +708,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         di.T_u = misc[3];  // one tile per unit
         di.flags1 = shared_qb ? 3 : 1;
         di.T = di.T_u + ceil_div(di.cc[0], BN) + ceil_div(di.cc[1], BN);
+        if constexpr (RUNS) {
+          const bool wins = kind == DSA_KIND_VS_WINDOWS;
+          di.rt[0] = wins && live[0] ? misc[4] : 0;
+          di.rt[1] = wins && live[1] && !shared_qb ? misc[5] : 0;
+          if (!wins || !live[0]) di.rn[0] = 0;
+          if (!wins || !live[1]) di.rn[1] = 0;
+          if (wins && shared_qb) {  // half 1 reads the block's runs through half 0's tiles
+            di.rbeg[1] = di.rbeg[0];
+            di.rn[1] = di.rn[0];
+            di.rr1[1] = di.rr1[0];
+          }
+          di.T += di.rt[0] + di.rt[1];
+        }
         di.tg = tg_dec;
         // publish the item (its slot is free once both consumers read item kc - 2)
         const int slot = kc & 1;
@@ -639,6 +758,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       named_barrier(1, 64);
       if (misc[9] == 0) { go = false; return; }
       int t = di.T_u;
+      if constexpr (RUNS) t += di.rt[0] + di.rt[1];
       for (int hh = 0; go && hh < 2; ++hh) {
         const int nt = ceil_div(di.cc[hh], BN);
         const int cflags = hh ? 2 : di.flags1;
@@ -682,7 +802,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 int v = j;
                 if (j >= 0) {
                   const int u = j / UNIT;
-                  const int cov = (int)((b0[u >> 5] >> (u & 31)) & 1u) | ((int)((b1[u >> 5] >> (u & 31)) & 1u) << 1);
+                  int cov = (int)((b0[u >> 5] >> (u & 31)) & 1u) | ((int)((b1[u >> 5] >> (u & 31)) & 1u) << 1);
+                  if constexpr (RUNS) {
+                    // a column inside a slash run of the half counts once
+                    if (di.rn[0] > 0 && key_in_runs(a.dist + di.rbeg[0], di.rn[0], di.rr1[0], j)) cov |= 1;
+                    if (di.rn[1] > 0 && key_in_runs(a.dist + di.rbeg[1], di.rn[1], di.rr1[1], j)) cov |= 2;
+                  }
                   v = j | (cov << 24);
                 }
                 cj[slot] = v;
@@ -833,7 +958,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tmem_ld32(s_t + 32, s + 32);
         // allowed-key bits of this row, 32 columns per word
         uint32_t mw[2];
-        if (si.type == 0) {
+        if (RUNS && si.type == 2) {
+          // keys si.u .. si.u + ncols - 1 of the half's runs, causal
+          const int lim = (si.flags & hbit) ? min(si.ncols, row - si.u + 1) : 0;
+          mw[0] = low_bits(lim);
+          mw[1] = low_bits(lim - 32);
+        } else if (si.type == 0) {
           const bool oks = (si.flags & hbit) != 0;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -1045,7 +1175,7 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int H, int64_t t
   return r == CUDA_SUCCESS;
 }
 
-template <int D>
+template <int D, bool RUNS>
 dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const void* V, const dsa_indices& idx,
                     void* O, float* lse, cudaStream_t stream, unsigned* status) {
   CUtensorMap mq, mk, mv;
@@ -1090,7 +1220,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   int smem = Smem<D>::bytes(a.nwords);
   // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, RUNS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   const int n_items = a.n_qtiles * p.Hq;
   if (n_items == 0) return DSA_OK;
@@ -1100,7 +1230,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = n_items < 2 * sms ? n_items : 2 * sms;
-  e = launch_pdl(sparse_attn_kernel<D>, dim3(grid), dim3(NTHREADS), (size_t)smem, stream, mq, mk, mv, a);
+  e = launch_pdl(sparse_attn_kernel<D, RUNS>, dim3(grid), dim3(NTHREADS), (size_t)smem, stream, mq, mk, mv, a);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;
@@ -1115,8 +1245,15 @@ bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int N, int 
 
 dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K, const void* V,
                               const dsa_indices& idx, void* O, float* lse, cudaStream_t stream, unsigned* status) {
-  if (p.d == 128) return launch_d<128>(p, Q, K, V, idx, O, lse, stream, status);
-  if (p.d == 64) return launch_d<64>(p, Q, K, V, idx, O, lse, stream, status);
+  // the kernel with slash-run tiles only when a VS_WINDOWS head is present: the
+  // other kinds keep the smaller code of the plain one
+  const bool runs = (idx.kinds_present >> DSA_KIND_VS_WINDOWS) & 1;
+  if (p.d == 128)
+    return runs ? launch_d<128, true>(p, Q, K, V, idx, O, lse, stream, status)
+                : launch_d<128, false>(p, Q, K, V, idx, O, lse, stream, status);
+  if (p.d == 64)
+    return runs ? launch_d<64, true>(p, Q, K, V, idx, O, lse, stream, status)
+                : launch_d<64, false>(p, Q, K, V, idx, O, lse, stream, status);
   return DSA_ERR_UNSUPPORTED;
 }
 

@@ -25,7 +25,7 @@ enum : unsigned {
   DETAIL_WAIT_SELFTEST = 9,
   DETAIL_CAP_BLK = 20, DETAIL_CAP_COL = 21, DETAIL_CAP_DIST = 22,
   DETAIL_BAD_BLOCK = 30, DETAIL_BAD_COL = 31, DETAIL_BAD_DIST = 32,
-  DETAIL_BAD_BLKPTR = 33, DETAIL_BAD_COLPTR = 34, DETAIL_BAD_DISTPTR = 35,
+  DETAIL_BAD_BLKPTR = 33, DETAIL_BAD_COLPTR = 34, DETAIL_BAD_DISTPTR = 35, DETAIL_BAD_KIND = 36,
 };
 
 __device__ __forceinline__ void report(unsigned* status, unsigned code, unsigned detail) {

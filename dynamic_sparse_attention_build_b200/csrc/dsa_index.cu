@@ -69,11 +69,15 @@ struct ConvTab {
 };
 
 struct Layout {
-  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_chunk, vs_nchunks, vs_lmax, nuh, sel_ri, sel_nx;
+  int Hq, Hkv, G, N, d, B, nqb, nkw, nbh, nvs, vs_chunk, vs_nchunks, vs_lmax, nuh, sel_ri, sel_nx, dtmp_stride;
   int64_t off_kbar, off_sel, off_v, off_s, off_part, off_stat, off_dtmp, off_dbits, off_spart, off_upart, total;
 };
 
 __host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) & ~int64_t(255); }
+
+// Vertical-Slash kinds: the estimate and its top-k are shared; they differ in
+// how the chosen slashes are covered (aligned blocks, or exact per-block runs).
+__host__ __device__ inline bool is_vs_kind(int k) { return k == DSA_KIND_VS || k == DSA_KIND_VS_WINDOWS; }
 
 // order-preserving float -> uint32 key
 __device__ __forceinline__ uint32_t fkey(float f) {
@@ -236,7 +240,7 @@ __global__ void k_head_info(const __grid_constant__ HeadTab ht, int Hq, int32_t*
   const int h = blockIdx.x * blockDim.x + threadIdx.x;
   if (h >= Hq) return;
   if (h == 0) dist_ptr[0] = 0;
-  if (ht.kind[h] != DSA_KIND_VS) dist_ptr[1 + h] = 0;
+  if (!is_vs_kind(ht.kind[h])) dist_ptr[1 + h] = 0;
   head_info[h * 4 + 0] = ht.kind[h];
   head_info[h * 4 + 1] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.sink[h] : 0;
   head_info[h * 4 + 2] = ht.kind[h] == DSA_KIND_ASHAPE ? ht.window[h] : 0;
@@ -263,8 +267,8 @@ __global__ void k_ashape_count(const __grid_constant__ HeadTab ht, Layout L, int
     blk_ptr[0] = 0;
     col_ptr[0] = 0;
   }
-  if (kind != DSA_KIND_VS) col_ptr[1 + h * L.nqb + qb] = 0;
-  if (kind == DSA_KIND_VS) blk_ptr[1 + h * L.nqb + qb] = 0;
+  if (!is_vs_kind(kind)) col_ptr[1 + h * L.nqb + qb] = 0;
+  if (is_vs_kind(kind)) blk_ptr[1 + h * L.nqb + qb] = 0;
   if (kind != DSA_KIND_ASHAPE) return;
   int a, w;
   ashape_range(qb, L.B, L.N, ht.sink[h], ht.window[h], &a, &w);
@@ -1141,37 +1145,53 @@ k_vs_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtenso
         const int jlim = min(j1, jt + VT_ROWS) - 1;  // the sub-tile's last key
         const bool nomask = jlim <= i0[wslot] && jt + VT_ROWS <= j1;
         const int ilim = i0[wslot] + rbase;  // row of column c is ilim + c
-        float v = 0.f, dacc = 0.f;
+        // two independent chains (columns 0..31 and 32..63) halve the serial
+        // shuffle chain: chain A holds diagonals t = 0..62 (win[t]), chain B
+        // t = 32..94 (win[64 + t - 32]); the merge adds both
+        float va = 0.f, vb = 0.f, da = 0.f, db = 0.f;
         const float4* rm4 = reinterpret_cast<const float4*>(rowm + VT_HALF * ch);
 #pragma unroll
-        for (int c4 = 0; c4 < VT_HALF / 4; ++c4) {
-          const float4 m4 = rm4[c4];
-          const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 ma = rm4[c4], mb = rm4[8 + c4];
+          const float mma[4] = {ma.x, ma.y, ma.z, ma.w}, mmb[4] = {mb.x, mb.y, mb.z, mb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int c = c4 * 4 + e;
-            const bool ok_ij = nomask || (kv && j <= ilim + c);
-            const float p = ok_ij ? ex2_approx(fmaf(x[c], sc, -mm[e])) : 0.f;
-            v += p;
-            dacc += p;
-            if (lane == 31) win[c] = dacc;          // diagonal t = c is complete
-            if (c + 1 < VT_HALF) {
-              dacc = __shfl_up_sync(0xffffffffu, dacc, 1);
-              if (lane == 0) dacc = 0.f;            // diagonal t = c + 32 starts
+            const bool oka = nomask || (kv && j <= ilim + c);
+            const bool okb = nomask || (kv && j <= ilim + 32 + c);
+            const float pa = oka ? ex2_approx(fmaf(x[c], sc, -mma[e])) : 0.f;
+            const float pb = okb ? ex2_approx(fmaf(x[32 + c], sc, -mmb[e])) : 0.f;
+            va += pa;
+            vb += pb;
+            da += pa;
+            db += pb;
+            if (lane == 31) {  // diagonals t = c (chain A) and t = 32 + c (chain B) are complete
+              win[c] = da;
+              win[64 + c] = db;
+            }
+            if (c + 1 < 32) {
+              da = __shfl_up_sync(0xffffffffu, da, 1);
+              db = __shfl_up_sync(0xffffffffu, db, 1);
+              if (lane == 0) da = db = 0.f;  // diagonals t = c + 32, c + 64 start
             }
           }
         }
-        if (lane < 31) win[VT_HALF + 30 - lane] = dacc;  // diagonals t = 64 .. 94
+        if (lane < 31) {  // chain A: t = 32 .. 62; chain B: t = 64 .. 94
+          win[62 - lane] = da;
+          win[64 + 62 - lane] = db;
+        }
+        const float v = va + vb;
+        float vtot = v;
         if (LP != 64) {
           // one head over both column halves: the two warps of a quadrant add
           // their key sums in a fixed order (half 0 + half 1)
           if (ch == 1) vsum[lr] = v;
           named_barrier(1, VT_COMPUTE);
-          if (ch == 0) v += vsum[lr];
+          if (ch == 0) vtot = v + vsum[lr];
         }
         if (kv && (LP == 64 ? hs[wslot] >= 0 : ch == 0)) {
           float* vout = reinterpret_cast<float*>(ws + L.off_v);
-          vout[(int64_t)vsl[wslot] * L.N + j] = v;
+          vout[(int64_t)vsl[wslot] * L.N + j] = LP == 64 ? v : vtot;
         }
         named_barrier(1, VT_COMPUTE);
         // merge the warps' windows into the chunk window in a fixed order.
@@ -1192,7 +1212,8 @@ k_vs_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtenso
             if (ws_ != s) continue;
             const int rb = LP == 64 ? 0 : VT_HALF * wch;
             const int tw = idx - (base + rb - 32 * wq);
-            if (tw >= 0 && tw < VT_WW) acc += wins[w * VT_WW + tw];
+            if (tw >= 0 && tw <= 62) acc += wins[w * VT_WW + tw];            // chain A
+            if (tw >= 32 && tw <= 94) acc += wins[w * VT_WW + 64 + tw - 32];  // chain B
           }
           cwin[s * (CHK + VT_ROWS) + idx] = acc;
         }
@@ -1315,6 +1336,67 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
 // slashes.  One flag byte per key block (plain stores: every writer writes 1),
 // then one bitmap word per 32 blocks from a warp ballot, and the ascending list
 // from a scan of the per-word counts.  Dynamic shared memory: nkw * 32 bytes.
+// Slash runs of a VS_WINDOWS head (MInference summary, "3つの疎パターン": slash
+// lines).  Query block qb (rows r0..r1, height L) reaches on slash o the keys
+// i - o for r0 <= i <= r1, i >= o: the window [r0 - o, r1 - o] clipped at key 0,
+// i.e. the offset interval [o, o + L - 1] mirrored at r1.  Windows of slashes
+// closer than L + 1 touch, so a block's runs are the merged intervals of the
+// dilated offsets, mirrored: one list per block height (every block has height
+// B except a shorter last one).  Output (n, n_last = intervals of the two
+// heights): out[0] = n, out[1] = n_last, out[2 + 2k] = a_k, out[3 + 2k] = b_k
+// (k < n, ascending, disjoint, not touching), then the n_last intervals of the
+// last block's height the same way; *len = 2 + 2 (n + n_last).  S (ascending, -1 padded) is the head's slash list.
+// One CTA of up to 1024 threads.
+__device__ void vs_runs(const HeadTab& ht, const Layout& L, const int32_t* S, int32_t* out, int32_t* len) {
+  __shared__ int scan[96];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  const int h = ht.vhead[blockIdx.x];
+  const int ns = min(ht.n_slash[h], L.N);
+  const int last_h = L.N - (L.nqb - 1) * L.B;  // height of the last block
+  int pos = 2;
+  for (int pass = 0; pass < 2; ++pass) {
+    const int Lh = pass == 0 ? L.B : last_h;
+    int base = 0;  // intervals so far in this pass
+    for (int k0 = 0; k0 < ns; k0 += blockDim.x) {
+      const int k = k0 + tid;
+      const int o = k < ns ? S[k] : -1;
+      const int op = (k > 0 && k < ns) ? S[k - 1] : -1;
+      const bool valid = o >= 0;
+      // a new interval starts where the previous window ends more than one key
+      // away: o > o_prev + L
+      const bool start = valid && (k == 0 || op < 0 || o > op + Lh);
+      const int on = (k + 1 < ns) ? S[k + 1] : -1;
+      const bool end = valid && (k + 1 >= ns || on < 0 || on > o + Lh);
+      // block-wide exclusive scan of `start`
+      const unsigned bal = __ballot_sync(0xffffffffu, start);
+      if (lane == 0) scan[warp] = __popc(bal);
+      __syncthreads();
+      if (warp == 0) {
+        int c = lane < nw ? scan[lane] : 0;
+        int incl = c;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, d);
+          if (lane >= d) incl += y;
+        }
+        if (lane < nw) scan[32 + lane] = incl - c;
+        if (lane == 31) scan[64] = incl;
+      }
+      __syncthreads();
+      // interval index of k: intervals started before this chunk + those started
+      // at or before k in it, minus one (k lies in the last one started)
+      const int id = base + scan[32 + warp] + __popc(bal & ((2u << lane) - 1u)) - 1;
+      if (start) out[pos + 2 * id] = o;
+      if (end) out[pos + 2 * id + 1] = o + Lh - 1;
+      base += scan[64];
+      __syncthreads();
+    }
+    if (tid == 0) out[pass] = base;
+    pos += 2 * base;
+  }
+  if (tid == 0) *len = pos;
+}
+
 __global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                   const int32_t* slash_idx, int slash_stride, int32_t* dist_ptr) {
   pdl_prologue();
@@ -1323,8 +1405,12 @@ __global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTa
   const int vslot = blockIdx.x;
   const int h = ht.vhead[vslot];
   uint32_t* dbits = reinterpret_cast<uint32_t*>(ws + L.off_dbits) + (int64_t)vslot * L.nkw;
-  int32_t* dtmp = reinterpret_cast<int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.nqb;
+  int32_t* dtmp = reinterpret_cast<int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.dtmp_stride;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  if (ht.kind[h] == DSA_KIND_VS_WINDOWS) {
+    vs_runs(ht, L, slash_idx + (int64_t)h * slash_stride, dtmp, dist_ptr + 1 + h);
+    return;
+  }
   for (int i = threadIdx.x; i < L.nkw * 8; i += blockDim.x) reinterpret_cast<uint32_t*>(flag)[i] = 0u;
   __syncthreads();
   const int ns = min(ht.n_slash[h], L.N);
@@ -1369,6 +1455,22 @@ __global__ void __launch_bounds__(1024) k_vs_dist(const __grid_constant__ HeadTa
   }
 }
 
+// Key j lies in a slash run of query block qb (last row r1) iff r1 - j falls in
+// one of the block height's offset intervals (vs_runs layout; the last block
+// may be shorter and has its own list): a binary search over ascending a_k.
+__device__ __forceinline__ bool in_runs(const int32_t* runs, bool last_block, int r1, int j) {
+  const int n = runs[0], n_last = runs[1];
+  const int32_t* iv = runs + 2 + (last_block ? 2 * n : 0);
+  const int m = last_block ? n_last : n;
+  const int d = r1 - j;
+  int lo = 0, hi = m;  // first interval with a > d
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (iv[2 * mid] <= d) lo = mid + 1; else hi = mid;
+  }
+  return lo > 0 && d <= iv[2 * (lo - 1) + 1];
+}
+
 // columns of (VS head, query block): j in V, j <= qb*B+B-1, (qb - j/B) not in D.
 // One warp per query block, eight per CTA; the CTA stages the D bitmap and a
 // window of the (ascending) vertical list in shared memory once for its warps.
@@ -1392,7 +1494,12 @@ __global__ void __launch_bounds__(256) k_vs_cols(const __grid_constant__ HeadTab
   const int32_t* V = vert_idx + (int64_t)h * vert_stride;
   const int nv = min(ht.n_vert[h], L.N);
   const int lim = qb * L.B + L.B - 1;
+  const int lim_r1 = min(L.N - 1, lim);  // the block's last row
   const int row = h * L.nqb + qb;
+  // VS_WINDOWS: the head's run intervals (vs_runs) replace the distance bitmap
+  const int32_t* runs = ht.kind[h] == DSA_KIND_VS_WINDOWS
+                            ? reinterpret_cast<const int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.dtmp_stride
+                            : nullptr;
   bool active = qb < L.nqb;
   int pos = 0;
   if (FILL && active) {
@@ -1413,8 +1520,12 @@ __global__ void __launch_bounds__(256) k_vs_cols(const __grid_constant__ HeadTab
         const int j = (t < cn) ? vwin[t] : -1;
         bool take = false;
         if (j >= 0 && j <= lim) {
-          const int delta = qb - j / L.B;
-          take = !((dsh[delta >> 5] >> (delta & 31)) & 1u);
+          if (runs != nullptr) {
+            take = !in_runs(runs, qb == L.nqb - 1, lim_r1, j);
+          } else {
+            const int delta = qb - j / L.B;
+            take = !((dsh[delta >> 5] >> (delta & 31)) & 1u);
+          }
         }
         const unsigned m = __ballot_sync(0xffffffffu, take);
         if (FILL && take) col_idx[pos + __popc(m & ((1u << lane) - 1u))] = j;
@@ -1472,7 +1583,7 @@ __global__ void k_blk_fill(const __grid_constant__ HeadTab ht, Layout L, const u
   pdl_prologue();
   const int h = blockIdx.y;
   const int kind = ht.kind[h];
-  if (kind == DSA_KIND_VS) return;
+  if (is_vs_kind(kind)) return;
   const int qb = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (qb >= L.nqb) return;
@@ -1525,7 +1636,7 @@ __global__ void k_dist_fill(const __grid_constant__ HeadTab ht, Layout L, const 
     if (threadIdx.x == 0) report(status, DSA_ERR_CAPACITY, DETAIL_CAP_DIST);
     return;
   }
-  const int32_t* dtmp = reinterpret_cast<const int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.nqb;
+  const int32_t* dtmp = reinterpret_cast<const int32_t*>(ws + L.off_dtmp) + (int64_t)vslot * L.dtmp_stride;
   for (int t = threadIdx.x; t < end - beg; t += blockDim.x) dist[beg + t] = dtmp[t];
 }
 
@@ -1584,7 +1695,16 @@ __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head
     if (threadIdx.x == 0) report(status, DSA_ERR_DEVICE, detail);
     return false;
   };
-  if (kind == DSA_KIND_VS) {
+  const int32_t* runs = nullptr;  // VS_WINDOWS: the head's run intervals
+  if (kind == DSA_KIND_VS_WINDOWS) {
+    const int beg = dist_ptr[h], end = dist_ptr[h + 1];
+    const bool ok = row_ok(beg, end, dist_cap, DETAIL_BAD_DISTPTR) && end - beg >= 2 &&
+                    2 + 2 * ((int64_t)dist[beg] + dist[beg + 1]) == end - beg;
+    if (!ok && end - beg >= 0 && threadIdx.x == 0) report(status, DSA_ERR_DEVICE, DETAIL_BAD_DISTPTR);
+    runs = ok ? dist + beg : nullptr;
+    lst = dist;
+    nl = 0;
+  } else if (kind == DSA_KIND_VS) {
     const int beg = dist_ptr[h], end = dist_ptr[h + 1];
     const bool ok = row_ok(beg, end, dist_cap, DETAIL_BAD_DISTPTR);
     lst = ok ? dist + beg : dist;
@@ -1609,13 +1729,29 @@ __global__ void k_count_pairs(int Hq, int N, int B, int nqb, const int32_t* head
       tot += (int64_t)nrows * (nrows + 1) / 2;
     }
   }
+  if (runs != nullptr) {
+    // run [lo, hi] (keys) of this block: row i counts min(i, hi) - lo + 1 keys
+    // when i >= lo, all hi - lo + 1 once i > hi
+    const bool lastb = qb == nqb - 1;
+    const int nr = lastb ? runs[1] : runs[0];
+    const int32_t* iv = runs + 2 + (lastb ? 2 * runs[0] : 0);
+    for (int k = threadIdx.x; k < nr; k += blockDim.x) {
+      const int hi = r1 - iv[2 * k], lo = max(0, r1 - iv[2 * k + 1]);
+      if (hi < lo) continue;
+      const int64_t x0 = max(r0, lo) - lo + 1, x1 = min(r1, hi) - lo + 1;
+      if (x1 >= x0) tot += (x0 + x1) * (x1 - x0 + 1) / 2;
+      const int64_t full_rows = max(0, r1 - max(r0, hi + 1) + 1);
+      tot += full_rows * (hi - lo + 1);
+    }
+  }
   int cb = col_ptr[h * nqb + qb], ce = col_ptr[h * nqb + qb + 1];
   if (!row_ok(cb, ce, col_cap, DETAIL_BAD_COLPTR)) cb = ce = 0;
   for (int e = cb + threadIdx.x; e < ce; e += blockDim.x) {
     const int j = col_idx[e];
     if (j < 0 || j > r1) continue;
     const int kb = j / B;
-    const bool covered = dsel ? sorted_contains(lst, nl, qb - kb) : sorted_contains(lst, nl, kb);
+    const bool covered = runs != nullptr ? in_runs(runs, qb == nqb - 1, r1, j)
+                                         : (dsel ? sorted_contains(lst, nl, qb - kb) : sorted_contains(lst, nl, kb));
     if (covered) continue;
     tot += r1 - max(j, r0) + 1;
   }
@@ -1641,6 +1777,7 @@ dsa_status check_pattern(const dsa_problem& p, const dsa_pattern& q) {
       if (q.sink < 0 || q.window < 1) return DSA_ERR_INVALID_ARG;
       return DSA_OK;
     case DSA_KIND_VS:
+    case DSA_KIND_VS_WINDOWS:
       if (q.last_q < 1 || q.n_vert < 0 || q.n_slash < 0) return DSA_ERR_INVALID_ARG;
       if (q.last_q > VS_MAXL) return DSA_ERR_UNSUPPORTED;
       return DSA_OK;
@@ -1700,6 +1837,7 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   L->nbh = 0;
   L->nvs = 0;
   L->nuh = 0;
+  L->dtmp_stride = ceil_div(p.N, p.block);
   L->sel_ri = sel_blocks_per_cta(p.block);
   L->sel_nx = ceil_div(L->nqb, L->sel_ri);
   L->vs_lmax = 0;
@@ -1778,7 +1916,14 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
       const int nv = std::min(q.n_vert, N), ns = std::min(q.n_slash, N);
       vstride = std::max(vstride, nv);
       sstride = std::max(sstride, ns);
-      dcap += std::min<int64_t>(2 * (int64_t)ns, nqb);
+      if (q.kind == DSA_KIND_VS_WINDOWS) {
+        // run list: [n, n_last, then n (a, b) offset intervals for full blocks,
+        // then n_last for a shorter last block], each at most ns intervals
+        dcap += 2 + 4 * (int64_t)ns;
+        L->dtmp_stride = std::max<int>(L->dtmp_stride, 2 + 4 * ns);
+      } else {
+        dcap += std::min<int64_t>(2 * (int64_t)ns, nqb);
+      }
       for (int qb = 0; qb < nqb; ++qb) ccap += std::min<int64_t>(nv, (int64_t)qb * B + B);
       L->vs_lmax = std::max(L->vs_lmax, 16 * vs_rows_pad(std::min(q.last_q, N)));
     }
@@ -1799,7 +1944,7 @@ dsa_status make_layout(const dsa_problem& p, const dsa_pattern* pats, Layout* L,
   }
   L->off_part = off; off = align256(off + (int64_t)L->nvs * vs_parts * VS_MAXL * 2 * 4);
   L->off_stat = off; off = align256(off + (int64_t)L->nvs * VS_MAXL * 2 * 4);
-  L->off_dtmp = off; off = align256(off + (int64_t)L->nvs * nqb * 4);
+  L->off_dtmp = off; off = align256(off + (int64_t)L->nvs * L->dtmp_stride * 4);
   L->off_dbits = off; off = align256(off + (int64_t)L->nvs * L->nkw * 4);
   // per-chunk windows of the slash sums (chunk + VS_MAXL offsets each)
   L->off_spart = off; off = align256(off + (int64_t)L->nvs * vs_wins * 4);
@@ -1830,7 +1975,7 @@ void make_vs_tiles(const HeadTab& ht, const Layout& L, VsTiles* vt) {
   for (int g = 0; g < L.Hkv; ++g) {
     int pend = -1;  // a head of <= 64 rows waiting for a partner
     for (int h = g * L.G; h < (g + 1) * L.G; ++h) {
-      if (ht.kind[h] != DSA_KIND_VS) continue;
+      if (!is_vs_kind(ht.kind[h])) continue;
       const int lq = std::min(ht.last_q[h], L.N);
       if (lq > 64) {
         vt->h0[vt->n] = h, vt->h1[vt->n] = -1, vt->lp[vt->n] = VT_ROWS, vt->n++;

@@ -65,8 +65,10 @@ typedef enum dsa_kind {
     DSA_KIND_BLOCK_TOPK = 2,      /* MInference block-sparse: top-k pooled block scores, J <= I */
     DSA_KIND_BLOCK_THRESHOLD = 3, /* FlashPrefill: P_IJ >= alpha * max_J P_IJ, plus sink/local */
     DSA_KIND_MOBA = 4,            /* MoBA: top-k over J < I plus the own block I */
-    DSA_KIND_UNIFIED = 5          /* FlashPrefill discovery: vertical, diagonal and block
+    DSA_KIND_UNIFIED = 5,         /* FlashPrefill discovery: vertical, diagonal and block
                                      shapes at once from the pooled block scores */
+    DSA_KIND_VS_WINDOWS = 6       /* Vertical-Slash whose slashes are covered by their exact
+                                     key runs per query block instead of aligned blocks */
 } dsa_kind;
 
 /*
@@ -143,7 +145,16 @@ typedef struct dsa_pattern {
  *                                 UNIFIED heads (ascending, -1 padded).
  *   slash_idx [Hq * slash_stride]: chosen slash offsets o = i - j of VS heads, diagonal block
  *                                 distances d of UNIFIED heads (ascending, -1 padded).
- * dsa_sparse_prefill reads only head_info, blk_*, dist*, col_*.
+ * VS_WINDOWS heads keep no blocks; their dist row is the slash-run list
+ *   [n, n_last, a_0, b_0, ..., a_{n-1}, b_{n-1}, then n_last pairs]: the merged offset
+ *   intervals [a, b] of the chosen slashes dilated by the block height (the first
+ *   n for full blocks, the last n_last for a shorter last block); query block qb
+ *   (last row r1) keeps the key runs [max(0, r1 - b), r1 - a].  Their columns lie
+ *   outside those runs.
+ * kinds_present: bit k set when some head has kind k.  dsa_sparse_prefill reads it
+ *   to choose its kernel (a VS_WINDOWS head met without bit 6 is reported as
+ *   DSA_ERR_DEVICE and left empty); dsa_build_indices does not read it.
+ * dsa_sparse_prefill reads only head_info, blk_*, dist*, col_*, kinds_present.
  */
 typedef struct dsa_indices {
     int32_t* head_info;
@@ -157,6 +168,8 @@ typedef struct dsa_indices {
     int32_t* slash_idx;
     int64_t blk_cap, dist_cap, col_cap;
     int32_t vert_stride, slash_stride;
+    int32_t kinds_present;  /* bit k set when some head has kind k (dsa_kind) */
+    int32_t reserved;
 } dsa_indices;
 
 /* Sizes for one (problem, patterns) pair: element counts of every index array

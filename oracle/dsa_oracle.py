@@ -69,7 +69,8 @@ BLOCK_TOPK = "block_topk"
 BLOCK_THRESHOLD = "block_threshold"
 MOBA = "moba"
 UNIFIED = "unified"
-KINDS = (ASHAPE, VS, BLOCK_TOPK, BLOCK_THRESHOLD, MOBA, UNIFIED)
+VS_WINDOWS = "vs_windows"   # VS with slash_cover="windows"
+KINDS = (ASHAPE, VS, BLOCK_TOPK, BLOCK_THRESHOLD, MOBA, UNIFIED, VS_WINDOWS)
 
 
 def n_blocks(N: int, B: int) -> int:
@@ -325,6 +326,9 @@ def build_head_index(Qh, Kh, pattern: dict, B: int, conv=None) -> HeadIndex:
     N, d = Kh.shape
     nqb = n_blocks(N, B)
     kind = pattern["kind"]
+    if kind == VS_WINDOWS:
+        pattern = dict(pattern, kind=VS, slash_cover="windows")
+        kind = VS
     hi = HeadIndex(kind=kind, B=B, N=N)
     empty = np.zeros(0, np.int64)
     if kind == ASHAPE:

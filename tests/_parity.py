@@ -20,7 +20,10 @@ def oracle_heads_to_lists(heads):
         d = dict(kind=hi.kind, sink=hi.sink, window=hi.window,
                  blocks=[np.asarray(b) for b in hi.blocks],
                  cols=[np.asarray(c) for c in hi.cols])
-        if hi.kind == orc.VS:
+        if hi.kind == orc.VS and hi.runs is not None:
+            d["kind"] = "vs_windows"
+            d["dist"] = runs_list_from_slashes(hi.S, hi.B, hi.N)
+        elif hi.kind == orc.VS:
             d["dist"] = np.asarray(hi.D)
         out.append(d)
     return out
@@ -29,12 +32,16 @@ def oracle_heads_to_lists(heads):
 def gpu_lists_to_oracle_heads(bufs, N, B):
     """Library index buffers -> oracle HeadIndex objects (VS blocks rebuilt from D
     with the oracle's own rule, so the oracle evaluates exactly the GPU's mask)."""
-    kinds = {0: orc.ASHAPE, 1: orc.VS, 2: orc.BLOCK_TOPK, 3: orc.BLOCK_THRESHOLD, 4: orc.MOBA, 5: orc.UNIFIED}
+    kinds = {0: orc.ASHAPE, 1: orc.VS, 2: orc.BLOCK_TOPK, 3: orc.BLOCK_THRESHOLD, 4: orc.MOBA, 5: orc.UNIFIED,
+             6: orc.VS}
     heads = []
     nqb = (N + B - 1) // B
     for hl in bufs.host_lists():
         hi = orc.HeadIndex(kind=kinds[hl["kind"]], B=B, N=N, sink=hl["sink"], window=hl["window"])
-        if hi.kind == orc.VS:
+        if hl["kind"] == 6:
+            hi.runs = [runs_of_block(hl["dist"], qb, B, N) for qb in range(nqb)]
+            hi.blocks = [np.zeros(0, np.int64)] * nqb
+        elif hi.kind == orc.VS:
             D = np.asarray(hl["dist"], np.int64)
             hi.D = D
             hi.blocks = [np.sort(qb - D[D <= qb]) for qb in range(nqb)]
@@ -43,6 +50,38 @@ def gpu_lists_to_oracle_heads(bufs, N, B):
         hi.cols = [np.asarray(c, np.int64) for c in hl["cols"]]
         heads.append(hi)
     return heads
+
+
+def runs_list_from_slashes(S, B, N):
+    """The library's slash-run list of a VS_WINDOWS head from its slash offsets
+    S: [n, n_last, then (a, b) offset intervals [o, o + L - 1] merged when they
+    overlap or touch, for blocks of height B, then for the last block's height]."""
+    S = np.sort(np.asarray(S, np.int64))
+    nqb = (N + B - 1) // B
+    out = []
+    counts = []
+    for L in (B, N - (nqb - 1) * B):
+        iv = []
+        for o in S:
+            if iv and o <= iv[-1][1] + 1:
+                iv[-1][1] = max(iv[-1][1], int(o) + L - 1)
+            else:
+                iv.append([int(o), int(o) + L - 1])
+        counts.append(len(iv))
+        out += [x for p in iv for x in p]
+    return np.asarray(counts + out, np.int64)
+
+
+def runs_of_block(lst, qb, B, N):
+    """Key runs [first, last] (ascending) of query block qb from a slash-run list."""
+    lst = np.asarray(lst, np.int64)
+    n, n_last = int(lst[0]), int(lst[1])
+    nqb = (N + B - 1) // B
+    last = qb == nqb - 1
+    iv = lst[2 + (2 * n if last else 0): 2 + 2 * n + (2 * n_last if last else 0)].reshape(-1, 2)
+    r1 = min(N - 1, qb * B + B - 1)
+    runs = [[max(0, r1 - b), r1 - a] for a, b in iv if r1 - a >= 0]
+    return np.asarray(sorted(runs), np.int64).reshape(-1, 2)
 
 
 def to64(t):

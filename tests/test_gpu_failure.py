@@ -80,7 +80,8 @@ def _clone_bufs(dsa, bufs):
                         head_info=bufs.head_info.clone(), blk_ptr=bufs.blk_ptr.clone(),
                         blk_idx=bufs.blk_idx.clone(), dist_ptr=bufs.dist_ptr.clone(), dist=bufs.dist.clone(),
                         col_ptr=bufs.col_ptr.clone(), col_idx=bufs.col_idx.clone(),
-                        vert_idx=bufs.vert_idx.clone(), slash_idx=bufs.slash_idx.clone())
+                        vert_idx=bufs.vert_idx.clone(), slash_idx=bufs.slash_idx.clone(),
+                        kinds_present=bufs.kinds_present)
 
 
 @pytest.mark.parametrize("which", ["blk_past_cap", "blk_negative", "col_past_cap", "col_reversed", "dist_past_cap"])

@@ -12,8 +12,8 @@ import torch
 
 import synth
 from oracle import dsa_oracle as orc
-from tests._parity import (assert_close_outputs, assert_lse_close, gpu_lists_to_oracle_heads,
-                           threshold_set_ok, to64, topk_set_ok)
+from tests._parity import (assert_close_outputs, assert_lse_close, gpu_lists_to_oracle_heads, runs_list_from_slashes,
+                           runs_of_block, threshold_set_ok, to64, topk_set_ok)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,6 +45,18 @@ def check_indices(bufs, ref_heads, pats, N, B, convs_ref=None):
             assert list(g["dist"]) == list(D), f"head {h} distances"
             for qb in range(nqb):
                 want = orc.vs_columns(np.asarray(g["vert"], np.int64), D, qb, B)
+                assert list(g["cols"][qb]) == list(want), (h, qb)
+        elif kind == "vs_windows":
+            ok, msg = topk_set_ok(g["vert"], r.V, r.vscore, p["n_vert"])
+            assert ok, f"head {h} verticals: {msg}"
+            ok, msg = topk_set_ok(g["slash"], r.S, r.sscore, p["n_slash"])
+            assert ok, f"head {h} slashes: {msg}"
+            S = np.asarray(g["slash"], np.int64)
+            assert list(g["dist"]) == list(runs_list_from_slashes(S, B, N)), f"head {h} run list"
+            for qb in range(nqb):
+                runs = runs_of_block(g["dist"], qb, B, N)
+                assert np.array_equal(runs, orc.vs_slash_runs(S, qb, B, N)), (h, qb)
+                want = orc.vs_window_columns(np.asarray(g["vert"], np.int64), runs, qb, B)
                 assert list(g["cols"][qb]) == list(want), (h, qb)
         elif kind == "unified":
             # the kept verticals and diagonals against the oracle's (tie-aware at
@@ -135,6 +147,25 @@ def test_mixed_gqa_ragged(dsa):
             dict(kind="block_topk", topk=100),
             dict(kind="vs", last_q=128, n_vert=0, n_slash=1),
             dict(kind="ashape", sink=0, window=1)]
+    run(dsa, Q, K, V, pats, B)
+
+
+@pytest.mark.parametrize("B", [64, 128])
+def test_vs_windows(dsa, B):
+    """Vertical-Slash heads whose slashes are covered by their exact key runs per
+    query block (tiles of 64 keys from any first key) next to every other kind in
+    one layer (the kernel with run tiles then serves them all), with few, many and
+    clustered slashes, a ragged length and GQA."""
+    N, d = 1400, 128
+    Q, K, V = synth.random_qkv(8, 2, N, d, seed=51 + B)
+    pats = [dict(kind="vs_windows", last_q=64, n_vert=40, n_slash=3),
+            dict(kind="vs_windows", last_q=32, n_vert=200, n_slash=300),
+            dict(kind="ashape", sink=70, window=200),
+            dict(kind="vs", last_q=64, n_vert=50, n_slash=20),
+            dict(kind="block_topk", topk=3),
+            dict(kind="vs_windows", last_q=100, n_vert=0, n_slash=40),
+            dict(kind="block_threshold", alpha=0.5),
+            dict(kind="unified", alpha=0.6)]
     run(dsa, Q, K, V, pats, B)
 
 

@@ -493,3 +493,15 @@ def test_unified_finds_planted_vertical_and_diagonal(rng):
     assert 7 in vert and 3 in diag
     for I in range(10, n):
         assert {0, 7, I - 3, I} <= set(blocks[I])
+
+
+def test_runs_list_helpers_match_the_oracle_runs(rng):
+    """The test helpers that read the library's slash-run lists (offset intervals
+    merged at the block height, mirrored at a block's last row) give exactly the
+    oracle's runs for every query block, ragged last block included."""
+    from tests._parity import runs_list_from_slashes, runs_of_block
+    for N, B, ns in ((300, 16, 7), (257, 32, 40), (100, 64, 3), (1000, 64, 200)):
+        S = np.sort(rng.choice(N, size=ns, replace=False))
+        lst = runs_list_from_slashes(S, B, N)
+        for qb in range((N + B - 1) // B):
+            assert np.array_equal(runs_of_block(lst, qb, B, N), orc.vs_slash_runs(S, qb, B, N)), (N, B, qb)
