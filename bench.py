@@ -103,10 +103,10 @@ def algorithmic_index_bytes(w, pats):
     byt = 0
     kv_read = set()
     for h, p in enumerate(pats):
-        if p["kind"] in ("block_topk", "block_threshold", "moba"):
+        if p["kind"] in ("block_topk", "block_threshold", "moba", "unified"):
             byt += N * d * 2
             kv_read.add(h // G)
-        elif p["kind"] == "vs":
+        elif p["kind"] in ("vs", "vs_windows"):
             byt += min(p["last_q"], N) * d * 2 + 2 * 2 * 4 * N
             kv_read.add(h // G)
     byt += len(kv_read) * N * d * 2
@@ -158,6 +158,53 @@ def build_workload(w, device, seed_offset=0):
         G = w["Hq"] // w["Hkv"]
         pats = [dict(p, conv=convs[h // G]) if p["kind"] == "moba" else p for h, p in enumerate(pats)]
     return Q, K, V, pats
+
+
+def key_tiles_per_item(bufs, N, B):
+    """64-key tiles the attention kernel runs per 128-row item, from the index
+    lists, the kernel's own tiling: per item the union of its two 64-row halves'
+    64-key units of listed blocks, plus each half's slash-run tiles (64 keys from
+    each run's first key) and gathered column tiles (a half that shares its query
+    block with the other adds none of its own); averaged over items."""
+    nqb = (N + B - 1) // B
+    tiles = items = 0
+    for hl in bufs.host_lists():
+        for r0 in range(0, N, 128):
+            units = set()
+            t = 0
+            seen = set()
+            for hh in (0, 1):
+                rs = r0 + 64 * hh
+                if rs >= N:
+                    continue
+                qb, r1h = rs // B, min(N - 1, rs + 63)
+                if hl["kind"] == 1:
+                    blocks = [qb - int(dd) for dd in hl["dist"] if dd <= qb]
+                elif hl["kind"] == 6:
+                    blocks = []
+                else:
+                    blocks = [int(x) for x in hl["blocks"][qb]]
+                for kb in blocks:
+                    for u in range(kb * B // 64, (kb * B + B) // 64):
+                        if u * 64 <= r1h:
+                            units.add(u)
+                if qb in seen:
+                    continue
+                seen.add(qb)
+                if hl["kind"] == 6:
+                    lst = hl["dist"]
+                    n, nl = int(lst[0]), int(lst[1])
+                    last = qb == nqb - 1
+                    iv = lst[2 + (2 * n if last else 0): 2 + 2 * n + (2 * nl if last else 0)].reshape(-1, 2)
+                    r1 = min(N - 1, qb * B + B - 1)
+                    for a, b in iv:
+                        hi, lo = r1 - int(a), max(0, r1 - int(b))
+                        if hi >= lo:
+                            t += (hi - lo) // 64 + 1
+                t += (len(hl["cols"][qb]) + 63) // 64
+            tiles += t + len(units)
+            items += 1
+    return tiles / max(1, items)
 
 
 def kernel_launches_per_step(pats):
@@ -247,6 +294,8 @@ def build_arg_parser():
     ap.add_argument("--N", type=int, default=0, help="override the token count (smaller profiling cases)")
     ap.add_argument("--B", type=int, default=0, help="override the block size (the MoBA workload's B sweep)")
     ap.add_argument("--conv", type=int, default=-1, help="override the MoBA key-conv width (0 = off)")
+    ap.add_argument("--slash-cover", default="blocks", choices=["blocks", "windows"],
+                    help="VS heads: cover the slashes by aligned key blocks or by their exact key runs")
     ap.add_argument("--shard-heads", action="store_true",
                     help="strong scaling: the ranks split ONE layer by KV groups (default: one layer per rank)")
     ap.add_argument("--gather", action="store_true",
@@ -303,6 +352,8 @@ def main():
         import datetime
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=dev)
+    if args.slash_cover == "windows":
+        w = dict(w, name=w["name"] + "_slash_runs")
     if args.shard_heads:
         # every rank builds the same layer and keeps its KV groups (heads are independent)
         from dynamic_sparse_attention_build_b200 import shard
@@ -312,6 +363,8 @@ def main():
     else:
         Q, K, V, pats = build_workload(w, dev, seed_offset=rank)
     N, Hq, d = w["N"], Q.shape[0], w["d"]
+    if args.slash_cover == "windows":
+        pats = [dict(p, kind="vs_windows") if p["kind"] == "vs" else p for p in pats]
     gather = args.shard_heads and args.gather and world > 1
     pats_c = dsa.make_patterns(pats)
     bufs = dsa.build_indices(Q, K, pats_c, w["B"])
@@ -322,6 +375,7 @@ def main():
     if st != 0:
         raise RuntimeError(f"device status {st} detail {det}")
     pairs = dsa.count_pairs(Q, K, bufs).sum().item()
+    tiles_item = key_tiles_per_item(bufs, N, w["B"]) if N <= 65536 else None
     f_sel = 4.0 * d * pairs
     causal_pairs = Hq * N * (N + 1) / 2
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -419,6 +473,7 @@ def main():
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "strong" if args.shard_heads else "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w["name"], "Hq": Hq, "Hkv": w["Hkv"], "N": N, "d": d, "block": w["B"],
+                   "slash_cover": args.slash_cover,
                    "key_conv_width": int(w.get("conv_width", 0) or 0),
                    "patterns": PATTERN_TEXT.get(w["mix"], w["mix"]),
                    "l2": "flushed by a 256 MiB write before every timed step (outside its events)",
@@ -431,6 +486,7 @@ def main():
                      "work": f"F_sel = 4*d*|M| = {f_sel:.4e} FLOP per launch ({pairs} allowed pairs)"},
         "attention": {"ms": ms_attn, "tflops": tflops, "frac_peak": tflops / peak_tf,
                       "frac_sustained_peak": (tflops / peak_sus) if peak_sus else None,
+                      "key_tiles_per_item": tiles_item,
                       "density_vs_causal": pairs / causal_pairs},
         "index_build": {"ms": ms_build, "algorithmic_bytes": idx_bytes, "gbs": idx_gbs,
                         "frac_hbm": idx_gbs / pk["hbm_gbs"], "hbm_peak_source": pk_src},

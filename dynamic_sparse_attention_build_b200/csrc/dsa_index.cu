@@ -23,6 +23,8 @@
 
 #include <algorithm>
 
+#include <cooperative_groups.h>
+
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 
@@ -773,7 +775,6 @@ __global__ void __launch_bounds__(1024) k_unified_merge(const __grid_constant__ 
   uint32_t* vb = reinterpret_cast<uint32_t*>(um + 2 * nqb);  // [nkw] vertical bits
   uint32_t* db = vb + L.nkw;                                  // [nkw] diagonal bits
   __shared__ float red[2][32];
-  __shared__ int cnt[2][32];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* up = reinterpret_cast<const float*>(ws + L.off_upart) + (int64_t)uslot * L.sel_nx * 2 * nqb;
   float mv = 0.f, mg = 0.f;
@@ -1305,31 +1306,200 @@ __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint
   }
 }
 
-// exact top-k of v (blockIdx.y == 0) or s (== 1) of one VS head, ascending, -1 padded
+// Exact top-k of v (blockIdx.y == 0) or s (== 1) of one VS head, ascending, -1
+// padded: one cluster of 1 to VT_CL CTAs per (head, array), each CTA owning a
+// contiguous segment (one CTA for short arrays, where the cluster's exchanges
+// cost more than its bandwidth gains).  Three radix passes of 12, 12 and 8 bits: each CTA counts
+// its segment's keys that match the prefix so far into its own 4096-bin
+// histogram; CTA 0 of the cluster adds the cluster's histograms through
+// distributed shared memory, finds the digit holding the k-th key and hands it
+// to every CTA.  Then each CTA counts its keys above the k-th and equal to it,
+// learns the counts of the CTAs before it (again through distributed shared
+// memory) and writes its selected keys at their ascending positions (ties go to
+// the lower index, as in the CTA-wide select).  The histogram increments are
+// aggregated per warp (one atomic per distinct bin): the first pass's 12 bits
+// are the sign, the exponent and 3 mantissa bits, so most keys share a few bins.
+constexpr int VT_CL = 8;
+
+// CTAs per top-k cluster for arrays of n keys
+inline int vs_topk_cluster(int n) { return n <= (1 << 16) ? 1 : (n <= (1 << 18) ? 4 : VT_CL); }
+
+template <typename Loader, typename Emit>
+__device__ void ordered_select_range(const Loader& load, int beg_all, int end_all, uint32_t T, int take_eq,
+                                     int eq_base0, int out_base0, int* red, const Emit& emit) {
+  const int nw = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n = end_all - beg_all;
+  const int seg = ceil_div(ceil_div(max(n, 1), nw), 32) * 32;
+  const int beg = beg_all + min(n, warp * seg), end = beg_all + min(n, warp * seg + seg);
+  int gt = 0, eq = 0;
+  for (int i = beg + lane; i < end; i += 32) {
+    const uint32_t key = fkey(load(i));
+    gt += key > T;
+    eq += key == T;
+  }
+  gt = warp_sum_int(gt);
+  eq = warp_sum_int(eq);
+  if (lane == 0) {
+    red[2 * warp] = gt;
+    red[2 * warp + 1] = eq;
+  }
+  __syncthreads();
+  int eq_run = eq_base0, gt_before = 0;
+  for (int w = 0; w < warp; ++w) {
+    gt_before += red[2 * w];
+    eq_run += red[2 * w + 1];
+  }
+  __syncthreads();
+  int pos = out_base0 + gt_before + min(eq_run, take_eq) - min(eq_base0, take_eq);
+  for (int i0 = beg; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    const uint32_t key = i < end ? fkey(load(i)) : 0u;
+    const bool iseq = i < end && key == T;
+    bool sel = i < end && key > T;
+    const unsigned eqm = __ballot_sync(0xffffffffu, iseq);
+    if (iseq && eq_run + __popc(eqm & ((1u << lane) - 1u)) < take_eq) sel = true;
+    eq_run += __popc(eqm);
+    const unsigned sm = __ballot_sync(0xffffffffu, sel);
+    if (sel) emit(i, pos + __popc(sm & ((1u << lane) - 1u)));
+    pos += __popc(sm);
+  }
+}
+
 __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTab ht, Layout L, uint8_t* ws,
                                                   int32_t* vert_idx, int vert_stride, int32_t* slash_idx,
                                                   int slash_stride) {
   pdl_prologue();
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
   __shared__ int hist[RADIX_BINS];
   __shared__ int red[80];
-  const int vslot = blockIdx.x;
+  __shared__ int xfer[4];  // from CTA 0: digit, keys above it; segment counts gt, eq
+  const int rank = (int)cluster.block_rank();
+  const int ncl = (int)cluster.num_blocks();
+  const int vslot = blockIdx.x / ncl;
   const int which = blockIdx.y;
   const int h = ht.vhead[vslot];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const float* arr = reinterpret_cast<const float*>(ws + (which == 0 ? L.off_v : L.off_s)) + (int64_t)vslot * L.N;
   const int k = min(which == 0 ? ht.n_vert[h] : ht.n_slash[h], L.N);
   int32_t* out = which == 0 ? vert_idx + (int64_t)h * vert_stride : slash_idx + (int64_t)h * slash_stride;
   const int stride = which == 0 ? vert_stride : slash_stride;
-  for (int i = k + threadIdx.x; i < stride; i += blockDim.x) out[i] = -1;
-  if (k <= 0) return;
-  auto load = [&](int i) { return arr[i]; };
+  const int seg = ceil_div(ceil_div(L.N, ncl), 32) * 32;
+  const int beg = min(L.N, rank * seg), end = min(L.N, beg + seg);
+  for (int i = k + rank * blockDim.x + tid; i < stride; i += ncl * blockDim.x) out[i] = -1;
+  if (k <= 0) return;  // the whole cluster leaves together (k is the same for all)
   if (k >= L.N) {
-    for (int i = threadIdx.x; i < L.N; i += blockDim.x) out[i] = i;
+    for (int i = beg + tid; i < end; i += blockDim.x) out[i] = i;
     return;
   }
-  uint32_t T;
-  int take_eq;
-  radix_kth(load, L.N, k, hist, red, &T, &take_eq);
-  ordered_select(load, L.N, T, take_eq, red, [&](int i, int pos) { out[pos] = i; });
+  uint32_t prefix = 0, mask = 0;
+  int need = k;
+  for (int pass = 0; pass < 3; ++pass) {
+    const int shift = pass == 0 ? 20 : (pass == 1 ? 8 : 0);
+    const uint32_t dmask = pass == 2 ? 0xffu : 0xfffu;
+    for (int i = tid; i < RADIX_BINS; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    for (int i0 = beg; i0 < end; i0 += RB * blockDim.x) {
+      uint32_t key[RB];
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        const int i = i0 + q * blockDim.x + tid;
+        key[q] = (i < end) ? fkey(arr[i]) : 0u;
+      }
+#pragma unroll
+      for (int q = 0; q < RB; ++q) {
+        const int i = i0 + q * blockDim.x + tid;
+        const bool act = i < end && (key[q] & mask) == prefix;
+        const unsigned am = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const int bin = (int)((key[q] >> shift) & dmask);
+          const unsigned same = __match_any_sync(am, bin);
+          if ((same & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(same));
+        }
+      }
+    }
+    cluster.sync();  // every CTA's histogram is complete
+    if (rank == 0) {
+      // add the other CTAs' histograms into this one, then find the digit:
+      // thread t takes bins RADIX_BINS-1-t*bpt downwards; an exclusive scan of
+      // the per-thread sums is the count of keys in higher bins
+      for (int r = 1; r < ncl; ++r) {
+        const int* rh = cluster.map_shared_rank(hist, r);
+        for (int i = tid; i < RADIX_BINS; i += blockDim.x) hist[i] += rh[i];
+      }
+      __syncthreads();
+      const int bpt = RADIX_BINS / blockDim.x;
+      const int top = RADIX_BINS - 1 - tid * bpt;
+      int tot = 0;
+      for (int q = 0; q < bpt; ++q) tot += hist[top - q];
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (lane == 31) red[2 + warp] = incl;
+      __syncthreads();
+      int above = incl - tot;
+      for (int w = 0; w < warp; ++w) above += red[2 + w];
+      if (above < need && above + tot >= need) {
+        for (int q = 0; q < bpt; ++q) {
+          const int c = hist[top - q];
+          if (above + c >= need) {
+            for (int r = 0; r < ncl; ++r) {
+              int* rx = cluster.map_shared_rank(xfer, r);
+              rx[0] = top - q;
+              rx[1] = above;
+            }
+            break;
+          }
+          above += c;
+        }
+      }
+    }
+    cluster.sync();  // the digit is in every CTA's xfer; CTA 0 is done reading histograms
+    prefix |= (uint32_t)xfer[0] << shift;
+    mask |= dmask << shift;
+    need -= xfer[1];
+  }
+  const uint32_t T = prefix;
+  const int take_eq = need;
+  // counts of this CTA's segment, shared with the cluster
+  int gt = 0, eq = 0;
+  for (int i = beg + tid; i < end; i += blockDim.x) {
+    const uint32_t key = fkey(arr[i]);
+    gt += key > T;
+    eq += key == T;
+  }
+  gt = warp_sum_int(gt);
+  eq = warp_sum_int(eq);
+  if (lane == 0) {
+    red[2 * warp] = gt;
+    red[2 * warp + 1] = eq;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int g = 0, e = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+      g += red[2 * w];
+      e += red[2 * w + 1];
+    }
+    xfer[2] = g;
+    xfer[3] = e;
+  }
+  cluster.sync();
+  int gt_before = 0, eq_before = 0;
+  for (int r = 0; r < rank; ++r) {
+    const int* rx = cluster.map_shared_rank(xfer, r);
+    gt_before += rx[2];
+    eq_before += rx[3];
+  }
+  cluster.sync();  // no CTA leaves while another may still read its counts
+  __syncthreads();
+  auto load = [&](int i) { return arr[i]; };
+  ordered_select_range(load, beg, end, T, take_eq, eq_before, gt_before + min(eq_before, take_eq), red,
+                       [&](int i, int pos) { out[pos] = i; });
 }
 
 // block distances D of one VS head: {floor(o/B), ceil(o/B)} for the chosen
@@ -2086,8 +2256,9 @@ dsa_status launch_build_indices(const dsa_problem& p, const void* Q, const void*
     s = (p.d == 128) ? launch_vs<128>(ht, vt, L, p, Q, K, ws, st, status)
                      : launch_vs<64>(ht, vt, L, p, Q, K, ws, st, status);
     if (s != DSA_OK) return s;
-    DSA_CK(launch_pdl(k_vs_topk, dim3(L.nvs, 2), dim3(1024), 0, st, ht, L, ws, out.vert_idx, out.vert_stride,
-                      out.slash_idx, out.slash_stride));
+    const int ncl = vs_topk_cluster(p.N);
+    DSA_CK(launch_pdl_cluster(k_vs_topk, dim3(L.nvs * ncl, 2), dim3(1024), ncl, st, ht, L, ws, out.vert_idx,
+                              out.vert_stride, out.slash_idx, out.slash_stride));
     DSA_CK(launch_pdl(k_vs_dist, dim3(L.nvs), dim3(1024), (size_t)L.nkw * 32, st, ht, L, ws, out.slash_idx,
                       out.slash_stride, out.dist_ptr));
     DSA_CK(launch_pdl(k_vs_cols<false>, dim3(ceil_div(L.nqb, 8), L.nvs), dim3(256), 0, st, ht, L, ws, out.vert_idx,

@@ -242,3 +242,28 @@ def test_index_build_is_deterministic(dsa):
                  "slash_idx"):
         assert torch.equal(getattr(a, name), getattr(b, name)), name
     assert any(p["kind"] == "vs" for p in pats)
+
+
+@pytest.mark.parametrize("N", [70000, 300001])
+def test_vs_topk_multi_cta(dsa, N):
+    """The VS top-k runs as a cluster of CTAs for long arrays (4 CTAs above 65,536
+    keys, 8 above 262,144), each owning a contiguous segment: the selected sets
+    against the oracle's scores (tie-aware), ascending, for a large k, a small k
+    and k at the array length's scale; two builds give identical lists."""
+    pats = [dict(kind="vs", last_q=64, n_vert=1000, n_slash=6096), dict(kind="vs", last_q=32, n_vert=3, n_slash=1),
+            dict(kind="vs", last_q=64, n_vert=5000, n_slash=N - 5)]
+    Q, K, _ = synth.random_qkv(3, 1, N, 128, seed=N % 97)
+    Qd, Kd = Q.cuda(), K.cuda()
+    a = dsa.build_indices(Qd, Kd, pats, 64)
+    b = dsa.build_indices(Qd, Kd, pats, 64)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == (0, 0)
+    assert torch.equal(a.vert_idx, b.vert_idx) and torch.equal(a.slash_idx, b.slash_idx)
+    lists = a.host_lists()
+    k64 = to64(K[0])
+    for h, p in enumerate(pats):
+        v, s = orc.vs_estimate(to64(Q[h]), k64, p["last_q"])
+        for got, sc, k in ((lists[h]["vert"], v, p["n_vert"]), (lists[h]["slash"], s, p["n_slash"])):
+            assert len(got) == k and np.all(np.diff(got) > 0), (h, k)
+            ok, msg = topk_set_ok(got, orc.topk_indices(sc, k), sc, k)
+            assert ok, f"head {h}, k {k}: {msg}"
