@@ -878,13 +878,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const uint32_t use = (g >> 1) & 1;
             if (!mbar_wait_ool(&bars[B_KFULL + b], use, limit, a.status, DETAIL_WAIT_K, abort_flag, kMmaSuspend)) { ok = false; break; }
             seen[11] = g + 1;
-            // the buffer still holds P(g-2) until that P.V has finished; its
-            // V-empty commit says so (a per-buffer barrier: at an item boundary
-            // P(g-1) V(g-1) has been issued too, so B_ODONE could be two phases on)
-            if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_O, abort_flag, kMmaSuspend)) {
-              ok = false;
-              break;
-            }
+            // the buffer still holds P(g-2), which P(g-2) V(g-2) reads; that
+            // product was issued by this thread before this one, and the
+            // tensor core runs one thread's MMAs in issue order, so its reads of
+            // P precede this product's writes of S without a wait here
             tc_fence_after();
             mma_qk_tile<D / 16>(tmem_base + S_COL + 64 * b, q_desc, b ? k_desc1 : k_desc0, IDESC_QK);
             tc_commit(&bars[B_SFULL + b]);
