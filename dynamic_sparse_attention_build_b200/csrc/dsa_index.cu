@@ -292,15 +292,16 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // h = c / 2 (sigmoid(c) = (1 + tanh(c / 2)) / 2): one tanh.approx (relative error
 // about 2^-11, far below what routing on pooled keys can see) instead of an
 // exponential and a division; the halving is folded into the weights and bias.
-template <int W>
+// sw: the head's weights as [W][D] and its bias as [D], halved, in shared memory.
+template <int W, int D>
 __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts, int c0, int r0, int r1,
-                                              const float* cw, const float* cb, float* acc) {
+                                              const float* sw, float* acc) {
   float wt[W][8], bias[8], win[W][8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    bias[i] = 0.5f * cb[c0 + i];
+    bias[i] = sw[W * D + c0 + i];
 #pragma unroll
-    for (int t = 0; t < W; ++t) wt[t][i] = 0.5f * cw[(c0 + i) * W + t];
+    for (int t = 0; t < W; ++t) wt[t][i] = sw[t * D + c0 + i];
   }
   // before row r is shifted in, win[t] = k[r - 1 - t] (t < W - 1); after the
   // shift win[t] = k[r - t].  Rows before 0 are zero (causal, zero padded).
@@ -313,15 +314,26 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
 #pragma unroll
     for (int i = 0; i < 8; ++i) win[t][i] = __bfloat162float(e[i]);
   }
+  // software pipelined: the next four rows are in flight while these four are
+  // computed
+  uint4 nxt[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    nxt[u] = (r0 + u < r1) ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r0 + u) * ts + c0))
+                           : make_uint4(0, 0, 0, 0);
   for (int r = r0; r < r1; r += 4) {
     uint4 raw[4];
 #pragma unroll
-    for (int u = 0; u < 4; ++u)
-      raw[u] = (r + u < r1) ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r + u) * ts + c0))
-                            : make_uint4(0, 0, 0, 0);
+    for (int u = 0; u < 4; ++u) {
+      raw[u] = nxt[u];
+      nxt[u] = (r + 4 + u < r1) ? __ldg(reinterpret_cast<const uint4*>(X + (int64_t)(r + 4 + u) * ts + c0))
+                                : make_uint4(0, 0, 0, 0);
+    }
+    // rows past r1 (the run's last step) are computed and dropped: no branch
+    // between the four rows, so their chains overlap
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      if (r + u >= r1) break;
+      const float keep = (r + u < r1) ? 1.f : 0.f;
 #pragma unroll
       for (int t = W - 1; t > 0; --t) {
 #pragma unroll
@@ -335,7 +347,7 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
         float h = bias[i];
 #pragma unroll
         for (int t = 0; t < W; ++t) h = fmaf(wt[t][i], win[t][i], h);
-        acc[i] += win[0][i] + fmaf(h, tanh_approx(h), h);
+        acc[i] = fmaf(keep, win[0][i] + fmaf(h, tanh_approx(h), h), acc[i]);
       }
     }
   }
@@ -344,29 +356,38 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
 // ---------------------------------------------------------------------------
 // key mean pooling (+ optional causal depthwise key conv with SiLU and residual)
 // ---------------------------------------------------------------------------
-// grid: (nqb, Hkv); KV heads that no block head reads are skipped.  Queries are
-// pooled inside k_block_select.  CW = 0: plain mean, for the KV heads without a
-// key conv; CW = W in 1..8: the conv of width W, for the KV heads with that
-// width (one launch per width present, so each instantiation holds exactly the
-// registers its width needs).
+// grid: (ceil(nqb / bpc), Hkv); KV heads that no block head reads are skipped.
+// Queries are pooled inside k_block_select.  CW = 0: plain mean, for the KV heads
+// without a key conv, one block per CTA (bpc = 1); CW = W in 1..8: the conv of
+// width W, for the KV heads with that width (one launch per width present, so
+// each instantiation holds exactly the registers its width needs), bpc blocks
+// per CTA (see conv_blocks_per_cta).
 template <int D, int CW>
 __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct, Layout L,
-                                              const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws) {
+                                              const __nv_bfloat16* K, int64_t k_hs, int64_t k_ts, uint8_t* ws,
+                                              int bpc) {
   pdl_prologue();
   constexpr int TPR = D / 8;          // threads per row, 8 channels each
   constexpr int RG = 256 / TPR;       // rows in flight
   __shared__ float part[RG][D];
-  const int b = blockIdx.x;
+  __shared__ float sw[CW > 0 ? (CW + 1) * D : 1];  // conv weights [CW][D] and bias [D], halved
+  const int b0 = blockIdx.x * bpc;  // the CTA's first block
   const int kvh = blockIdx.y;
   if (!ct.need[kvh] || ct.width[kvh] != CW) return;
+  if constexpr (CW > 0) {
+    // coalesced: consecutive threads read consecutive weights (stored [D][CW])
+    for (int i = threadIdx.x; i < CW * D; i += blockDim.x) sw[(i % CW) * D + i / CW] = 0.5f * ct.w[kvh][i];
+    for (int i = threadIdx.x; i < D; i += blockDim.x) sw[CW * D + i] = 0.5f * ct.b[kvh][i];
+    __syncthreads();
+  }
   const __nv_bfloat16* X = K + kvh * k_hs;
   const int64_t ts = k_ts;
-  // the pooled row as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
-  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b) * 2 * D;
+  // pooled rows as bf16 hi[D] then lo[D], hi + lo ~ the fp32 mean
+  __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(ws + L.off_kbar) + ((int64_t)kvh * L.nqb + b0) * 2 * D;
   const int rg = threadIdx.x / TPR;
   const int c0 = (threadIdx.x % TPR) * 8;
-  const int r_beg = b * L.B;
-  const int r_end = min(L.N, r_beg + L.B);
+  const int r_beg = b0 * L.B;
+  const int r_end = min(L.N, r_beg + bpc * L.B);
   float acc[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -391,24 +412,37 @@ __global__ void __launch_bounds__(256) k_pool(const __grid_constant__ ConvTab ct
       for (int i = 0; i < 8; ++i) acc[i] += __bfloat162float(e[i]);
     }
   } else {
-    // each row group takes a contiguous run of the block's rows (the conv window
-    // slides along it)
-    const int run = (r_end - r_beg + RG - 1) / RG;
+    // each row group takes a contiguous run of rows (the conv window slides along
+    // it); with several blocks per CTA the runs tile the blocks exactly, so each
+    // run lies in one block
+    const int run = ceil_div(bpc * L.B, RG);
     const int r0 = min(r_end, r_beg + rg * run), r1 = min(r_end, r0 + run);
-    conv_rows_sum<CW>(X, ts, c0, r0, r1, ct.w[kvh], ct.b[kvh], acc);
+    conv_rows_sum<CW, D>(X, ts, c0, r0, r1, sw, acc);
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) part[rg][c0 + i] = acc[i];
   __syncthreads();
   if (threadIdx.x < D) {
-    float s = 0.f;
-    for (int g = 0; g < RG; ++g) s += part[g][threadIdx.x];
-    const float x = s / (float)(r_end - r_beg);
-    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
-    out[threadIdx.x] = hi;
-    out[D + threadIdx.x] = __float2bfloat16_rn(x - __bfloat162float(hi));
+    const int gpb = RG / bpc;  // row groups per block
+    for (int j = 0; j < bpc; ++j) {
+      const int rows = min(L.N, r_beg + (j + 1) * L.B) - (r_beg + j * L.B);
+      if (rows <= 0) break;
+      float s = 0.f;
+      for (int g = j * gpb; g < (j + 1) * gpb; ++g) s += part[g][threadIdx.x];
+      const float x = s / (float)rows;
+      const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+      out[(int64_t)j * 2 * D + threadIdx.x] = hi;
+      out[(int64_t)j * 2 * D + D + threadIdx.x] = __float2bfloat16_rn(x - __bfloat162float(hi));
+    }
   }
 }
+
+// Blocks per CTA of the conv pooling: enough for 512 rows when the block size
+// divides 512 (32-row runs per row group: the W - 1 rows before each run are
+// loaded again, and the CTA's set-up is paid once per 512 rows), else one.
+// bpc divides the row groups (16 for d = 128, 32 for d = 64), so a block is an
+// exact number of runs.
+inline int conv_blocks_per_cta(int B) { return (B < 512 && 512 % B == 0) ? 512 / B : 1; }
 
 // the plain pooling for the KV heads without a conv and one launch per conv width present
 template <int D>
@@ -417,17 +451,15 @@ cudaError_t launch_pool(const ConvTab& ct, const Layout& L, const __nv_bfloat16*
   bool has[9] = {};
   for (int h = 0; h < L.Hkv; ++h)
     if (ct.need[h]) has[ct.width[h] < 0 || ct.width[h] > 8 ? 0 : ct.width[h]] = true;
-  const dim3 grid(L.nqb, L.Hkv), block(256);
+  const int bpc = conv_blocks_per_cta(L.B);
+  const dim3 grid(L.nqb, L.Hkv), cgrid(ceil_div(L.nqb, bpc), L.Hkv), block(256);
   cudaError_t e = cudaSuccess;
-  if (has[0]) e = launch_pdl(k_pool<D, 0>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[1]) e = launch_pdl(k_pool<D, 1>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[2]) e = launch_pdl(k_pool<D, 2>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[3]) e = launch_pdl(k_pool<D, 3>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[4]) e = launch_pdl(k_pool<D, 4>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[5]) e = launch_pdl(k_pool<D, 5>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[6]) e = launch_pdl(k_pool<D, 6>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[7]) e = launch_pdl(k_pool<D, 7>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
-  if (e == cudaSuccess && has[8]) e = launch_pdl(k_pool<D, 8>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws);
+  if (has[0]) e = launch_pdl(k_pool<D, 0>, grid, block, 0, st, ct, L, k, k_hs, k_ts, ws, 1);
+#define DSA_CONV_POOL(W) \
+  if (e == cudaSuccess && has[W]) e = launch_pdl(k_pool<D, W>, cgrid, block, 0, st, ct, L, k, k_hs, k_ts, ws, bpc);
+  DSA_CONV_POOL(1) DSA_CONV_POOL(2) DSA_CONV_POOL(3) DSA_CONV_POOL(4)
+  DSA_CONV_POOL(5) DSA_CONV_POOL(6) DSA_CONV_POOL(7) DSA_CONV_POOL(8)
+#undef DSA_CONV_POOL
   return e;
 }
 
@@ -453,10 +485,7 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, const uint32_t* a, uint
 }
 
 constexpr int SEL_RI = 16;  // query blocks per CTA
-#ifndef DSA_SEL_NT
-#define DSA_SEL_NT 512
-#endif
-constexpr int SEL_NT = DSA_SEL_NT;  // threads per CTA
+constexpr int SEL_NT = 512;  // threads per CTA
 constexpr int SEL_NW = SEL_NT / 32;
 // score row stride in floats: 8 past a multiple of 32 so the 8-byte stores of
 // one half-warp (rows g..g+3, columns 2 t4) hit 16 distinct bank pairs

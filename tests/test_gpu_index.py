@@ -198,6 +198,28 @@ def test_moba(dsa, B, conv):
         rows=np.r_[0:64, 500:600, w["N"] - 200:w["N"]])
 
 
+@pytest.mark.parametrize("d", [64, 128])
+def test_moba_conv_widths(dsa, d):
+    """Each key-conv width has its own pooling instantiation: five KV heads with
+    widths 1, 3, 5 and 8 and one without a conv (five launches), non-zero biases,
+    a ragged last block, and runs of rows that start inside the previous block
+    (the causal window reaches back across the block boundary)."""
+    N, B = 1100, 128
+    widths = [1, 3, 5, 8, 0]
+    Q, K, V = synth.random_qkv(5, 5, N, d, seed=77 + d)
+    g = torch.Generator().manual_seed(5 + d)
+    convs = [None if W == 0 else (torch.randn(d, W, generator=g) * 0.5, torch.randn(d, generator=g) * 0.3)
+             for W in widths]
+    pats = [dict(kind="moba", topk=3) for _ in widths]
+    dpats = [dict(p, conv=(c[0].cuda(), c[1].cuda())) if c is not None else p for p, c in zip(pats, convs)]
+    bufs = dsa.build_indices(Q.cuda(), K.cuda(), dpats, B)
+    torch.cuda.synchronize()
+    assert dsa.device_status() == (0, 0)
+    oconvs = [None if c is None else (c[0].double().numpy(), c[1].double().numpy()) for c in convs]
+    ref = orc.build_indices(to64(Q), to64(K), pats, B, oconvs)
+    check_indices(bufs, ref, pats, N, B)
+
+
 def test_threshold_topics(dsa):
     w = synth.workload(3, N=4096, Hq=4, Hkv=2)
     Q, K, V, planted = synth.make_inputs(w)
