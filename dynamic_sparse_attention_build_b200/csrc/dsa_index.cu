@@ -1345,9 +1345,7 @@ __global__ void k_vs_rowstats(const __grid_constant__ HeadTab ht, Layout L, uint
 // to every CTA.  Then each CTA counts its keys above the k-th and equal to it,
 // learns the counts of the CTAs before it (again through distributed shared
 // memory) and writes its selected keys at their ascending positions (ties go to
-// the lower index, as in the CTA-wide select).  The histogram increments are
-// aggregated per warp (one atomic per distinct bin): the first pass's 12 bits
-// are the sign, the exponent and 3 mantissa bits, so most keys share a few bins.
+// the lower index, as in the CTA-wide select).
 constexpr int VT_CL = 8;
 
 // CTAs per top-k cluster for arrays of n keys
@@ -1439,13 +1437,7 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
 #pragma unroll
       for (int q = 0; q < RB; ++q) {
         const int i = i0 + q * blockDim.x + tid;
-        const bool act = i < end && (key[q] & mask) == prefix;
-        const unsigned am = __ballot_sync(0xffffffffu, act);
-        if (act) {
-          const int bin = (int)((key[q] >> shift) & dmask);
-          const unsigned same = __match_any_sync(am, bin);
-          if ((same & ((1u << lane) - 1u)) == 0u) atomicAdd(&hist[bin], __popc(same));
-        }
+        if (i < end && (key[q] & mask) == prefix) atomicAdd(&hist[(key[q] >> shift) & dmask], 1);
       }
     }
     cluster.sync();  // every CTA's histogram is complete
@@ -1494,37 +1486,39 @@ __global__ void __launch_bounds__(1024) k_vs_topk(const __grid_constant__ HeadTa
   }
   const uint32_t T = prefix;
   const int take_eq = need;
-  // counts of this CTA's segment, shared with the cluster
-  int gt = 0, eq = 0;
-  for (int i = beg + tid; i < end; i += blockDim.x) {
-    const uint32_t key = fkey(arr[i]);
-    gt += key > T;
-    eq += key == T;
-  }
-  gt = warp_sum_int(gt);
-  eq = warp_sum_int(eq);
-  if (lane == 0) {
-    red[2 * warp] = gt;
-    red[2 * warp + 1] = eq;
-  }
-  __syncthreads();
-  if (tid == 0) {
-    int g = 0, e = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-      g += red[2 * w];
-      e += red[2 * w + 1];
-    }
-    xfer[2] = g;
-    xfer[3] = e;
-  }
-  cluster.sync();
+  // counts of the segments before this CTA's (none for a one-CTA cluster)
   int gt_before = 0, eq_before = 0;
-  for (int r = 0; r < rank; ++r) {
-    const int* rx = cluster.map_shared_rank(xfer, r);
-    gt_before += rx[2];
-    eq_before += rx[3];
+  if (ncl > 1) {
+    int gt = 0, eq = 0;
+    for (int i = beg + tid; i < end; i += blockDim.x) {
+      const uint32_t key = fkey(arr[i]);
+      gt += key > T;
+      eq += key == T;
+    }
+    gt = warp_sum_int(gt);
+    eq = warp_sum_int(eq);
+    if (lane == 0) {
+      red[2 * warp] = gt;
+      red[2 * warp + 1] = eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      int g = 0, e = 0;
+      for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+        g += red[2 * w];
+        e += red[2 * w + 1];
+      }
+      xfer[2] = g;
+      xfer[3] = e;
+    }
+    cluster.sync();
+    for (int r = 0; r < rank; ++r) {
+      const int* rx = cluster.map_shared_rank(xfer, r);
+      gt_before += rx[2];
+      eq_before += rx[3];
+    }
+    cluster.sync();  // no CTA leaves while another may still read its counts
   }
-  cluster.sync();  // no CTA leaves while another may still read its counts
   __syncthreads();
   auto load = [&](int i) { return arr[i]; };
   ordered_select_range(load, beg, end, T, take_eq, eq_before, gt_before + min(eq_before, take_eq), red,
@@ -1751,23 +1745,44 @@ __global__ void __launch_bounds__(1024) k_scan(int32_t* p0, int n0, int64_t cap0
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int seg = ceil_div(ceil_div(n, 32), 32) * 32;
   const int beg = min(n, warp * seg), end = min(n, beg + seg);
+  // eight loads in flight per lane in both passes (the segment is too long for
+  // shared memory at a million tokens)
+  constexpr int U = 8;
   int s = 0;
-  for (int i = beg + lane; i < end; i += 32) s += p[i];
+  for (int i0 = beg; i0 < end; i0 += 32 * U) {
+    int v[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * 32 + lane;
+      v[u] = (i < end) ? p[i] : 0;
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) s += v[u];
+  }
   s = warp_sum_int(s);
   if (lane == 0) wsum[warp] = s;
   __syncthreads();
   int carry = 0;
   for (int w = 0; w < warp; ++w) carry += wsum[w];
-  for (int i0 = beg; i0 < end; i0 += 32) {
-    const int i = i0 + lane;
-    int v = (i < end) ? p[i] : 0;
+  for (int i0 = beg; i0 < end; i0 += 32 * U) {
+    int v[U];
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += y;
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * 32 + lane;
+      v[u] = (i < end) ? p[i] : 0;
     }
-    if (i < end) p[i] = v + carry;
-    carry += __shfl_sync(0xffffffffu, v, 31);
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int i = i0 + u * 32 + lane;
+      int x = v[u];
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (i < end) p[i] = x + carry;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0 && n > 0 && (int64_t)p[n - 1] > cap) {
