@@ -374,7 +374,11 @@ __device__ __forceinline__ bool key_in_runs(const int32_t* iv, int n, int r1, in
   return lo > 0 && d <= iv[2 * (lo - 1) + 1];
 }
 
-template <int D, bool RUNS>
+// RUNS: slash-run tiles (some head is VS_WINDOWS).  COLS: gathered column tiles
+// (some head is VS or VS_WINDOWS); without them the decoders, the gatherers and
+// the softmax carry no column code, which keeps the kernel's instruction
+// footprint small for layers of block kinds only.
+template <int D, bool RUNS, bool COLS>
 __global__ void __launch_bounds__(NTHREADS, 2)
 sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ AttnArgs a) {
@@ -614,13 +618,13 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (dtid == 32) {
         // column lists: independent of the block lists, read in parallel with them
         int ce0 = 0, ce1 = 0, cb0 = 0, cb1 = 0;
-        if (live[0]) {
+        if (COLS && live[0]) {
           const int r = h * a.nqb + qbh[0];
           cb0 = a.col_ptr[r];
           ce0 = a.col_ptr[r + 1];
           checked_row(cb0, ce0, a.col_cap, a.status, DETAIL_BAD_COLPTR);
         }
-        if (live[1] && !shared_qb) {
+        if (COLS && live[1] && !shared_qb) {
           const int r = h * a.nqb + qbh[1];
           cb1 = a.col_ptr[r];
           ce1 = a.col_ptr[r + 1];
@@ -669,15 +673,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             report_bad_row(a.status, DETAIL_BAD_KIND);  // this build's kernel has no run tiles
           }
         } else if (kind == DSA_KIND_VS) {
-          int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
-          checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
-          for (int e = beg + dtid; e < end; e += 64) {
-            const int delta = a.dist[e];
-            if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
-            if (delta > qb) continue;
-            const int kb = qb - delta;
-            for (int u = kb * upb; u < kb * upb + upb; ++u)
-              if (u * UNIT <= r1) atomicOr(&bb[u >> 5], 1u << (u & 31));
+          if constexpr (COLS) {
+            int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
+            checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
+            for (int e = beg + dtid; e < end; e += 64) {
+              const int delta = a.dist[e];
+              if (delta < 0) { report(a.status, DSA_ERR_DEVICE, DETAIL_BAD_DIST); continue; }
+              if (delta > qb) continue;
+              const int kb = qb - delta;
+              for (int u = kb * upb; u < kb * upb + upb; ++u)
+                if (u * UNIT <= r1) atomicOr(&bb[u >> 5], 1u << (u & 31));
+            }
+          } else {
+            report_bad_row(a.status, DETAIL_BAD_KIND);  // this build's kernel has no column tiles
           }
         } else {
           const int r = h * a.nqb + qb;
@@ -759,7 +767,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       if (misc[9] == 0) { go = false; return; }
       int t = di.T_u;
       if constexpr (RUNS) t += di.rt[0] + di.rt[1];
-      for (int hh = 0; go && hh < 2; ++hh) {
+      for (int hh = 0; COLS && go && hh < 2; ++hh) {
         const int nt = ceil_div(di.cc[hh], BN);
         const int cflags = hh ? 2 : di.flags1;
         for (int ct = 0; ct < nt; ++ct, ++t) {
@@ -960,7 +968,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           const int lim = (si.flags & hbit) ? min(si.ncols, row - si.u + 1) : 0;
           mw[0] = low_bits(lim);
           mw[1] = low_bits(lim - 32);
-        } else if (si.type == 0) {
+        } else if (!COLS || si.type == 0) {
           const bool oks = (si.flags & hbit) != 0;
 #pragma unroll
           for (int k = 0; k < 2; ++k) {
@@ -1172,7 +1180,7 @@ bool make_map(CUtensorMap* map, const void* base, int d, int N, int H, int64_t t
   return r == CUDA_SUCCESS;
 }
 
-template <int D, bool RUNS>
+template <int D, bool RUNS, bool COLS>
 dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const void* V, const dsa_indices& idx,
                     void* O, float* lse, cudaStream_t stream, unsigned* status) {
   CUtensorMap mq, mk, mv;
@@ -1217,7 +1225,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   int smem = Smem<D>::bytes(a.nwords);
   // at most two CTAs per SM: each holds 256 of the 512 TMEM columns
   if (smem < 80 * 1024) smem = 80 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, RUNS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<D, RUNS, COLS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return cuda_fail(e);
   const int n_items = a.n_qtiles * p.Hq;
   if (n_items == 0) return DSA_OK;
@@ -1227,7 +1235,7 @@ dsa_status launch_d(const dsa_problem& p, const void* Q, const void* K, const vo
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return cuda_fail(e);
   const int grid = n_items < 2 * sms ? n_items : 2 * sms;
-  e = launch_pdl(sparse_attn_kernel<D, RUNS>, dim3(grid), dim3(NTHREADS), (size_t)smem, stream, mq, mk, mv, a);
+  e = launch_pdl(sparse_attn_kernel<D, RUNS, COLS>, dim3(grid), dim3(NTHREADS), (size_t)smem, stream, mq, mk, mv, a);
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e);
   return DSA_OK;
@@ -1242,15 +1250,19 @@ bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int N, int 
 
 dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K, const void* V,
                               const dsa_indices& idx, void* O, float* lse, cudaStream_t stream, unsigned* status) {
-  // the kernel with slash-run tiles only when a VS_WINDOWS head is present: the
-  // other kinds keep the smaller code of the plain one
+  // the kernel with slash-run tiles only when a VS_WINDOWS head is present, and
+  // with column tiles only when a VS kind is: the other kinds keep the smaller
+  // code of the plainer instantiations
   const bool runs = (idx.kinds_present >> DSA_KIND_VS_WINDOWS) & 1;
+  const bool cols = runs || ((idx.kinds_present >> DSA_KIND_VS) & 1);
   if (p.d == 128)
-    return runs ? launch_d<128, true>(p, Q, K, V, idx, O, lse, stream, status)
-                : launch_d<128, false>(p, Q, K, V, idx, O, lse, stream, status);
+    return runs ? launch_d<128, true, true>(p, Q, K, V, idx, O, lse, stream, status)
+                : (cols ? launch_d<128, false, true>(p, Q, K, V, idx, O, lse, stream, status)
+                        : launch_d<128, false, false>(p, Q, K, V, idx, O, lse, stream, status));
   if (p.d == 64)
-    return runs ? launch_d<64, true>(p, Q, K, V, idx, O, lse, stream, status)
-                : launch_d<64, false>(p, Q, K, V, idx, O, lse, stream, status);
+    return runs ? launch_d<64, true, true>(p, Q, K, V, idx, O, lse, stream, status)
+                : (cols ? launch_d<64, false, true>(p, Q, K, V, idx, O, lse, stream, status)
+                        : launch_d<64, false, false>(p, Q, K, V, idx, O, lse, stream, status));
   return DSA_ERR_UNSUPPORTED;
 }
 
