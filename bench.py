@@ -163,9 +163,10 @@ def build_workload(w, device, seed_offset=0):
 def key_tiles_per_item(bufs, N, B):
     """64-key tiles the attention kernel runs per 128-row item, from the index
     lists, the kernel's own tiling: per item the union of its two 64-row halves'
-    64-key units of listed blocks, plus each half's slash-run tiles (64 keys from
-    each run's first key) and gathered column tiles (a half that shares its query
-    block with the other adds none of its own); averaged over items."""
+    64-key units (of listed blocks, or touched by the slash runs of the half's
+    query block), each unit only up to the half's last row, plus the gathered
+    column tiles (a half that shares its query block with the other adds none of
+    its own); averaged over items."""
     nqb = (N + B - 1) // B
     tiles = items = 0
     for hl in bufs.host_lists():
@@ -178,19 +179,6 @@ def key_tiles_per_item(bufs, N, B):
                 if rs >= N:
                     continue
                 qb, r1h = rs // B, min(N - 1, rs + 63)
-                if hl["kind"] == 1:
-                    blocks = [qb - int(dd) for dd in hl["dist"] if dd <= qb]
-                elif hl["kind"] == 6:
-                    blocks = []
-                else:
-                    blocks = [int(x) for x in hl["blocks"][qb]]
-                for kb in blocks:
-                    for u in range(kb * B // 64, (kb * B + B) // 64):
-                        if u * 64 <= r1h:
-                            units.add(u)
-                if qb in seen:
-                    continue
-                seen.add(qb)
                 if hl["kind"] == 6:
                     lst = hl["dist"]
                     n, nl = int(lst[0]), int(lst[1])
@@ -200,7 +188,19 @@ def key_tiles_per_item(bufs, N, B):
                     for a, b in iv:
                         hi, lo = r1 - int(a), max(0, r1 - int(b))
                         if hi >= lo:
-                            t += (hi - lo) // 64 + 1
+                            units.update(range(lo // 64, min(hi, r1h) // 64 + 1))
+                else:
+                    if hl["kind"] == 1:
+                        blocks = [qb - int(dd) for dd in hl["dist"] if dd <= qb]
+                    else:
+                        blocks = [int(x) for x in hl["blocks"][qb]]
+                    for kb in blocks:
+                        for u in range(kb * B // 64, (kb * B + B) // 64):
+                            if u * 64 <= r1h:
+                                units.add(u)
+                if qb in seen:
+                    continue
+                seen.add(qb)
                 t += (len(hl["cols"][qb]) + 63) // 64
             tiles += t + len(units)
             items += 1

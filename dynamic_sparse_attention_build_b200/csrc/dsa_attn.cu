@@ -68,10 +68,11 @@ constexpr bool kLoaderSuspend = true;
 constexpr bool kMmaSuspend = true;
 
 struct StageInfo {
-  int type;   // 0 = key unit, 1 = column tile, 2 = slash-run tile
-  int u;      // unit id (type 0), first key (type 2)
+  int type;   // 0 = key unit, 1 = column tile, 3 = key unit of slash runs
+  int u;      // unit id (types 0 and 3)
   int flags;  // bit h: half h of the rows uses this tile
-  int ncols;  // valid columns (type 1), valid keys from the first (type 2)
+  int ncols;  // valid columns (type 1)
+  uint32_t m[4];  // type 3: the unit's keys inside half h's runs, bits m[2h] | m[2h + 1] << 32
 };
 
 struct ItemInfo {
@@ -88,9 +89,9 @@ struct DecInfo {
   int flags1;  // halves that use half 0's column tiles (3 when both halves share a query block)
   int cc[2], cb[2];  // column count / first column of each half
   // slash runs (VS_WINDOWS heads): per half, the interval list of its query
-  // block's height (an index into dist), its length, the block's last row, and
-  // the run tiles it gives (half 1 has none when both halves share the block)
-  int rbeg[2], rn[2], rr1[2], rt[2];
+  // block's height (an index into dist), its length and the block's last row
+  int wins;  // the item's head is VS_WINDOWS: its units carry run masks
+  int rbeg[2], rn[2], rr1[2];
 };
 
 struct AttnArgs {
@@ -350,16 +351,24 @@ static __device__ __noinline__ void drain_loads(uint64_t* bars, const int* misc,
   }
 }
 
-// The run tiles of one slash-run list (VS_WINDOWS): interval [a, b] of offsets
-// is the key run [max(0, r1 - b), r1 - a], cut into 64-key tiles from its first
-// key.  Threads tid0, tid0 + nt, ... share the intervals; returns their share.
-__device__ __forceinline__ int run_tiles(const int32_t* iv, int n, int r1, int tid0, int nt) {
-  int c = 0;
-  for (int k = tid0; k < n; k += nt) {
-    const int hi = r1 - iv[2 * k], lo = max(0, r1 - iv[2 * k + 1]);
-    if (hi >= lo) c += (hi - lo) / UNIT + 1;
+// Slash runs (VS_WINDOWS): offset interval [a, b] of a block whose last row is
+// r1 is the key run [max(0, r1 - b), r1 - a]; the intervals ascend, so the runs
+// descend in key order.  The bits of keys u0 .. u0 + 63 inside the runs; *c is
+// a cursor (start: n - 1) for units visited in ascending order.
+__device__ __forceinline__ uint64_t unit_run_mask(const int32_t* iv, int n, int r1, int u0, int* c) {
+  int k = *c;
+  while (k >= 0 && r1 - iv[2 * k] < u0) --k;  // runs wholly below this unit
+  *c = k;
+  uint64_t m = 0;
+  for (; k >= 0; --k) {
+    const int lo = max(0, r1 - iv[2 * k + 1]), hi = r1 - iv[2 * k];
+    if (lo > u0 + 63) break;
+    const int x = max(lo, u0) - u0, y = min(hi, u0 + 63) - u0;
+    if (y < x) continue;
+    const uint64_t top = (y == 63) ? ~0ull : ((1ull << (y + 1)) - 1ull);
+    m |= top & ~((1ull << x) - 1ull);
   }
-  return c;
+  return m;
 }
 
 // Key j lies in one of the runs of a list (offset intervals [a_k, b_k],
@@ -374,7 +383,7 @@ __device__ __forceinline__ bool key_in_runs(const int32_t* iv, int n, int r1, in
   return lo > 0 && d <= iv[2 * (lo - 1) + 1];
 }
 
-// RUNS: slash-run tiles (some head is VS_WINDOWS).  COLS: gathered column tiles
+// RUNS: units with slash-run masks (some head is VS_WINDOWS).  COLS: gathered column tiles
 // (some head is VS or VS_WINDOWS); without them the decoders, the gatherers and
 // the softmax carry no column code, which keeps the kernel's instruction
 // footprint small for layers of block kinds only.
@@ -470,6 +479,7 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         bool ok = true;
         int w = 0;
         uint32_t pend = b0[0] | b1[0];
+        int rc[2] = {di.rn[0] - 1, di.rn[1] - 1};  // run cursors (VS_WINDOWS items)
         for (int t = 0; t < di.T_u; ++t) {
           const int g = di.tg + t;
           const int b = g & 1;
@@ -490,6 +500,20 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           si.u = u;
           si.flags = (int)((b0[w] >> bit) & 1u) | ((int)((b1[w] >> bit) & 1u) << 1);
           si.ncols = 0;
+          if constexpr (RUNS) {
+            if (di.wins) {
+              // the unit's keys inside each half's runs (the softmax masks the rest)
+              si.type = 3;
+#pragma unroll
+              for (int hh = 0; hh < 2; ++hh) {
+                uint64_t m = 0;
+                if ((si.flags >> hh) & 1)
+                  m = unit_run_mask(a.dist + di.rbeg[hh], di.rn[hh], di.rr1[hh], u * UNIT, &rc[hh]);
+                si.m[2 * hh] = (uint32_t)m;
+                si.m[2 * hh + 1] = (uint32_t)(m >> 32);
+              }
+            }
+          }
           mbar_arrive(&bars[B_INFO + g % NINFO]);
           uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
           uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
@@ -503,49 +527,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
           mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
           pv[b] = g;
           for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, u * UNIT, di.kvh);
-        }
-        if constexpr (RUNS) {
-          // slash-run tiles (VS_WINDOWS): 64 keys from any first key, TMA boxes
-          // at that key row; half 0's runs (both halves' when they share the
-          // query block), then half 1's
-          int t = di.T_u;
-          for (int hh = 0; ok && hh < 2; ++hh) {
-            if (di.rt[hh] == 0) continue;
-            const int32_t* iv = a.dist + di.rbeg[hh];
-            const int fl = hh == 0 ? di.flags1 : 2;
-            for (int k = 0; ok && k < di.rn[hh]; ++k) {
-              const int hi = di.rr1[hh] - iv[2 * k], lo = max(0, di.rr1[hh] - iv[2 * k + 1]);
-              for (int st = lo; ok && st <= hi; st += UNIT, ++t) {
-                const int g = di.tg + t;
-                const int b = g & 1;
-                const uint32_t use = (g >> 1) & 1;
-                if (!mbar_wait_ool(&bars[B_KEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
-                                   kLoaderSuspend)) {
-                  ok = false;
-                  break;
-                }
-                StageInfo& si = info[g % NINFO];
-                si.type = 2;
-                si.u = st;
-                si.flags = fl;
-                si.ncols = min(UNIT, hi - st + 1);
-                mbar_arrive(&bars[B_INFO + g % NINFO]);
-                uint8_t* kst = sm + L::K_OFF + b * DS * KSLAB;
-                uint8_t* vst = sm + L::V_OFF + b * DS * KSLAB;
-                mbar_arrive_expect_tx(&bars[B_KFULL + b], DS * KSLAB);
-                pk[b] = g;
-                for (int c = 0; c < DS; ++c) tma_load_3d(kst + c * KSLAB, &tmK, &bars[B_KFULL + b], c * 64, st, di.kvh);
-                if (!mbar_wait_ool(&bars[B_VEMPTY + b], use ^ 1, limit, a.status, DETAIL_WAIT_EMPTY, abort_flag,
-                                   kLoaderSuspend)) {
-                  ok = false;
-                  break;
-                }
-                mbar_arrive_expect_tx(&bars[B_VFULL + b], DS * KSLAB);
-                pv[b] = g;
-                for (int c = 0; c < DS; ++c) tma_load_3d(vst + c * KSLAB, &tmV, &bars[B_VFULL + b], c * 64, st, di.kvh);
-              }
-            }
-          }
         }
         if (!ok) break;
         mbar_arrive(&bars[B_UNITS]);  // this item's bitmaps are no longer read here
@@ -576,10 +557,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         misc[10] = next_item;
         next_item = (int)gridDim.x + sched_next(a.sched, a.epoch);  // fetched one item ahead
         misc[3] = 0;
-        if constexpr (RUNS) {
-          misc[4] = 0;
-          misc[5] = 0;
-        }
       }
       named_barrier(1, 64);
       const int item = misc[10];
@@ -643,9 +620,9 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         const int r1 = r1h[hh];
         if (kind == DSA_KIND_VS_WINDOWS) {
           if constexpr (RUNS) {
-            // the slash runs of the half's query block (both halves share them
-            // when they share the block): count their 64-key tiles
-            if (hh == 1 && shared_qb) continue;
+            // the slash runs of the half's query block: every 64-key unit they
+            // touch (up to the half's last row) joins the half's unit bitmap; the
+            // producer attaches the run keys of each unit as a mask
             int beg = a.dist_ptr[h], end = a.dist_ptr[h + 1];
             checked_row(beg, end, a.dist_cap, a.status, DETAIL_BAD_DISTPTR);
             int n = 0, nl = 0;
@@ -661,16 +638,19 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
             const int r1b = min(a.N - 1, qb * a.B + a.B - 1);
             const int off = beg + 2 + (lastb ? 2 * n : 0);
             const int m = lastb ? nl : n;
-            int c = run_tiles(a.dist + off, m, r1b, dtid, 64);
-            c = warp_sum_int(c);
-            if (lane == 0 && c) atomicAdd(&misc[4 + hh], c);
+            for (int k = dtid; k < m; k += 64) {
+              const int hi = r1b - a.dist[off + 2 * k], lo = max(0, r1b - a.dist[off + 2 * k + 1]);
+              if (hi < lo) continue;
+              const int uhi = min(hi, r1) / UNIT;
+              for (int u = lo / UNIT; u <= uhi; ++u) atomicOr(&bb[u >> 5], 1u << (u & 31));
+            }
             if (dtid == 0) {
               dec[s].rbeg[hh] = off;
               dec[s].rn[hh] = m;
               dec[s].rr1[hh] = r1b;
             }
           } else {
-            report_bad_row(a.status, DETAIL_BAD_KIND);  // this build's kernel has no run tiles
+            report_bad_row(a.status, DETAIL_BAD_KIND);  // this build's kernel has no run masks
           }
         } else if (kind == DSA_KIND_VS) {
           if constexpr (COLS) {
@@ -716,18 +696,12 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         di.T_u = misc[3];  // one tile per unit
         di.flags1 = shared_qb ? 3 : 1;
         di.T = di.T_u + ceil_div(di.cc[0], BN) + ceil_div(di.cc[1], BN);
+        di.wins = 0;
         if constexpr (RUNS) {
           const bool wins = kind == DSA_KIND_VS_WINDOWS;
-          di.rt[0] = wins && live[0] ? misc[4] : 0;
-          di.rt[1] = wins && live[1] && !shared_qb ? misc[5] : 0;
+          di.wins = wins ? 1 : 0;
           if (!wins || !live[0]) di.rn[0] = 0;
           if (!wins || !live[1]) di.rn[1] = 0;
-          if (wins && shared_qb) {  // half 1 reads the block's runs through half 0's tiles
-            di.rbeg[1] = di.rbeg[0];
-            di.rn[1] = di.rn[0];
-            di.rr1[1] = di.rr1[0];
-          }
-          di.T += di.rt[0] + di.rt[1];
         }
         di.tg = tg_dec;
         // publish the item (its slot is free once both consumers read item kc - 2)
@@ -766,7 +740,6 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
       named_barrier(1, 64);
       if (misc[9] == 0) { go = false; return; }
       int t = di.T_u;
-      if constexpr (RUNS) t += di.rt[0] + di.rt[1];
       for (int hh = 0; COLS && go && hh < 2; ++hh) {
         const int nt = ceil_div(di.cc[hh], BN);
         const int cflags = hh ? 2 : di.flags1;
@@ -810,7 +783,10 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
                 int v = j;
                 if (j >= 0) {
                   const int u = j / UNIT;
-                  int cov = (int)((b0[u >> 5] >> (u & 31)) & 1u) | ((int)((b1[u >> 5] >> (u & 31)) & 1u) << 1);
+                  // (the units of a VS_WINDOWS item hold only its run keys: there the
+                  // runs alone decide)
+                  int cov = di.wins ? 0
+                                    : ((int)((b0[u >> 5] >> (u & 31)) & 1u) | ((int)((b1[u >> 5] >> (u & 31)) & 1u) << 1));
                   if constexpr (RUNS) {
                     // a column inside a slash run of the half counts once
                     if (di.rn[0] > 0 && key_in_runs(a.dist + di.rbeg[0], di.rn[0], di.rr1[0], j)) cov |= 1;
@@ -963,11 +939,11 @@ sparse_attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constan
         tmem_ld32(s_t + 32, s + 32);
         // allowed-key bits of this row, 32 columns per word
         uint32_t mw[2];
-        if (RUNS && si.type == 2) {
-          // keys si.u .. si.u + ncols - 1 of the half's runs, causal
-          const int lim = (si.flags & hbit) ? min(si.ncols, row - si.u + 1) : 0;
-          mw[0] = low_bits(lim);
-          mw[1] = low_bits(lim - 32);
+        if (RUNS && si.type == 3) {
+          // the unit's keys inside the half's runs, causal
+          const bool oks = (si.flags & hbit) != 0;
+#pragma unroll
+          for (int k = 0; k < 2; ++k) mw[k] = oks ? (si.m[2 * half + k] & low_bits(row - (si.u * UNIT + k * 32) + 1)) : 0u;
         } else if (!COLS || si.type == 0) {
           const bool oks = (si.flags & hbit) != 0;
 #pragma unroll
@@ -1250,7 +1226,7 @@ bool make_tma_map_bf16_3d(CUtensorMap* map, const void* base, int d, int N, int 
 
 dsa_status launch_sparse_attn(const dsa_problem& p, const void* Q, const void* K, const void* V,
                               const dsa_indices& idx, void* O, float* lse, cudaStream_t stream, unsigned* status) {
-  // the kernel with slash-run tiles only when a VS_WINDOWS head is present, and
+  // the kernel with slash-run masks only when a VS_WINDOWS head is present, and
   // with column tiles only when a VS kind is: the other kinds keep the smaller
   // code of the plainer instantiations
   const bool runs = (idx.kinds_present >> DSA_KIND_VS_WINDOWS) & 1;

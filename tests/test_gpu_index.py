@@ -153,9 +153,10 @@ def test_mixed_gqa_ragged(dsa):
 @pytest.mark.parametrize("B", [64, 128])
 def test_vs_windows(dsa, B):
     """Vertical-Slash heads whose slashes are covered by their exact key runs per
-    query block (tiles of 64 keys from any first key) next to every other kind in
-    one layer (the kernel with run tiles then serves them all), with few, many and
-    clustered slashes, a ragged length and GQA."""
+    query block (every aligned 64-key unit a run touches, with the run keys as a
+    per-half mask) next to every other kind in one layer (the kernel with run
+    masks then serves them all), with few, many and clustered slashes, a ragged
+    length and GQA."""
     N, d = 1400, 128
     Q, K, V = synth.random_qkv(8, 2, N, d, seed=51 + B)
     pats = [dict(kind="vs_windows", last_q=64, n_vert=40, n_slash=3),
