@@ -293,15 +293,43 @@ __device__ __forceinline__ float tanh_approx(float x) {
 // about 2^-11, far below what routing on pooled keys can see) instead of an
 // exponential and a division; the halving is folded into the weights and bias.
 // sw: the head's weights as [W][D] and its bias as [D], halved, in shared memory.
+// (a.x, a.y) * (b.x, b.y) + (c.x, c.y) and (a.x + b.x, a.y + b.y) as one packed
+// f32x2 instruction each (per-lane rounding as fmaf / an add: the same values)
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  uint64_t av, bv, cv, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(bv) : "f"(b.x), "f"(b.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(cv) : "f"(c.x), "f"(c.y));
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(av), "l"(bv), "l"(cv));
+  float2 o;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+  return o;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  uint64_t av, bv, r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(av) : "f"(a.x), "f"(a.y));
+  asm("mov.b64 %0, {%1, %2};" : "=l"(bv) : "f"(b.x), "f"(b.y));
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(av), "l"(bv));
+  float2 o;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(o.x), "=f"(o.y) : "l"(r));
+  return o;
+}
+// the two bf16 of a 32-bit word as floats (a bf16 is the high half of its float)
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
 template <int W, int D>
 __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts, int c0, int r0, int r1,
                                               const float* sw, float* acc) {
-  float wt[W][8], bias[8], win[W][8];
+  // channels in pairs (c0 + 2j, c0 + 2j + 1), j < 4: packed f32x2 arithmetic
+  float2 wt[W][4], bias[4], win[W][4], acc2[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    bias[i] = sw[W * D + c0 + i];
+  for (int j = 0; j < 4; ++j) {
+    bias[j] = make_float2(sw[W * D + c0 + 2 * j], sw[W * D + c0 + 2 * j + 1]);
+    acc2[j] = make_float2(0.f, 0.f);
 #pragma unroll
-    for (int t = 0; t < W; ++t) wt[t][i] = sw[t * D + c0 + i];
+    for (int t = 0; t < W; ++t) wt[t][j] = make_float2(sw[t * D + c0 + 2 * j], sw[t * D + c0 + 2 * j + 1]);
   }
   // before row r is shifted in, win[t] = k[r - 1 - t] (t < W - 1); after the
   // shift win[t] = k[r - t].  Rows before 0 are zero (causal, zero padded).
@@ -310,9 +338,9 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
     const int rr = r0 - 1 - t;
     uint4 raw = make_uint4(0, 0, 0, 0);
     if (rr >= 0 && r0 < r1) raw = __ldg(reinterpret_cast<const uint4*>(X + (int64_t)rr * ts + c0));
-    const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw);
+    const uint32_t* wv = reinterpret_cast<const uint32_t*>(&raw);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) win[t][i] = __bfloat162float(e[i]);
+    for (int j = 0; j < 4; ++j) win[t][j] = bf16x2_to_float2(wv[j]);
   }
   // software pipelined: the next four rows are in flight while these four are
   // computed
@@ -333,23 +361,31 @@ __device__ __forceinline__ void conv_rows_sum(const __nv_bfloat16* X, int64_t ts
     // between the four rows, so their chains overlap
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const float keep = (r + u < r1) ? 1.f : 0.f;
+      const float kf = (r + u < r1) ? 1.f : 0.f;
+      const float2 keep = make_float2(kf, kf);
 #pragma unroll
       for (int t = W - 1; t > 0; --t) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) win[t][i] = win[t - 1][i];
+        for (int j = 0; j < 4; ++j) win[t][j] = win[t - 1][j];
       }
-      const __nv_bfloat16* e = reinterpret_cast<const __nv_bfloat16*>(&raw[u]);
+      const uint32_t* wv = reinterpret_cast<const uint32_t*>(&raw[u]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) win[0][i] = __bfloat162float(e[i]);
+      for (int j = 0; j < 4; ++j) win[0][j] = bf16x2_to_float2(wv[j]);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float h = bias[i];
+      for (int j = 0; j < 4; ++j) {
+        float2 h = bias[j];
 #pragma unroll
-        for (int t = 0; t < W; ++t) h = fmaf(wt[t][i], win[t][i], h);
-        acc[i] = fmaf(keep, win[0][i] + fmaf(h, tanh_approx(h), h), acc[i]);
+        for (int t = 0; t < W; ++t) h = ffma2(wt[t][j], win[t][j], h);
+        const float2 th = make_float2(tanh_approx(h.x), tanh_approx(h.y));
+        // k + SiLU(conv) = k + (h + h tanh h)
+        acc2[j] = ffma2(keep, fadd2(win[0][j], ffma2(h, th, h)), acc2[j]);
       }
     }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    acc[2 * j] = acc2[j].x;
+    acc[2 * j + 1] = acc2[j].y;
   }
 }
 
