@@ -152,8 +152,10 @@ typedef struct dsa_pattern {
  *   (last row r1) keeps the key runs [max(0, r1 - b), r1 - a].  Their columns lie
  *   outside those runs.
  * kinds_present: bit k set when some head has kind k.  dsa_sparse_prefill reads it
- *   to choose its kernel (a VS_WINDOWS head met without bit 6 is reported as
- *   DSA_ERR_DEVICE and left empty); dsa_build_indices does not read it.
+ *   to choose its kernel (column tiles only when bit 1 or bit 6 is set, slash-run
+ *   masks only when bit 6 is: a VS head met without bit 1, or a VS_WINDOWS head
+ *   without bit 6, is reported as DSA_ERR_DEVICE and left empty);
+ *   dsa_build_indices does not read it.
  * dsa_sparse_prefill reads only head_info, blk_*, dist*, col_*, kinds_present.
  */
 typedef struct dsa_indices {
