@@ -167,3 +167,29 @@ def test_abort_with_loads_in_flight_leaves_the_next_launch_exact(dsa):
     assert dsa.device_status() == (0, 0)
     assert torch.equal(O, O_ref) and torch.equal(lse, lse_ref)
     assert B.dsa_set_wait_limit(61 * 10**9) == B.DSA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("kind", ["vs", "vs_windows"])
+def test_kind_missing_from_kinds_present_is_reported(dsa, kind):
+    """dsa_sparse_prefill picks its kernel from kinds_present (column tiles only
+    with a VS kind, slash-run masks only with VS_WINDOWS).  Lists whose
+    kinds_present omits a kind that a head has: that head is reported
+    (DSA_ERR_DEVICE, detail 36) and left empty (O = 0, LSE = -inf), the other
+    heads equal the run with the right bits."""
+    from dynamic_sparse_attention_build_b200 import _binding as B
+    N, d, Bk = 700, 64, 64
+    Q, K, V = synth.random_qkv(2, 1, N, d, seed=9)
+    Qd, Kd, Vd = Q.cuda(), K.cuda(), V.cuda()
+    pats = [dict(kind="block_topk", topk=3), dict(kind=kind, last_q=16, n_vert=20, n_slash=6)]
+    good = dsa.build_indices(Qd, Kd, pats, Bk)
+    O_good, lse_good = dsa.sparse_prefill(Qd, Kd, Vd, good, want_lse=True)
+    assert dsa.device_status() == (0, 0)
+    bad = _clone_bufs(dsa, good)
+    bad.kinds_present = 1 << B.DSA_KIND_BLOCK_TOPK
+    bad.__post_init__()
+    O_bad, lse_bad = dsa.sparse_prefill(Qd, Kd, Vd, bad, want_lse=True)
+    status, det = dsa.device_status()
+    assert status == B.DSA_ERR_DEVICE and det == 36, (status, det)
+    assert torch.equal(O_bad[0], O_good[0]) and torch.equal(lse_bad[0], lse_good[0])
+    assert not O_bad[1].any() and torch.isinf(lse_bad[1]).all()
+    assert dsa.device_status() == (0, 0)
