@@ -17,6 +17,12 @@
 //     halves that listed it (the other half masks it out);
 //   * column lists are gathered into dense 64-key tiles (gather-and-densify); a
 //     column inside a block the half already keeps is masked out;
+//   * slash runs of VS_WINDOWS heads (exact key runs per query block) join the
+//     unit bitmaps: every unit a run touches, carrying each half's run keys as
+//     a 64-bit mask;
+//   * three instantiations, chosen from the index's kinds_present: block kinds
+//     only (no column code), with column tiles, with column tiles and run masks
+//     (the smaller code keeps short items out of instruction-cache misses);
 //   * warps 2-3 (decoders) fetch items, turn an item's lists into bitmap set
 //     (item & 1) up to one item ahead, publish it, and gather its column rows;
 //     warp 0 (one thread) loads each item's Q and issues the TMA loads
@@ -30,7 +36,8 @@
 //   * TMEM (256 columns per CTA): O at [0, 128), two S buffers of 64 columns at
 //     128 and 192.  S(t+1) = Q K(t+1)^T is computed while the softmax works on
 //     S(t); the softmax writes P(t) as bf16 pairs over the first 32 columns of its
-//     S buffer and O += P(t) V(t) reads it from there;
+//     S buffer and O += P(t) V(t) reads it from there; S(t+2) is issued right
+//     after that P.V (one thread's MMAs run in order);
 //   * the running max is only raised when it grows by more than 2^32; only then
 //     does the softmax wait for the previous P.V and rescale O, so in the common
 //     case the softmax of one tile overlaps the P.V of the one before;
